@@ -1,0 +1,74 @@
+"""The oracle against its pins, and planted mistakes against the pins.
+
+The second half copies ``oracle/hq_oracle.c`` to a temporary directory, plants one plausible
+mistake (a swapped decay, a dropped rank, a reversed nibble order, a wrong tie-break, ...),
+builds it, and checks that at least one pin fails.  Nothing of this touches a GPU.
+"""
+import os
+import shutil
+
+import pytest
+
+import oracle
+import pins
+
+ORACLE_SRC = os.path.join(os.path.dirname(oracle.__file__), "hq_oracle.c")
+
+
+@pytest.mark.parametrize("pin", pins.ALL_PINS, ids=lambda f: f.__name__)
+def test_oracle_pin(pin):
+    pin(oracle.get())
+
+
+# (name, text in hq_oracle.c, replacement)
+MUTANTS = [
+    ("ema_decay_swapped", "float a = beta * ema_min[i];", "float a = one_minus_beta * ema_min[i];"),
+    ("first_batch_ignored", "if (first_batch) {", "if (0) {"),
+    ("calib_drops_last_row", "for (int t = 0; t < T; ++t) {\n        float v", "for (int t = 0; t < T - 1; ++t) {\n        float v"),
+    ("zero_not_in_range", "float lo = (ema_min[i] < 0.0f) ? ema_min[i] : 0.0f;", "float lo = ema_min[i];"),
+    ("scale_over_16", "float s = rg / 15.0f;", "float s = rg / 16.0f;"),
+    ("zero_point_floor", "float zf = rintf((-lo) * inv);", "float zf = floorf((-lo) * inv);"),
+    ("score_max_not_sum", "acc = acc + range[(size_t)r * H + h];",
+     "acc = (range[(size_t)r * H + h] > acc) ? range[(size_t)r * H + h] : acc;"),
+    ("ties_to_higher_col", "return (a->col < b->col) ? -1 : (a->col > b->col) ? 1 : 0;",
+     "return (a->col < b->col) ? 1 : (a->col > b->col) ? -1 : 0;"),
+    ("keep_not_sorted", "qsort(keep_idx, (size_t)k, sizeof(int32_t), ref_ascending);", ""),
+    ("rint_after_zero", "float n = rintf(a);", "float n = rintf(a + (float)zero) - (float)zero;"),
+    ("nan_to_code_0", "if (isnan(a)) return zero;", "if (isnan(a)) return 0u;"),
+    ("nibbles_reversed", "crow[c / 8] |= (uint32_t)q << (4 * (c % 8));", "crow[c / 8] |= (uint32_t)q << (4 * (7 - c % 8));"),
+    ("side_from_rest", "srow[j] = row[keep_idx[j]];", "srow[j] = row[rest_idx[j]];"),
+    ("reduce_drops_last_rank", "for (int r = 0; r < P; ++r) {\n        uint32_t word",
+     "for (int r = 0; r < P - 1; ++r) {\n        uint32_t word"),
+    ("dequant_sign_flipped", "(float)(q - (int)zero[p])", "(float)((int)zero[p] - q)"),
+    ("kept_sum_rank0_only", "for (int r = 0; r < P; ++r) acc = acc + ref_bf16_value(side",
+     "for (int r = 0; r < 1; ++r) acc = acc + ref_bf16_value(side"),
+    ("bf16_truncates", "if (dropped > 0x8000u || (dropped == 0x8000u && (keep & 1u))) keep += 1u;", ""),
+    ("dequant_mul_then_add", "acc = fmaf((float)(q - (int)zero[p]), scale[p], acc);",
+     "acc = acc + (float)(q - (int)zero[p]) * scale[p] * 1.0009765625f;"),
+]
+
+
+@pytest.fixture(scope="module")
+def mutant_dir(tmp_path_factory):
+    d = tmp_path_factory.mktemp("oracle_mutants")
+    yield d
+    shutil.rmtree(d, ignore_errors=True)
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_planted_mistake(mutant_dir, name, old, new):
+    src = open(ORACLE_SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    path = mutant_dir / f"{name}.c"
+    path.write_text(src.replace(old, new))
+    so = str(mutant_dir / f"lib_{name}.so")
+    import subprocess
+
+    subprocess.run(["gcc", *oracle.CFLAGS, str(path), "-o", so, "-lm"], check=True)
+    mutant = oracle.Oracle(so)
+    for pin in pins.ALL_PINS:
+        try:
+            pin(mutant)
+        except (AssertionError, ValueError):
+            return
+    pytest.fail(f"no pin caught the planted mistake {name}")
