@@ -29,7 +29,8 @@
  *   R9  dequant-reduce of a non-kept column: acc = +0; for r = 0..P-1:
  *       acc = fma(float(q_r - zero_r), scale_r, acc)  (one rounding per rank).
  *   R10 kept column: acc = +0; for r = 0..P-1: acc = acc + float(side_r).
- *   R11 output: fp32, or bf16 by round-to-nearest-even with NaN -> 0x7FC0.
+ *   R11 output: fp32, or bf16 by round-to-nearest-even; a NaN result is written as the
+ *       canonical quiet NaN in both types (0x7FC00000 / 0x7FC0).
  *   R12 the fused compress-reduce equals quantize-pack followed by dequant-reduce.
  *   R14 parameters are computed for every column, kept ones included (unused there).
  * Calibration detail: batch min/max ignore NaN (no comparison with NaN is true); a batch
@@ -51,6 +52,15 @@ static float ref_bf16_value(uint16_t b) {
   float f;
   memcpy(&f, &u, sizeof f);
   return f;
+}
+
+/* A NaN result as the canonical quiet NaN 0x7FC00000 (R11); other values unchanged. */
+static float ref_canonical(float f) {
+  if (!isnan(f)) return f;
+  const uint32_t q = 0x7FC00000u;
+  float c;
+  memcpy(&c, &q, sizeof c);
+  return c;
 }
 
 /* float -> bf16 bits, round to nearest, ties to even; NaN -> 0x7FC0 (R11). */
@@ -248,7 +258,7 @@ void hq_ref_dequant_reduce(const uint32_t* codes, const uint16_t* side, int P, i
       float acc = 0.0f;
       for (int r = 0; r < P; ++r) acc = acc + ref_bf16_value(side[((size_t)r * T + t) * k + j]);
       size_t o = (size_t)t * H + keep_idx[j];
-      if (out_f32) ((float*)out)[o] = acc;
+      if (out_f32) ((float*)out)[o] = ref_canonical(acc);
       else ((uint16_t*)out)[o] = ref_bf16_round(acc);
     }
     for (int c = 0; c < Hr; ++c) {
@@ -261,7 +271,7 @@ void hq_ref_dequant_reduce(const uint32_t* codes, const uint16_t* side, int P, i
         acc = fmaf((float)(q - (int)zero[p]), scale[p], acc);
       }
       size_t o = (size_t)t * H + h;
-      if (out_f32) ((float*)out)[o] = acc;
+      if (out_f32) ((float*)out)[o] = ref_canonical(acc);
       else ((uint16_t*)out)[o] = ref_bf16_round(acc);
     }
   }

@@ -293,6 +293,30 @@ def pin_reduce_all_kept(o):
     assert np.array_equal(outb, f32_to_bf16_torch(want)), "bf16 output = RNE of the fp32 sum"
 
 
+def pin_nan_outputs(o):
+    """Reading R11: a NaN sum is written as the canonical quiet NaN in both output types; a NaN
+    in a 4-bit feature quantizes to the zero point and so adds exactly 0 (reading R6)."""
+    P, T, H, k = 2, 1, 16, 8
+    emin = np.full((P, H), -2.0, np.float32)
+    emax = np.full((P, H), 2.0, np.float32)
+    emax[:, :k] = 100.0                     # features 0..7 are kept
+    sel = o.select_topk(emin, emax, k)
+    assert sel["keep_idx"].tolist() == list(range(k))
+    vals = np.zeros((P, T, H), np.float32)
+    vals[0, 0, 0] = np.nan                  # kept: NaN + 0
+    vals[0, 0, 1], vals[1, 0, 1] = np.inf, -np.inf   # kept: inf + -inf
+    vals[0, 0, 2] = -np.nan                 # kept: negative NaN payload
+    vals[0, 0, 8], vals[1, 0, 8] = np.nan, 1.0       # 4-bit: NaN -> zero point, adds 0
+    x = f32_to_bf16_torch(vals.ravel()).reshape(P, T, H)
+    x[0, 0, 2] = 0xFFC1
+    of = o.compress_reduce(x, sel["keep_idx"], sel["rest_idx"], sel["scale"], sel["inv_scale"], sel["zero"], out_f32=True)
+    ob = o.compress_reduce(x, sel["keep_idx"], sel["rest_idx"], sel["scale"], sel["inv_scale"], sel["zero"])
+    bits = of.view(np.uint32)
+    assert bits[0, 0] == bits[0, 1] == bits[0, 2] == 0x7FC00000, [hex(b) for b in bits[0, :3]]
+    assert ob[0, 0] == ob[0, 1] == ob[0, 2] == 0x7FC0
+    assert np.isfinite(of[0, 8]) and abs(float(of[0, 8]) - 1.0) <= float(sel["scale"][1, 8]) / 2 * 1.0001
+
+
 def pin_reduce_dequant_sum(o):
     """Each reduced element is sum_r (q_r - zero_r) * scale_r of its own codes, within the
     rounding of P fp32 steps; kept ones are the sum of the side values."""
@@ -427,6 +451,6 @@ ALL_PINS = [
     pin_bf16_round, pin_quantize_golden, pin_quantize_nearest_grid, pin_params_golden,
     pin_params_closed_form, pin_calibrate_single_batch, pin_calibrate_ema, pin_select_golden,
     pin_select_brute_force, pin_pack_golden, pin_pack_unpack, pin_reduce_all_kept,
-    pin_reduce_dequant_sum, pin_reduce_error_bound, pin_irwin_hall, pin_outliers_selected,
+    pin_nan_outputs, pin_reduce_dequant_sum, pin_reduce_error_bound, pin_irwin_hall, pin_outliers_selected,
     pin_selection_benefit,
 ]

@@ -42,6 +42,7 @@ MUTANTS = [
     ("dequant_sign_flipped", "(float)(q - (int)zero[p])", "(float)((int)zero[p] - q)"),
     ("kept_sum_rank0_only", "for (int r = 0; r < P; ++r) acc = acc + ref_bf16_value(side",
      "for (int r = 0; r < 1; ++r) acc = acc + ref_bf16_value(side"),
+    ("fp32_nan_payload_kept", "if (!isnan(f)) return f;", "return f;"),
     ("bf16_truncates", "if (dropped > 0x8000u || (dropped == 0x8000u && (keep & 1u))) keep += 1u;", ""),
     ("dequant_mul_then_add", "acc = fmaf((float)(q - (int)zero[p]), scale[p], acc);",
      "acc = acc + (float)(q - (int)zero[p]) * scale[p] * 1.0009765625f;"),
