@@ -1,0 +1,501 @@
+#!/usr/bin/env python
+"""Throughput of the hybrid BF16/Int4 partial-sum compression path on B200.
+
+One step is one pass of the whole path over one batch of P ranks' bf16 partial sums, resident in
+HBM: hq_calibrate (one more moving-average update), hq_select_topk, hq_quantize_pack and
+hq_dequant_reduce (``--path split``, the default) or hq_compress_reduce (``--path fused``).
+``value`` is partial-sum bytes (P*T*H*2 per step, all ranks) per second over the timed steps.
+
+Prints one JSON line.  ``--impl reference`` times the CPU oracle instead (the reference arm of
+this benchmark: a plain single-threaded C restatement of the method).  Under torchrun each rank
+runs an independent replica on its own GPU (the method has no data-path collective on one node
+here); the timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "partial-sum GB/s compressed+reduced (1 B200), % of HBM peak; compression ratio"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["hq", "reference"], default="hq")
+    ap.add_argument("--path", choices=["split", "fused"], default="split")
+    ap.add_argument("--workload", default="prefill70b")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args()
+
+
+def workload(name: str) -> synth.Config:
+    if name in synth.CONFIGS:
+        return synth.CONFIGS[name]
+    for c in synth.sweep_configs():
+        if c.name == name:
+            return c
+    raise SystemExit(f"unknown workload {name}")
+
+
+def describe(cfg: synth.Config) -> str:
+    dist = {"normal": "N(0, std_h)", "student_t3": "Student-t(3) x std_h", "uniform": "U(-1,1)"}[cfg.dist]
+    s = f"{cfg.name}: P={cfg.P} ranks, bf16 partial sums [T={cfg.T}, H={cfg.H}], k={cfg.k} kept, {dist}"
+    if cfg.dist != "uniform":
+        s += f", std_h ~ LogNormal(0,{cfg.sigma}), {cfg.n_out} outlier cols x{cfg.out_mult:g}"
+    if cfg.spike_p:
+        s += f", spikes p={cfg.spike_p} x{cfg.spike_mult:g}"
+    return s + f"; {cfg.calib_batches} calib batches of {cfg.calib_T} rows, EMA {cfg.beta}"
+
+
+def algo_bytes(cfg: synth.Config) -> dict:
+    """Bytes each call must move (reads + writes), parameters included."""
+    P, T, H, k = cfg.P, cfg.T, cfg.H, cfg.k
+    Hr = H - k
+    params = P * H * (4 + 4 + 1)
+    return {
+        "calibrate": P * T * H * 2 + 4 * P * H * 4,
+        "select": 2 * P * H * 4 + params + H * 4,
+        "quantize_pack": P * T * H * 2 + P * T * Hr // 2 + P * T * k * 2 + P * H * 5 + H * 4,
+        "dequant_reduce": P * T * Hr // 2 + P * T * k * 2 + T * H * 2 + P * H * 5 + H * 4,
+        "compress_reduce": P * T * H * 2 + T * H * 2 + params + H * 4,
+    }
+
+
+def compression_ratio(cfg):
+    return (16.0 * cfg.H) / (4.0 * (cfg.H - cfg.k) + 16.0 * cfg.k)
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs: copy bandwidth)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (no MEASURED_PEAKS.json)"
+
+
+# ---------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------------------------
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    def __init__(self, gpu_index: int, enabled: bool):
+        self.proc = None
+        self.gpu = gpu_index
+        if enabled:
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--query-gpu={CLOCK_FIELDS}", "--format=csv,noheader,nounits",
+                     "-lms", "100", "-i", str(gpu_index)],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except OSError:
+                self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [p.strip() for p in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+# ---------------------------------------------------------------------------------------------
+# distributed plumbing (replicas; the max-over-ranks timing is the only collective)
+# ---------------------------------------------------------------------------------------------
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        backend = "nccl" if args.impl == "hq" else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline leg and the reference arm)
+# ---------------------------------------------------------------------------------------------
+class OracleStep:
+    """The whole path on the CPU oracle over rows [0, S) of the workload's evaluation batch."""
+
+    def __init__(self, cfg, x_rows: np.ndarray):
+        import oracle
+
+        self.o = oracle.get()
+        self.cfg = cfg
+        self.x = x_rows
+        self.emin, self.emax = self.o.calibrate(x_rows, cfg.beta, True)
+
+    def run(self, S: int) -> float:
+        cfg, o = self.cfg, self.o
+        xs = np.ascontiguousarray(self.x[:, :S])
+        t0 = time.perf_counter()
+        emin, emax = o.calibrate(xs, cfg.beta, False, self.emin, self.emax)
+        sel = o.select_topk(emin, emax, cfg.k)
+        codes, side = o.quantize_pack(xs, sel["keep_idx"], sel["rest_idx"], sel["inv_scale"], sel["zero"])
+        o.dequant_reduce(codes, side, cfg.H, sel["keep_idx"], sel["rest_idx"], sel["scale"], sel["zero"])
+        return time.perf_counter() - t0
+
+
+def host_rows(cfg, S, device=None):
+    """Rows [0, S) of the evaluation batch for all ranks (from the GPU generator when a GPU is
+    present -- the same values as the host generator -- else from the host generator)."""
+    cs, _ = synth.colscale(cfg)
+    if device is not None:
+        import torch
+
+        buf = torch.empty((cfg.P, cfg.T, cfg.H), dtype=torch.int16, device=device)
+        synth.fill_gpu(cfg, synth.EVAL, 0, buf, torch.from_numpy(cs).to(device))
+        out = buf[:, :S].cpu().numpy().view(np.uint16).copy()
+        del buf
+        return out
+    return synth.fill_cpu(cfg, synth.EVAL, 0, rows=(0, S), cs=cs)
+
+
+def cpu_rows_for(step: OracleStep, seconds: float, cap: int) -> tuple[int, float]:
+    """Rows per oracle step so that one step takes about `seconds`."""
+    probe = min(cap, 8)
+    dt = step.run(probe)
+    per_row = max(dt / probe, 1e-7)
+    return max(1, min(cap, int(seconds / per_row))), per_row
+
+
+def run_reference(args, cfg, world, rank):
+    if rank != 0:
+        return
+    budget = 150.0  # seconds for the whole --steps/--warmup run
+    cap = min(cfg.T, 4096)
+    x = host_rows(cfg, cap)
+    step = OracleStep(cfg, x)
+    S, per_row = cpu_rows_for(step, budget / max(1, args.steps + args.warmup), cap)
+    for _ in range(args.warmup):
+        step.run(S)
+    t = sum(step.run(S) for _ in range(args.steps))
+    part_bytes = cfg.P * S * cfg.H * 2
+    value = part_bytes * args.steps / t / 1e9
+    sample = (f"rows 0..{S - 1} of the evaluation batch, all {cfg.P} ranks, per step "
+              f"(calibrate + select + quantize-pack + dequant-reduce), single thread")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": 0,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": describe(cfg), "P": cfg.P, "T": cfg.T, "H": cfg.H, "k": cfg.k,
+                   "path": "split", "parallelism": "replicas"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "compression_ratio": compression_ratio(cfg),
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------------------------
+# the CUDA path
+# ---------------------------------------------------------------------------------------------
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "bit_tensor_activation_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM traffic per launch recorded by an ncu capture of the same kernel source, else None."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d.get(f"{kernel}@{workload}")
+        if e and e.get("source_hash") == kernel_source_hash():
+            return e["bytes_per_launch"]
+    except Exception:
+        pass
+    return None
+
+
+def run_hq(args, cfg, world, rank, local):
+    import torch
+
+    import bit_tensor_activation_b200 as hq
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    P, T, H, k = cfg.P, cfg.T, cfg.H, cfg.k
+
+    # ---- inputs resident in HBM: calibration state, then the evaluation batch ----------------
+    cs, _ = synth.colscale(cfg)
+    cs_dev = torch.from_numpy(cs).to(dev)
+    B = hq.Buffers(P, T, H, k, device=dev)
+    cal = torch.empty((P, cfg.calib_T, H), dtype=torch.int16, device=dev)
+    for b in range(cfg.calib_batches):
+        synth.fill_gpu(cfg, synth.CALIB, b, cal, cs_dev, T=cfg.calib_T)
+        hq.hq_calibrate(cal, B.ema_min, B.ema_max, cfg.beta, b == 0)
+    del cal
+    x = torch.empty((P, T, H), dtype=torch.int16, device=dev)
+    synth.fill_gpu(cfg, synth.EVAL, 0, x, cs_dev)
+    fused_out = torch.empty_like(B.out)
+    torch.cuda.synchronize()
+
+    names = (["calibrate", "select", "quantize_pack", "dequant_reduce"] if args.path == "split"
+             else ["calibrate", "select", "compress_reduce"])
+
+    def step_calls(xin):
+        yield lambda: hq.hq_calibrate(xin, B.ema_min, B.ema_max, cfg.beta, False)
+        yield lambda: hq.hq_select_topk(B.ema_min, B.ema_max, k, B.keep_idx, B.rest_idx, B.scale,
+                                        B.inv_scale, B.zero)
+        if args.path == "split":
+            yield lambda: hq.hq_quantize_pack(xin, B.keep_idx, B.rest_idx, B.inv_scale, B.zero, B.codes, B.side)
+            yield lambda: hq.hq_dequant_reduce(B.codes, B.side, B.keep_idx, B.rest_idx, B.scale, B.zero, B.out)
+        else:
+            yield lambda: hq.hq_compress_reduce(xin, B.keep_idx, B.rest_idx, B.scale, B.inv_scale, B.zero,
+                                                fused_out)
+
+    def run_steps(n, xin, events=None):
+        for i in range(n):
+            for j, call in enumerate(step_calls(xin)):
+                if events is not None:
+                    events[i][j].record(stream)
+                call()
+        if events is not None:
+            events[n][0].record(stream)
+
+    run_steps(args.warmup, x)
+    torch.cuda.synchronize()
+    st = hq.hq_read_device_error()
+    if st != hq.HQ_OK:
+        raise RuntimeError(f"device error after warm-up: {hq.hq_status_string(st)}")
+
+    K = args.steps
+    nk = len(names)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(nk)] for _ in range(K)]
+    events.append([torch.cuda.Event(enable_timing=True)])
+    t_begin = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local, not args.no_clocks)
+    time.sleep(0.3 if not args.no_clocks else 0.0)
+    wall0 = time.perf_counter()
+    t_begin.record(stream)
+    run_steps(K, x, events)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    clk = clocks.stop()
+    barrier(world)
+
+    ms_local = t_begin.elapsed_time(t_end)
+    ms = max_over_ranks(ms_local, world, dev)
+    per_kernel = {}
+    for j, n in enumerate(names):
+        tot = 0.0
+        for i in range(K):
+            nxt = events[i][j + 1] if j + 1 < nk else events[i + 1][0]
+            tot += events[i][j].elapsed_time(nxt)
+        per_kernel[n] = tot / K  # ms per launch (includes the launch gap on the stream)
+
+    # ---- alternate path, measured the same way for the record ---------------------------------
+    alt = {}
+    alt_path = "fused" if args.path == "split" else "split"
+    saved = args.path
+    args.path = alt_path
+    alt_names = (["calibrate", "select", "quantize_pack", "dequant_reduce"] if alt_path == "split"
+                 else ["calibrate", "select", "compress_reduce"])
+    Ka = max(3, min(K, 200))
+    run_steps(3, x)
+    a0 = torch.cuda.Event(enable_timing=True)
+    a1 = torch.cuda.Event(enable_timing=True)
+    aev = [[torch.cuda.Event(enable_timing=True) for _ in alt_names] for _ in range(Ka)]
+    aev.append([torch.cuda.Event(enable_timing=True)])
+    torch.cuda.synchronize()
+    a0.record(stream)
+    run_steps(Ka, x, aev)
+    a1.record(stream)
+    torch.cuda.synchronize()
+    args.path = saved
+    alt_kernels = {}
+    for j, n in enumerate(alt_names):
+        tot = sum(aev[i][j].elapsed_time(aev[i][j + 1] if j + 1 < len(alt_names) else aev[i + 1][0])
+                  for i in range(Ka))
+        alt_kernels[n] = tot / Ka
+    alt_ms = a0.elapsed_time(a1) / Ka
+    alt[alt_path] = {"ms_per_step": alt_ms, "value": P * T * H * 2 / (alt_ms * 1e-3) / 1e9,
+                     "kernel_ms": alt_kernels}
+
+    # ---- fused output equals split output on this workload ---------------------------------------
+    hq.hq_quantize_pack(x, B.keep_idx, B.rest_idx, B.inv_scale, B.zero, B.codes, B.side)
+    hq.hq_dequant_reduce(B.codes, B.side, B.keep_idx, B.rest_idx, B.scale, B.zero, B.out)
+    hq.hq_compress_reduce(x, B.keep_idx, B.rest_idx, B.scale, B.inv_scale, B.zero, fused_out)
+    fused_equal = bool(torch.equal(B.out.view(torch.int16), fused_out.view(torch.int16)))
+
+    # ---- e2e: public API with pinned host buffers, copies inside the timed region ----------------
+    e2e = None
+    if args.e2e_steps > 0:
+        xh = x.cpu().pin_memory()
+        oh = torch.empty(B.out.shape, dtype=B.out.dtype).pin_memory()
+        xd = torch.empty_like(x)
+        for _ in range(2):
+            xd.copy_(xh, non_blocking=True)
+            for call in step_calls(xd):
+                call()
+            oh.copy_(B.out, non_blocking=True)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            xd.copy_(xh, non_blocking=True)
+            for call in step_calls(xd):
+                call()
+            oh.copy_(B.out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world, dev)
+        e2e = {"value": world * P * T * H * 2 / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": xh.numel() * xh.element_size(),
+               "d2h_bytes_per_step": oh.numel() * oh.element_size(), "ms_per_step": e2e_ms}
+
+    st = hq.hq_read_device_error()
+    if st != hq.HQ_OK:
+        raise RuntimeError(f"device error: {hq.hq_status_string(st)}")
+
+    # ---- CPU baseline (rank 0, N = 1) -----------------------------------------------------------
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cap = min(T, 2048)
+        step = OracleStep(cfg, host_rows(cfg, cap, dev))
+        S, _ = cpu_rows_for(step, args.cpu_seconds, cap)
+        t = step.run(S)
+        cpu = {"value": P * S * H * 2 / t / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": f"rows 0..{S - 1} of the evaluation batch, all {P} ranks: calibrate + select + "
+                         f"quantize-pack + dequant-reduce, {t:.1f} s single-threaded"}
+
+    if rank != 0:
+        return
+    peak, peak_src = measured_peak()
+    ab = algo_bytes(cfg)
+    kernels = {}
+    for n, t_ms in per_kernel.items():
+        gbs = ab[n] / (t_ms * 1e-3) / 1e9
+        kernels[n] = {"us": 1e3 * t_ms, "bytes": ab[n], "GB/s": gbs, "frac": gbs / peak}
+    dominant = max(per_kernel, key=per_kernel.get)
+    dom_gbs = kernels[dominant]["GB/s"]
+    step_bytes = sum(ab[n] for n in names)
+    part_bytes = P * T * H * 2
+    value = world * part_bytes * K / (ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": describe(cfg), "P": P, "T": T, "H": H, "k": k, "path": args.path,
+                   "step": "+".join(names), "parallelism": "replicas" if world > 1 else "single GPU",
+                   "l2": f"inputs larger than L2 ({part_bytes / 2**20:.0f} MiB of partial sums per step), no flush"
+                   if part_bytes > 126e6 else "inputs smaller than L2 (L2-resident between steps)"},
+        "hbm_frac_step": step_bytes * K / (ms_local * 1e-3) / 1e9 / peak,
+        "compression_ratio": compression_ratio(cfg),
+        "elements_per_s": world * P * T * H * K / (ms * 1e-3),
+        "roofline": {"bound": "hbm", "kernel": dominant, "achieved": dom_gbs, "peak": peak, "unit": "GB/s",
+                     "frac": dom_gbs / peak, "traffic": ncu_traffic(dominant, cfg.name), "peak_source": peak_src,
+                     "bytes_per_launch": ab[dominant]},
+        "kernels": kernels,
+        "alt_paths": alt,
+        "fused_equals_split": fused_equal,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": len(names) * K,
+        "clocks": clk,
+        "wall_s_timed": wall,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    cfg = workload(args.workload)
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, cfg, world, rank)
+        else:
+            run_hq(args, cfg, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,263 @@
+// hq_api.cu -- the C ABI of libhq.so (declared in include/hq.h).
+//
+// One translation unit holds every kernel (so the device error word is a single symbol).  Each
+// entry point checks its arguments on the host, picks a launch shape, enqueues one kernel on the
+// caller's stream and returns; nothing is allocated and nothing waits, except
+// hq_read_device_error, which synchronises the stream it is given.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "hq.h"
+#include "hq_common.cuh"
+#include "k_calibrate.cuh"
+#include "k_dequant.cuh"
+#include "k_fused.cuh"
+#include "k_quantize.cuh"
+#include "k_select.cuh"
+
+namespace {
+
+constexpr int kMaxRanks = 64;
+constexpr int kMaxDevices = 64;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+hq_status check_shape(int P, int H, int k) {
+  if (P < 1 || P > kMaxRanks) return HQ_ERR_INVALID_ARG;
+  if (H < 8 || H > hq::kMaxH || (H % 8) != 0) return HQ_ERR_INVALID_ARG;
+  if (k < 0 || k > H || (k % 8) != 0) return HQ_ERR_INVALID_ARG;
+  return HQ_OK;
+}
+
+// Launch-shape facts cached per device: SM count and resident CTAs per SM of each kernel.
+struct DeviceInfo {
+  int sms = 0;
+  int qp_blocks = 0;
+  bool select_smem_set = false;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+hq_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (d.sms == 0) {
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return HQ_ERR_CUDA;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.qp_blocks, hq::quantize_pack_kernel,
+                                                      hq::kQpThreads, 0) != cudaSuccess)
+      return HQ_ERR_CUDA;
+    if (d.qp_blocks < 1) d.qp_blocks = 1;
+  }
+  *out = &d;
+  return HQ_OK;
+}
+
+hq_status launched() { return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA; }
+
+long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
+
+// Persistent grid: at most `resident` CTAs, at least one unit per CTA.
+void split_units(long long units, long long resident, unsigned* grid, long long* per_cta) {
+  long long g = resident < units ? resident : units;
+  if (g < 1) g = 1;
+  *per_cta = ceil_div(units, g);
+  *grid = (unsigned)ceil_div(units, *per_cta);
+}
+
+template <typename OutT>
+hq_status launch_dequant(const uint32_t* codes, const uint16_t* side, int P, int T, int H, int k,
+                         const int32_t* keep_idx, const float* scale, const uint8_t* zero, void* out,
+                         cudaStream_t st, const DeviceInfo& d) {
+  const int G = hq::dq_groups_for(P);
+  const int RL = hq::kDqThreads / G;
+  const int S = (H / 8 + G - 1) / G;
+  const int NB = (int)ceil_div(T, (long long)RL * hq::kDqRows);
+  const size_t smem = ((size_t)P * G * 16 + (size_t)RL * hq::kDqRows * hq::kDqKeptChunk) * sizeof(float);
+  auto kern = hq::dequant_reduce_kernel<OutT>;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return HQ_ERR_CUDA;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, hq::kDqThreads, smem) != cudaSuccess)
+    return HQ_ERR_CUDA;
+  if (per_sm < 1) per_sm = 1;
+  unsigned grid;
+  long long per;
+  split_units((long long)S * NB, (long long)d.sms * per_sm, &grid, &per);
+  kern<<<grid, hq::kDqThreads, smem, st>>>(codes, side, P, T, H, k, keep_idx, scale, zero,
+                                            static_cast<OutT*>(out), G, S, NB, per);
+  return launched();
+}
+
+template <typename OutT>
+hq_status launch_fused(const uint16_t* x, int P, int T, int H, int k, const int32_t* keep_idx,
+                       const float* scale, const float* inv_scale, const uint8_t* zero, void* out,
+                       cudaStream_t st, const DeviceInfo& d) {
+  const int RL = hq::kFuThreads / hq::kFuGroups;
+  const int S = (H / 8 + hq::kFuGroups - 1) / hq::kFuGroups;
+  const int NB = (int)ceil_div(T, (long long)RL * hq::kFuRows);
+  auto kern = hq::compress_reduce_kernel<OutT>;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, hq::kFuThreads, 0) != cudaSuccess)
+    return HQ_ERR_CUDA;
+  if (per_sm < 1) per_sm = 1;
+  unsigned grid;
+  long long per;
+  split_units((long long)S * NB, (long long)d.sms * per_sm, &grid, &per);
+  kern<<<grid, hq::kFuThreads, 0, st>>>(x, P, T, H, k, keep_idx, scale, inv_scale, zero,
+                                         static_cast<OutT*>(out), S, NB, per);
+  return launched();
+}
+
+}  // namespace
+
+extern "C" {
+
+hq_status hq_calibrate(const uint16_t* x, int P, int T, int H, float beta, int first_batch,
+                       float* ema_min, float* ema_max, void* stream) {
+  if (check_shape(P, H, 0) != HQ_OK || T < 1) return HQ_ERR_INVALID_ARG;
+  if (!(beta >= 0.0f && beta < 1.0f)) return HQ_ERR_INVALID_ARG;
+  if (!x || !ema_min || !ema_max) return HQ_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(ema_min, 16) || !aligned(ema_max, 16)) return HQ_ERR_MISALIGNED;
+  const float one_minus_beta = 1.0f - beta;
+  dim3 grid((unsigned)((H + hq::kCalCols - 1) / hq::kCalCols), (unsigned)P);
+  hq::calibrate_kernel<<<grid, hq::kCalThreads, 0, (cudaStream_t)stream>>>(
+      x, T, H, beta, one_minus_beta, first_batch ? 1 : 0, ema_min, ema_max);
+  return launched();
+}
+
+hq_status hq_select_topk(const float* ema_min, const float* ema_max, int P, int H, int k,
+                         int32_t* keep_idx, int32_t* rest_idx, float* scale, float* inv_scale,
+                         uint8_t* zero, void* stream) {
+  if (check_shape(P, H, k) != HQ_OK) return HQ_ERR_INVALID_ARG;
+  if (!ema_min || !ema_max || !scale || !inv_scale || !zero) return HQ_ERR_INVALID_ARG;
+  if ((k > 0 && !keep_idx) || (k < H && !rest_idx)) return HQ_ERR_INVALID_ARG;
+  if (!aligned(ema_min, 16) || !aligned(ema_max, 16) || !aligned(scale, 16) ||
+      !aligned(inv_scale, 16) || !aligned(zero, 16) || !aligned(keep_idx, 4) || !aligned(rest_idx, 4))
+    return HQ_ERR_MISALIGNED;
+  DeviceInfo* d = nullptr;
+  if (device_info(&d) != HQ_OK) return HQ_ERR_CUDA;
+  const size_t smem = (size_t)H * sizeof(uint32_t);
+  {
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    if (!d->select_smem_set) {
+      if (cudaFuncSetAttribute(hq::select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)(hq::kMaxH * sizeof(uint32_t))) != cudaSuccess)
+        return HQ_ERR_CUDA;
+      d->select_smem_set = true;
+    }
+  }
+  hq::select_topk_kernel<<<1, hq::kSelThreads, smem, (cudaStream_t)stream>>>(
+      ema_min, ema_max, P, H, k, keep_idx, rest_idx, scale, inv_scale, zero);
+  return launched();
+}
+
+hq_status hq_quantize_pack(const uint16_t* x, int P, int T, int H, int k, const int32_t* keep_idx,
+                           const int32_t* rest_idx, const float* inv_scale, const uint8_t* zero,
+                           uint32_t* codes, uint16_t* side, void* stream) {
+  if (check_shape(P, H, k) != HQ_OK || T < 0) return HQ_ERR_INVALID_ARG;
+  if (!inv_scale || !zero) return HQ_ERR_INVALID_ARG;
+  if ((k > 0 && !keep_idx) || (k < H && !rest_idx)) return HQ_ERR_INVALID_ARG;
+  if (T > 0 && (!x || (k > 0 && !side) || (k < H && !codes))) return HQ_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(side, 16) || !aligned(codes, 4) || !aligned(inv_scale, 16) ||
+      !aligned(zero, 16) || !aligned(keep_idx, 4) || !aligned(rest_idx, 4))
+    return HQ_ERR_MISALIGNED;
+  if (T == 0) return HQ_OK;
+  DeviceInfo* d = nullptr;
+  if (device_info(&d) != HQ_OK) return HQ_ERR_CUDA;
+  const int S = (H / 8 + hq::kQpGroups - 1) / hq::kQpGroups;
+  const long long units = (long long)P * S * T;
+  unsigned grid;
+  long long per;
+  split_units(ceil_div(units, hq::kQpRows), (long long)d->sms * d->qp_blocks, &grid, &per);
+  per *= hq::kQpRows;
+  grid = (unsigned)ceil_div(units, per);
+  hq::quantize_pack_kernel<<<grid, hq::kQpThreads, 0, (cudaStream_t)stream>>>(
+      x, P, T, H, k, keep_idx, rest_idx, inv_scale, zero, codes, side, S, per);
+  return launched();
+}
+
+hq_status hq_dequant_reduce(const uint32_t* codes, const uint16_t* side, int P, int T, int H, int k,
+                            const int32_t* keep_idx, const int32_t* rest_idx, const float* scale,
+                            const uint8_t* zero, void* out, hq_out_dtype out_dtype, void* stream) {
+  if (check_shape(P, H, k) != HQ_OK || T < 0) return HQ_ERR_INVALID_ARG;
+  if (out_dtype != HQ_OUT_BF16 && out_dtype != HQ_OUT_F32) return HQ_ERR_INVALID_ARG;
+  if (!scale || !zero) return HQ_ERR_INVALID_ARG;
+  if ((k > 0 && !keep_idx) || (k < H && !rest_idx)) return HQ_ERR_INVALID_ARG;
+  if (T > 0 && (!out || (k > 0 && !side) || (k < H && !codes))) return HQ_ERR_INVALID_ARG;
+  if (!aligned(out, 16) || !aligned(side, 16) || !aligned(codes, 4) || !aligned(scale, 16) ||
+      !aligned(zero, 16) || !aligned(keep_idx, 4) || !aligned(rest_idx, 4))
+    return HQ_ERR_MISALIGNED;
+  if (T == 0) return HQ_OK;
+  DeviceInfo* d = nullptr;
+  if (device_info(&d) != HQ_OK) return HQ_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (out_dtype == HQ_OUT_BF16)
+    return launch_dequant<uint16_t>(codes, side, P, T, H, k, keep_idx, scale, zero, out, st, *d);
+  return launch_dequant<float>(codes, side, P, T, H, k, keep_idx, scale, zero, out, st, *d);
+}
+
+hq_status hq_compress_reduce(const uint16_t* x, int P, int T, int H, int k, const int32_t* keep_idx,
+                             const int32_t* rest_idx, const float* scale, const float* inv_scale,
+                             const uint8_t* zero, void* out, hq_out_dtype out_dtype,
+                             uint32_t* codes_or_null, uint16_t* side_or_null, void* stream) {
+  if (check_shape(P, H, k) != HQ_OK || T < 0) return HQ_ERR_INVALID_ARG;
+  if (out_dtype != HQ_OUT_BF16 && out_dtype != HQ_OUT_F32) return HQ_ERR_INVALID_ARG;
+  if (!scale || !inv_scale || !zero) return HQ_ERR_INVALID_ARG;
+  if ((k > 0 && !keep_idx) || (k < H && !rest_idx)) return HQ_ERR_INVALID_ARG;
+  if (T > 0 && (!x || !out)) return HQ_ERR_INVALID_ARG;
+  const bool wire = codes_or_null || side_or_null;
+  if (T > 0 && wire && ((k > 0 && !side_or_null) || (k < H && !codes_or_null))) return HQ_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(out, 16) || !aligned(scale, 16) || !aligned(inv_scale, 16) ||
+      !aligned(zero, 16) || !aligned(keep_idx, 4) || !aligned(rest_idx, 4) ||
+      !aligned(codes_or_null, 4) || !aligned(side_or_null, 16))
+    return HQ_ERR_MISALIGNED;
+  if (T == 0) return HQ_OK;
+  DeviceInfo* d = nullptr;
+  if (device_info(&d) != HQ_OK) return HQ_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (wire) {
+    const hq_status q = hq_quantize_pack(x, P, T, H, k, keep_idx, rest_idx, inv_scale, zero,
+                                         codes_or_null, side_or_null, stream);
+    if (q != HQ_OK) return q;
+  }
+  if (out_dtype == HQ_OUT_BF16)
+    return launch_fused<uint16_t>(x, P, T, H, k, keep_idx, scale, inv_scale, zero, out, st, *d);
+  return launch_fused<float>(x, P, T, H, k, keep_idx, scale, inv_scale, zero, out, st, *d);
+}
+
+const char* hq_status_string(hq_status s) {
+  switch (s) {
+    case HQ_OK: return "HQ_OK";
+    case HQ_ERR_INVALID_ARG: return "HQ_ERR_INVALID_ARG";
+    case HQ_ERR_MISALIGNED: return "HQ_ERR_MISALIGNED";
+    case HQ_ERR_CUDA: return "HQ_ERR_CUDA";
+    case HQ_ERR_TIMEOUT: return "HQ_ERR_TIMEOUT";
+    case HQ_ERR_BAD_INDEX: return "HQ_ERR_BAD_INDEX";
+  }
+  return "HQ_ERR_UNKNOWN";
+}
+
+hq_status hq_read_device_error(void* stream) {
+  cudaStream_t st = (cudaStream_t)stream;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbolAsync(&v, hq::g_error_word, sizeof v, 0, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return HQ_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return HQ_ERR_CUDA;
+  const unsigned int zero = 0;
+  if (cudaMemcpyToSymbolAsync(hq::g_error_word, &zero, sizeof zero, 0, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return HQ_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return HQ_ERR_CUDA;
+  return (hq_status)v;
+}
+
+int64_t hq_wire_bytes_per_row(int H, int k) {
+  if (H < 0 || k < 0 || k > H) return -1;
+  return (int64_t)(H - k) / 2 + 2 * (int64_t)k;
+}
+
+}  // extern "C"

@@ -1,0 +1,106 @@
+// hq_common.cuh -- device helpers shared by the libhq kernels (sm_100a).
+//
+// Floating-point discipline: every float operation on the data path is written as an explicit
+// round-to-nearest intrinsic (__fmul_rn, __fadd_rn, __fmaf_rn, __fdiv_rn, __frcp_rn) and the
+// library is compiled with -fmad=false and without fast-math, so that each step is exactly one
+// IEEE-754 single-precision operation and denormals are kept.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "hq.h"
+
+namespace hq {
+
+// One error word per device; the first recorded status wins.  Read and cleared by
+// hq_read_device_error().
+__device__ unsigned int g_error_word = 0;
+
+__device__ __forceinline__ void record_error(hq_status s) {
+  atomicCAS(&g_error_word, 0u, (unsigned)s);
+}
+
+// bf16 halves of a 32-bit word -> fp32 (exact).
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Element i (0..7) of eight bf16 values held in a uint4.
+__device__ __forceinline__ float bf16_at(const uint4& v, int i) {
+  const uint32_t w = (i < 2) ? v.x : (i < 4) ? v.y : (i < 6) ? v.z : v.w;
+  return (i & 1) ? bf16_hi(w) : bf16_lo(w);
+}
+
+// Two fp32 -> two bf16 (round to nearest even), NaN -> 0x7FC0; a in the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+  if (a != a) r = (r & 0xFFFF0000u) | 0x7FC0u;
+  if (b != b) r = (r & 0x0000FFFFu) | 0x7FC00000u;
+  return r;
+}
+
+// Streaming 16-byte load: read once, do not keep in L1.
+__device__ __forceinline__ uint4 ld_stream16(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// Number of entries of the ascending array a[0..n) that are < key (lower bound).
+__device__ __forceinline__ int lower_bound_i32(const int32_t* __restrict__ a, int n, int key) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(a + mid) < key) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo;
+}
+
+// Kept-feature layout of one group of 8 consecutive features [h0, h0+8):
+//   j0    = number of kept features before h0 (index of the group's first kept in keep_idx)
+//   kmask = bit i set when feature h0+i is kept
+//   c0    = compact (rest_idx) position of the group's first non-kept feature = h0 - j0
+// Every keep_idx entry read is range-checked; a bad entry is recorded and ignored.
+struct GroupLayout {
+  int j0;
+  int c0;
+  uint32_t kmask;
+  int n;  // non-kept features in the group
+};
+
+__device__ __forceinline__ GroupLayout group_layout(const int32_t* __restrict__ keep_idx, int k, int H,
+                                                    int h0) {
+  GroupLayout L;
+  L.j0 = lower_bound_i32(keep_idx, k, h0);
+  const int j1 = lower_bound_i32(keep_idx, k, h0 + 8);
+  L.kmask = 0;
+  for (int j = L.j0; j < j1 && j < L.j0 + 8; ++j) {
+    const int d = __ldg(keep_idx + j) - h0;
+    if (d >= 0 && d < 8) L.kmask |= 1u << d;
+    else record_error(HQ_ERR_BAD_INDEX);
+  }
+  if (j1 - L.j0 > 8) record_error(HQ_ERR_BAD_INDEX);
+  L.n = 8 - __popc(L.kmask);
+  L.c0 = h0 - L.j0;
+  if (L.c0 < 0 || L.c0 > H - k) {
+    record_error(HQ_ERR_BAD_INDEX);
+    L.c0 = min(max(L.c0, 0), H - k);
+  }
+  return L;
+}
+
+// Column index read from keep_idx / rest_idx, clamped into [0, H) with the error recorded.
+__device__ __forceinline__ int checked_col(const int32_t* __restrict__ idx, int j, int H) {
+  int h = __ldg(idx + j);
+  if (h < 0 || h >= H) {
+    record_error(HQ_ERR_BAD_INDEX);
+    h = 0;
+  }
+  return h;
+}
+
+}  // namespace hq

@@ -1,0 +1,152 @@
+/*
+ * hq.h -- C ABI of libhq.so: hybrid BF16/Int4 compression of tensor-parallel partial sums on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method is the one summarised on the page "Revolutionizing LLM Inference: The Power of
+ * Efficient Low-Bit Communication" (about "Towards Efficient Low-Bit Communication for Tensor
+ * Parallel LLM Inference"):
+ *   - section "Combating Quantization Errors with Tensor Parallelism": each rank's partial sum
+ *     is quantized *before* the ranks synchronise, so the per-rank errors add up around zero;
+ *   - section "The Hybrid Quantization Algorithm": Calibration (per-feature moving averages of
+ *     the observed min and max on each device), Selection of High Precision Features (rank
+ *     features by quantization range, keep the top ones in BF16), Inference (the rest go to
+ *     4 bits; after communication everything is converted back and summed across devices).
+ * The page gives no formula, bit layout or interface; the exact arithmetic below is a stated
+ * reading of it (the readings are numbered R1..R14 where they are used).
+ *
+ * Notation: P ranks, T rows (tokens), H features (columns), k features kept in BF16, H' = H - k.
+ * One GPU simulates the P ranks: a tensor [P][T][H] holds every rank's partial sum, and the
+ * per-rank semantics are the same as for one real rank calling with P = 1 on its own slice.
+ *
+ * Conventions for every call:
+ *   - All arrays are dense, row-major, in device memory, owned by the caller.  The library
+ *     allocates nothing and keeps no state between calls (apart from one device error word, see
+ *     hq_read_device_error).  bf16 values are passed as their uint16_t bit patterns.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  Every call
+ *     only enqueues work on it and returns; results are ready when the stream reaches them.
+ *   - Arguments are checked on the host before anything is enqueued.  On a bad argument the
+ *     call returns HQ_ERR_INVALID_ARG or HQ_ERR_MISALIGNED and enqueues nothing.  A failed
+ *     launch returns HQ_ERR_CUDA.
+ *   - Shape limits: 1 <= P <= 64; 8 <= H <= 32768 with H % 8 == 0; 0 <= k <= H with k % 8 == 0.
+ *     A pointer to an array that is empty for the given sizes (keep_idx/side when k == 0,
+ *     rest_idx/codes when k == H, every per-row array when T == 0) may be NULL.
+ *   - Alignment: x, side, out, ema_min, ema_max, scale, inv_scale and zero 16 bytes; codes,
+ *     keep_idx and rest_idx 4 bytes.
+ *   - keep_idx must be strictly ascending with values in [0, H) and rest_idx must be its
+ *     ascending complement, as hq_select_topk writes them.  The kernels read every index
+ *     through range checks: an index outside [0, H) is not dereferenced, and the first one seen
+ *     sets the device error word to HQ_ERR_BAD_INDEX (the outputs are then unspecified).
+ *   - Outputs must not overlap inputs.
+ */
+#ifndef HQ_H
+#define HQ_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HQ_OK = 0,
+  HQ_ERR_INVALID_ARG = 1, /* a size, count, decay or NULL pointer outside the rules above   */
+  HQ_ERR_MISALIGNED = 2,  /* a pointer below its required alignment                          */
+  HQ_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed                     */
+  HQ_ERR_TIMEOUT = 4,     /* a bounded device-side wait gave up (device error word)          */
+  HQ_ERR_BAD_INDEX = 5    /* a kernel met an index outside [0, H) (device error word)        */
+} hq_status;
+
+typedef enum { HQ_OUT_BF16 = 0, HQ_OUT_F32 = 1 } hq_out_dtype;
+
+/*
+ * Calibration -- section "The Hybrid Quantization Algorithm", bullet "Calibration".
+ * Folds one calibration batch into the per-rank, per-feature moving averages of min and max
+ * (R1, R2): for each rank r and feature h, bmin/bmax = min/max over the batch's T rows of
+ * x[r][t][h] (NaN values are skipped; a result of -0 is stored as +0), then
+ *   first_batch != 0:  ema_min = bmin,  ema_max = bmax;
+ *   otherwise:         ema = beta*ema + (1-beta)*b, each product and the sum rounded to fp32,
+ *                      with (1-beta) itself computed in fp32.
+ *   x        bf16 [P][T][H], T >= 1
+ *   beta     decay, 0 <= beta < 1
+ *   ema_min, ema_max  float [P][H], read (unless first_batch) and written
+ */
+hq_status hq_calibrate(const uint16_t* x, int P, int T, int H, float beta, int first_batch,
+                       float* ema_min, float* ema_max, void* stream);
+
+/*
+ * Selection -- section "The Hybrid Quantization Algorithm", bullet "Selection of High
+ * Precision Features", with the 4-bit grid of bullet "Calibration" (R3, R4, R5, R14).
+ * For every rank and feature: lo = min(ema_min, 0), hi = max(ema_max, 0),
+ *   scale = (hi - lo)/15, inv_scale = 1/scale (both correctly rounded fp32),
+ *   zero  = clamp(rint(-lo * inv_scale), 0, 15)  (round half to even);
+ *   a scale that is 0, subnormal, infinite or NaN gives scale = inv_scale = 1, zero = 0.
+ * Score of a feature = sum over ranks, in rank order in fp32, of (hi - lo).  The k features with
+ * the largest scores are kept in BF16 (equal scores: lower feature index first).
+ *   ema_min, ema_max  float [P][H]
+ *   keep_idx int32 [k]    the kept features, ascending
+ *   rest_idx int32 [H-k]  all other features, ascending
+ *   scale, inv_scale float [P][H], zero uint8 [P][H]  (computed for kept features too)
+ */
+hq_status hq_select_topk(const float* ema_min, const float* ema_max, int P, int H, int k,
+                         int32_t* keep_idx, int32_t* rest_idx, float* scale, float* inv_scale,
+                         uint8_t* zero, void* stream);
+
+/*
+ * Quantize-pack, the sending side of bullet "Inference" (R6, R7).  For every rank r and row t:
+ *   side[r][t][j]  = x[r][t][keep_idx[j]]                     (bf16 bits, unchanged)
+ *   code of compact column c (feature h = rest_idx[c]):
+ *     q = clamp(rint(x * inv_scale[r][h]) + zero[r][h], 0, 15), the product in fp32,
+ *     round half to even; +-inf saturate to 15 / 0; NaN gives q = zero[r][h].
+ *   codes[r][t][c/8] holds code c in bits 4*(c%8) .. 4*(c%8)+3.
+ *   x     bf16 [P][T][H]      (T >= 0; T == 0 enqueues nothing)
+ *   codes uint32 [P][T][H'/8] -- the wire buffer of the 4-bit part
+ *   side  bf16 [P][T][k]      -- the wire buffer of the BF16 part
+ */
+hq_status hq_quantize_pack(const uint16_t* x, int P, int T, int H, int k, const int32_t* keep_idx,
+                           const int32_t* rest_idx, const float* inv_scale, const uint8_t* zero,
+                           uint32_t* codes, uint16_t* side, void* stream);
+
+/*
+ * Dequant-reduce, the receiving side of bullet "Inference": every rank's shard is converted back
+ * and the ranks are summed in rank order (R9, R10, R11).  For row t:
+ *   non-kept feature h = rest_idx[c]:  acc = +0;  for r = 0..P-1:
+ *       acc = fma(float(q_r - zero[r][h]), scale[r][h], acc)      (one rounding per rank)
+ *   kept feature h = keep_idx[j]:      acc = +0;  for r = 0..P-1:  acc = acc + side[r][t][j]
+ *   out[t][h] = acc as fp32 (HQ_OUT_F32), or rounded to bf16 nearest-even (HQ_OUT_BF16); a
+ *   NaN sum is written as the canonical quiet NaN (0x7FC00000 / 0x7FC0).
+ *   codes, side as written by hq_quantize_pack; out [T][H] of the chosen type.
+ */
+hq_status hq_dequant_reduce(const uint32_t* codes, const uint16_t* side, int P, int T, int H, int k,
+                            const int32_t* keep_idx, const int32_t* rest_idx, const float* scale,
+                            const uint8_t* zero, void* out, hq_out_dtype out_dtype, void* stream);
+
+/*
+ * Fused compress-reduce (section "Combating Quantization Errors with Tensor Parallelism": the
+ * partial sums are quantized and then summed): out equals hq_quantize_pack followed by
+ * hq_dequant_reduce, bit for bit (R12), computed from x in one pass without a wire buffer.
+ * If codes_or_null / side_or_null are not NULL the wire buffers are written too (by the
+ * quantize-pack kernel, i.e. x is read a second time in that case).
+ */
+hq_status hq_compress_reduce(const uint16_t* x, int P, int T, int H, int k, const int32_t* keep_idx,
+                             const int32_t* rest_idx, const float* scale, const float* inv_scale,
+                             const uint8_t* zero, void* out, hq_out_dtype out_dtype,
+                             uint32_t* codes_or_null, uint16_t* side_or_null, void* stream);
+
+/* A static string naming a status. */
+const char* hq_status_string(hq_status s);
+
+/*
+ * Synchronises `stream`, then returns and clears the device error word of the current device:
+ * HQ_OK if no kernel recorded an error since the last call, else the first recorded status
+ * (HQ_ERR_BAD_INDEX, HQ_ERR_TIMEOUT).  Returns HQ_ERR_CUDA if the synchronisation fails.
+ */
+hq_status hq_read_device_error(void* stream);
+
+/* Bytes of the two wire buffers per rank and row: 4-bit part (H-k)/2, BF16 part 2k. */
+int64_t hq_wire_bytes_per_row(int H, int k);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HQ_H */

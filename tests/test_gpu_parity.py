@@ -1,0 +1,223 @@
+"""CUDA path vs the CPU oracle, through the C ABI, on seeded synthetic inputs.
+
+Integer and index results (codes, zero points, keep/rest sets, side buffers) and the fp32 results
+(moving averages, scales, reduced outputs) must all be bit-identical: both sides evaluate the same
+sequence of correctly rounded fp32 operations, and the reduction order over ranks is fixed.
+Small and mid-size problems are compared element by element; the two full-size workloads
+(prefill 7B and 70B shapes) on sampled rows and columns the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+
+import synth
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+import bit_tensor_activation_b200 as hq  # noqa: E402
+import oracle  # noqa: E402
+from gpu_helpers import (DEV, assert_no_device_error, compare_all, f32bits, gpu_calibrate_batches,  # noqa: E402
+                         gpu_dequant, gpu_fused, gpu_quantize, gpu_select, params_to_dev, to_dev_u16, u16, u32)
+
+
+def _batches(cfg, cs, T=None):
+    return [synth.fill_cpu(cfg, synth.CALIB, b, T=cfg.calib_T if T is None else T, cs=cs)
+            for b in range(cfg.calib_batches)]
+
+
+@pytest.mark.parametrize("name", ["pr1", "decode"])
+def test_named_small_configs_bit_exact(name):
+    cfg = synth.CONFIGS[name]
+    cs, outl = synth.colscale(cfg)
+    ref = compare_all(cfg, _batches(cfg, cs), synth.fill_cpu(cfg, synth.EVAL, 0, cs=cs))
+    assert set(outl.tolist()) <= set(ref["sel"]["keep_idx"].tolist())
+
+
+# Mid-size shapes: several slices / row blocks with ragged tails, k = 0 and k = H, odd P.
+MID = [
+    synth.CONFIGS["prefill7b"].with_(name="7b_ragged", T=37, H=3000, k=96, n_out=40, calib_batches=3, calib_T=41),
+    synth.CONFIGS["prefill70b"].with_(name="70b_ragged", T=19, H=8200, k=264, n_out=100, calib_batches=2, calib_T=23),
+    synth.CONFIGS["decode"].with_(name="p3_k0", P=3, T=50, H=1032, k=0, calib_batches=2, calib_T=7),
+    synth.CONFIGS["decode"].with_(name="p5_kH", P=5, T=9, H=520, k=520, n_out=8, calib_batches=2, calib_T=5),
+    synth.CONFIGS["pr1"].with_(name="h8", P=4, T=33, H=8, k=8, n_out=1, calib_batches=2, calib_T=3),
+    synth.CONFIGS["pr1"].with_(name="h8k0", P=1, T=1, H=8, k=0, n_out=1, calib_batches=1, calib_T=1),
+    synth.CONFIGS["decode"].with_(name="p16", P=16, T=21, H=2048, k=32, calib_batches=2, calib_T=9),
+    synth.CONFIGS["decode"].with_(name="p64", P=64, T=5, H=264, k=16, n_out=8, calib_batches=1, calib_T=4),
+    synth.sweep_configs()[5].with_(name="sweep_mid", T=100, calib_batches=2, calib_T=64),
+]
+
+
+@pytest.mark.parametrize("cfg", MID, ids=[c.name for c in MID])
+def test_mid_shapes_bit_exact(cfg):
+    cs, _ = synth.colscale(cfg)
+    compare_all(cfg, _batches(cfg, cs), synth.fill_cpu(cfg, synth.EVAL, 0, cs=cs))
+
+
+def test_clustered_kept_features_bit_exact():
+    """Kept features in long runs (whole groups and slices kept) stress the compact layout."""
+    o = oracle.get()
+    rng = np.random.default_rng(3)
+    P, T, H, k = 3, 40, 2560, 1104
+    x = synth.fill_cpu(synth.CONFIGS["decode"].with_(P=P, T=T, H=H, n_out=4), synth.EVAL, 0,
+                       cs=np.ones(H))
+    emin = -np.ones((P, H), np.float32)
+    emax = np.ones((P, H), np.float32)
+    big = np.r_[0:8, 100:1100, 1500:1580, 2544:2560]  # runs across groups and 1024-feature slices
+    emax[:, big] = 50.0
+    emin[:, big] = -50.0
+    emax += rng.uniform(0, 0.01, (P, H)).astype(np.float32)
+    sel = o.select_topk(emin, emax, k)
+    assert set(big.tolist()) <= set(sel["keep_idx"].tolist())
+    prm = params_to_dev(sel)
+    B = gpu_select(torch.from_numpy(emin).to(DEV), torch.from_numpy(emax).to(DEV), k)
+    assert np.array_equal(B["keep_idx"].cpu().numpy(), sel["keep_idx"])
+    codes_r, side_r = o.quantize_pack(x, sel["keep_idx"], sel["rest_idx"], sel["inv_scale"], sel["zero"])
+    out_r = o.dequant_reduce(codes_r, side_r, H, sel["keep_idx"], sel["rest_idx"], sel["scale"], sel["zero"])
+    xd = to_dev_u16(x)
+    codes, side = gpu_quantize(xd, prm)
+    out = gpu_dequant(codes, side, prm, H)
+    fused, _, _ = gpu_fused(xd, prm)
+    assert_no_device_error()
+    assert np.array_equal(u32(codes), codes_r) and np.array_equal(u16(side), side_r)
+    assert np.array_equal(u16(out), out_r) and np.array_equal(u16(fused), out_r)
+
+
+def test_select_ties_and_special_values():
+    o = oracle.get()
+    P, H = 3, 4096
+    rng = np.random.default_rng(5)
+    emin = (-rng.integers(0, 4, (P, H))).astype(np.float32)   # many exact ties
+    emax = rng.integers(0, 4, (P, H)).astype(np.float32)
+    emin[0, 10], emax[0, 10] = np.nan, np.nan                  # NaN statistics -> range 0
+    emax[1, 20] = np.inf                                       # infinite range -> degenerate scale
+    emin[2, 30] = -np.inf
+    emin[1, 40], emax[1, 40] = -1e-39, 1e-39                   # subnormal scale -> degenerate
+    emin[2, 50], emax[2, 50] = 3e38, 3.3e38                    # huge but finite
+    emin[0, 60], emax[0, 60] = -3e38, 3e38                     # range overflows to inf
+    for k in (0, 8, 256, 2048, 4088, 4096):
+        sel = o.select_topk(emin, emax, k)
+        B = gpu_select(torch.from_numpy(emin).to(DEV), torch.from_numpy(emax).to(DEV), k)
+        assert_no_device_error()
+        assert np.array_equal(B["keep_idx"].cpu().numpy(), sel["keep_idx"]), k
+        assert np.array_equal(B["rest_idx"].cpu().numpy(), sel["rest_idx"]), k
+        assert np.array_equal(f32bits(B["scale"]), f32bits(sel["scale"]))
+        assert np.array_equal(f32bits(B["inv_scale"]), f32bits(sel["inv_scale"]))
+        assert np.array_equal(B["zero"].cpu().numpy(), sel["zero"])
+    all_equal = np.zeros((P, H), np.float32)
+    sel = o.select_topk(all_equal - 1, all_equal + 1, 64)
+    B = gpu_select(torch.from_numpy(all_equal - 1).to(DEV), torch.from_numpy(all_equal + 1).to(DEV), 64)
+    assert B["keep_idx"].cpu().numpy().tolist() == list(range(64)) == sel["keep_idx"].tolist()
+
+
+def test_special_input_values_bit_exact():
+    """NaN, +-inf, -0, huge and subnormal partial sums in x, and in calibration."""
+    o = oracle.get()
+    cfg = synth.CONFIGS["decode"].with_(P=4, T=24, H=1024, k=32, calib_batches=2, calib_T=16)
+    cs, _ = synth.colscale(cfg)
+    cal = _batches(cfg, cs)
+    cal[1][2, 3, 7] = 0x7FC0          # NaN in calibration
+    cal[0][1, :, 9] = 0x8000          # a column of -0
+    x = synth.fill_cpu(cfg, synth.EVAL, 0, cs=cs)
+    specials = [0x7FC0, 0xFFC1, 0x7F80, 0xFF80, 0x8000, 0x0001, 0x8001, 0x7F7F, 0xFF7F]
+    rng = np.random.default_rng(9)
+    for v in specials:
+        for _ in range(40):
+            x[rng.integers(cfg.P), rng.integers(cfg.T), rng.integers(cfg.H)] = v
+    compare_all(cfg, cal, x)
+
+
+def test_empty_rows_are_no_ops():
+    prm = params_to_dev(oracle.get().select_topk(-np.ones((2, 64), np.float32), np.ones((2, 64), np.float32), 8))
+    x = torch.empty((2, 0, 64), dtype=torch.int16, device=DEV)
+    codes, side = gpu_quantize(x, prm)
+    out = gpu_dequant(codes, side, prm, 64)
+    fused, _, _ = gpu_fused(x, prm)
+    assert out.numel() == 0 and fused.numel() == 0
+    assert_no_device_error()
+
+
+def test_bad_index_is_recorded_not_dereferenced():
+    """keep_idx holding an index outside [0, H): the kernels clamp it and report HQ_ERR_BAD_INDEX."""
+    P, T, H, k = 2, 8, 256, 8
+    prm = params_to_dev(oracle.get().select_topk(-np.ones((P, H), np.float32), np.ones((P, H), np.float32), k))
+    bad = prm["keep_idx"].clone()
+    bad[-1] = H + 1000
+    prm["keep_idx"] = bad
+    x = torch.zeros((P, T, H), dtype=torch.int16, device=DEV)
+    gpu_quantize(x, prm)
+    assert hq.hq_read_device_error() == hq.HQ_ERR_BAD_INDEX
+    assert hq.hq_read_device_error() == hq.HQ_OK, "reading clears the word"
+
+
+# ---------------------------------------------------------------------------------------------
+# Full-size workloads in the launch shapes the benchmark times
+# ---------------------------------------------------------------------------------------------
+def _gpu_batch(cfg, purpose, batch, cs_dev, T=None):
+    T = cfg.T if T is None else T
+    out = torch.empty((cfg.P, T, cfg.H), dtype=torch.int16, device=DEV)
+    synth.fill_gpu(cfg, purpose, batch, out, cs_dev, T=T)
+    return out
+
+
+@pytest.mark.parametrize("name", ["prefill7b", "prefill70b"])
+def test_full_size_calibration_sampled(name):
+    cfg = synth.CONFIGS[name]
+    cs, outl = synth.colscale(cfg)
+    cs_dev = torch.from_numpy(cs).to(DEV)
+    buf = torch.empty((cfg.P, cfg.calib_T, cfg.H), dtype=torch.int16, device=DEV)
+    emin = torch.empty((cfg.P, cfg.H), dtype=torch.float32, device=DEV)
+    emax = torch.empty_like(emin)
+    for b in range(cfg.calib_batches):
+        synth.fill_gpu(cfg, synth.CALIB, b, buf, cs_dev, T=cfg.calib_T)
+        hq.hq_calibrate(buf, emin, emax, cfg.beta, b == 0)
+    B = gpu_select(emin, emax, cfg.k)
+    assert_no_device_error()
+    keep = set(B["keep_idx"].cpu().numpy().tolist())
+    assert set(outl.tolist()) <= keep, "planted outlier columns must be selected"
+    gmin, gmax = emin.cpu().numpy(), emax.cpu().numpy()
+    o = oracle.get()
+    rng = np.random.default_rng(17)
+    cols = np.concatenate([rng.choice(cfg.H, 10, replace=False), outl[:2]])
+    for h in cols:
+        r = int(rng.integers(cfg.P))
+        cal = [synth.fill_cpu(cfg, synth.CALIB, b, ranks=(r, r + 1), cols=(int(h), int(h) + 1), T=cfg.calib_T, cs=cs)
+               for b in range(cfg.calib_batches)]
+        em, ex = o.calibrate_batches(cal, cfg.beta)
+        assert f32bits(gmin[r, h]) == f32bits(em[0, 0]) and f32bits(gmax[r, h]) == f32bits(ex[0, 0]), (r, h)
+
+
+@pytest.mark.parametrize("name", ["prefill7b", "prefill70b"])
+def test_full_size_select_quantize_reduce_sampled(name):
+    cfg = synth.CONFIGS[name]
+    o = oracle.get()
+    cs, outl = synth.colscale(cfg)
+    # statistics from a reduced calibration on the host (any statistics serve as select input)
+    cal = _batches(cfg.with_(calib_batches=4), cs, T=48)
+    emin, emax = o.calibrate_batches(cal, cfg.beta)
+    sel = o.select_topk(emin, emax, cfg.k)
+    B = gpu_select(torch.from_numpy(emin).to(DEV), torch.from_numpy(emax).to(DEV), cfg.k)
+    assert np.array_equal(B["keep_idx"].cpu().numpy(), sel["keep_idx"])
+    assert np.array_equal(B["rest_idx"].cpu().numpy(), sel["rest_idx"])
+    assert np.array_equal(f32bits(B["scale"]), f32bits(sel["scale"]))
+    assert np.array_equal(f32bits(B["inv_scale"]), f32bits(sel["inv_scale"]))
+    assert np.array_equal(B["zero"].cpu().numpy(), sel["zero"])
+    prm = params_to_dev(sel)
+    x = _gpu_batch(cfg, synth.EVAL, 0, torch.from_numpy(cs).to(DEV))
+    codes, side = gpu_quantize(x, prm)
+    out = gpu_dequant(codes, side, prm, cfg.H)
+    fused, _, _ = gpu_fused(x, prm)
+    assert_no_device_error()
+    assert torch.equal(out, fused), "fused == split over the whole output"
+    rng = np.random.default_rng(23)
+    rows = np.unique(np.concatenate([[0, cfg.T - 1], rng.integers(0, cfg.T, 10)]))
+    codes_h, side_h, out_h = u32(codes), u16(side), u16(out)
+    for t in rows:
+        xr = synth.fill_cpu(cfg, synth.EVAL, 0, rows=(int(t), int(t) + 1), cs=cs)
+        c_r, s_r = o.quantize_pack(xr, sel["keep_idx"], sel["rest_idx"], sel["inv_scale"], sel["zero"])
+        o_r = o.dequant_reduce(c_r, s_r, cfg.H, sel["keep_idx"], sel["rest_idx"], sel["scale"], sel["zero"])
+        assert np.array_equal(codes_h[:, t:t + 1], c_r), f"codes row {t}"
+        assert np.array_equal(side_h[:, t:t + 1], s_r), f"side row {t}"
+        assert np.array_equal(out_h[t:t + 1], o_r), f"out row {t}"
