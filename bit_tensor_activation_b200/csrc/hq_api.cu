@@ -47,8 +47,11 @@ hq_status device_info(DeviceInfo** out) {
   if (d.sms == 0) {
     if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return HQ_ERR_CUDA;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.qp_blocks, hq::quantize_pack_kernel,
-                                                      hq::kQpThreads, 0) != cudaSuccess)
+    const int qp_smem = (int)(hq::kQpWarps * sizeof(hq::QpWarpSmem));
+    if (cudaFuncSetAttribute(hq::quantize_pack_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             qp_smem) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.qp_blocks, hq::quantize_pack_kernel,
+                                                      hq::kQpThreads, qp_smem) != cudaSuccess)
       return HQ_ERR_CUDA;
     if (d.qp_blocks < 1) d.qp_blocks = 1;
   }
@@ -60,36 +63,34 @@ hq_status launched() { return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR
 
 long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
 
-// Persistent grid: at most `resident` CTAs, at least one unit per CTA.
-void split_units(long long units, long long resident, unsigned* grid, long long* per_cta) {
-  long long g = resident < units ? resident : units;
-  if (g < 1) g = 1;
-  *per_cta = ceil_div(units, g);
-  *grid = (unsigned)ceil_div(units, *per_cta);
+// Slices x row chunks for the dequant-reduce and fused kernels: one wave of CTAs at most.
+void slice_chunks(int T, int S, long long resident, int rows_per_block, int* chunks, int* rows_per_chunk) {
+  long long c = resident / S;
+  if (c < 1) c = 1;
+  const long long max_c = ceil_div(T, rows_per_block);
+  if (c > max_c) c = max_c;
+  long long rpc = ceil_div(ceil_div(T, c), rows_per_block) * rows_per_block;
+  *rows_per_chunk = (int)rpc;
+  *chunks = (int)ceil_div(T, rpc);
 }
 
 template <typename OutT>
 hq_status launch_dequant(const uint32_t* codes, const uint16_t* side, int P, int T, int H, int k,
                          const int32_t* keep_idx, const float* scale, const uint8_t* zero, void* out,
                          cudaStream_t st, const DeviceInfo& d) {
-  const int G = hq::dq_groups_for(P);
-  const int RL = hq::kDqThreads / G;
-  const int S = (H / 8 + G - 1) / G;
-  const int NB = (int)ceil_div(T, (long long)RL * hq::kDqRows);
-  const size_t smem = ((size_t)P * G * 16 + (size_t)RL * hq::kDqRows * hq::kDqKeptChunk) * sizeof(float);
+  const int S = (H + 8 * hq::kDqSliceGroups - 1) / (8 * hq::kDqSliceGroups);
+  const size_t smem = hq::dq_smem_bytes(P);
   auto kern = hq::dequant_reduce_kernel<OutT>;
-  if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return HQ_ERR_CUDA;
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, hq::kDqThreads, smem) != cudaSuccess)
     return HQ_ERR_CUDA;
   if (per_sm < 1) per_sm = 1;
-  unsigned grid;
-  long long per;
-  split_units((long long)S * NB, (long long)d.sms * per_sm, &grid, &per);
-  kern<<<grid, hq::kDqThreads, smem, st>>>(codes, side, P, T, H, k, keep_idx, scale, zero,
-                                            static_cast<OutT*>(out), G, S, NB, per);
+  int chunks, rpc;
+  slice_chunks(T, S, (long long)d.sms * per_sm, hq::kDqR, &chunks, &rpc);
+  kern<<<(unsigned)(S * chunks), hq::kDqThreads, smem, st>>>(codes, side, P, T, H, k, keep_idx, scale,
+                                                              zero, static_cast<OutT*>(out), S, chunks, rpc);
   return launched();
 }
 
@@ -97,19 +98,19 @@ template <typename OutT>
 hq_status launch_fused(const uint16_t* x, int P, int T, int H, int k, const int32_t* keep_idx,
                        const float* scale, const float* inv_scale, const uint8_t* zero, void* out,
                        cudaStream_t st, const DeviceInfo& d) {
-  const int RL = hq::kFuThreads / hq::kFuGroups;
-  const int S = (H / 8 + hq::kFuGroups - 1) / hq::kFuGroups;
-  const int NB = (int)ceil_div(T, (long long)RL * hq::kFuRows);
+  const int S = (H + 8 * hq::kFuSliceGroups - 1) / (8 * hq::kFuSliceGroups);
+  const size_t smem = hq::fu_smem_bytes(P);
   auto kern = hq::compress_reduce_kernel<OutT>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return HQ_ERR_CUDA;
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, hq::kFuThreads, 0) != cudaSuccess)
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, hq::kFuThreads, smem) != cudaSuccess)
     return HQ_ERR_CUDA;
   if (per_sm < 1) per_sm = 1;
-  unsigned grid;
-  long long per;
-  split_units((long long)S * NB, (long long)d.sms * per_sm, &grid, &per);
-  kern<<<grid, hq::kFuThreads, 0, st>>>(x, P, T, H, k, keep_idx, scale, inv_scale, zero,
-                                         static_cast<OutT*>(out), S, NB, per);
+  int chunks, rpc;
+  slice_chunks(T, S, (long long)d.sms * per_sm, hq::kFuR, &chunks, &rpc);
+  kern<<<(unsigned)(S * chunks), hq::kFuThreads, smem, st>>>(x, P, T, H, k, keep_idx, scale, inv_scale,
+                                                              zero, static_cast<OutT*>(out), S, chunks, rpc);
   return launched();
 }
 
@@ -169,14 +170,14 @@ hq_status hq_quantize_pack(const uint16_t* x, int P, int T, int H, int k, const 
   if (T == 0) return HQ_OK;
   DeviceInfo* d = nullptr;
   if (device_info(&d) != HQ_OK) return HQ_ERR_CUDA;
-  const int S = (H / 8 + hq::kQpGroups - 1) / hq::kQpGroups;
+  const int S = (H + 8 * hq::kQpSliceGroups - 1) / (8 * hq::kQpSliceGroups);
   const long long units = (long long)P * S * T;
-  unsigned grid;
-  long long per;
-  split_units(ceil_div(units, hq::kQpRows), (long long)d->sms * d->qp_blocks, &grid, &per);
-  per *= hq::kQpRows;
-  grid = (unsigned)ceil_div(units, per);
-  hq::quantize_pack_kernel<<<grid, hq::kQpThreads, 0, (cudaStream_t)stream>>>(
+  // one warp per resident warp slot, at least kQpR rows each
+  long long warps = (long long)d->sms * d->qp_blocks * hq::kQpWarps;
+  long long per = ceil_div(units, warps);
+  if (per < hq::kQpR) per = hq::kQpR;
+  const unsigned grid = (unsigned)ceil_div(ceil_div(units, per), hq::kQpWarps);
+  hq::quantize_pack_kernel<<<grid, hq::kQpThreads, hq::kQpWarps * sizeof(hq::QpWarpSmem), (cudaStream_t)stream>>>(
       x, P, T, H, k, keep_idx, rest_idx, inv_scale, zero, codes, side, S, per);
   return launched();
 }

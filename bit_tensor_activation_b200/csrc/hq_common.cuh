@@ -49,6 +49,23 @@ __device__ __forceinline__ uint4 ld_stream16(const void* p) {
   return v;
 }
 
+// cp.async copies global -> shared (completion tracked per thread with commit/wait groups;
+// cp.async.wait_group is a hardware wait, no spin loop).
+__device__ __forceinline__ void cp_async4(uint32_t smem_addr, const void* gptr) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr), "l"(gptr) : "memory");
+}
+__device__ __forceinline__ void cp_async16(uint32_t smem_addr, const void* gptr) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr), "l"(gptr) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
 // Number of entries of the ascending array a[0..n) that are < key (lower bound).
 __device__ __forceinline__ int lower_bound_i32(const int32_t* __restrict__ a, int n, int key) {
   int lo = 0, hi = n;

@@ -4,42 +4,45 @@
 // in rank order, acc = fma(float(q_r - zero_r), scale_r, acc) for 4-bit features and
 // acc = acc + side_r for kept ones.
 //
-// Work decomposition.  A CTA covers a slice of G groups of 8 consecutive output features
-// (G = 64 for P <= 8, fewer for more ranks so that the constants below fit) and RL = 256/G row
-// lanes; each thread owns one group and R rows of a row block, and keeps R x 8 fp32 sums in
-// registers while it walks the ranks in order.  Work units are (slice, row block), slice-major,
-// split into one contiguous run per CTA of a persistent grid.
+// Work decomposition.  A warp owns a slice of 32 groups of 8 consecutive output features (256
+// features, one group per lane) and a block of kDqR rows at a time; the 8 warps of a CTA share
+// one slice (so they share its per-(rank, feature) constants in shared memory) and split the
+// CTA's row range between them.  Nothing in the main loop synchronises more than one warp.
+//
+// Data movement.  For every (row block, rank) the warp stages the code words its 32 groups need
+// -- at most 35 consecutive words per row -- into shared memory with 4-byte cp.async copies,
+// kDqD tiles ahead of the tile it consumes (an 8-deep pipeline per warp, ~0.6 KB per tile), so
+// the latency of HBM is covered without holding the data in registers.  cp.async.wait_group is a
+// hardware wait: there is no spin loop.
 //
 // Codes of a group: its n non-kept features occupy compact positions c0..c0+n-1, i.e. at most
 // two consecutive words; a funnel shift brings them to bits 0..4n-1 of v, and feature i of the
-// group reads nibble j_i (its rank among the non-kept ones).  The nibble is turned into a float
-// without a conversion instruction: (nibble | 0x4B000000) is the float 2^23 + q, and adding the
-// constant -(2^23 + zero) gives q - zero exactly.  Per (rank, feature) the kernel needs scale
-// and that offset; they are written to shared memory once per slice (a kept feature gets scale 0
-// and offset -2^23, which leaves its sum untouched).
+// group reads nibble j_i (its rank among the group's non-kept features).  The nibble becomes a
+// float without a conversion instruction: (nibble | 0x4B000000) is the float 2^23 + q, and
+// adding the per-(rank, feature) constant -(2^23 + zero) gives q - zero exactly.  A kept feature
+// gets scale 0 and offset -2^23, which leaves its sum untouched; its sum over the side values is
+// computed by "kept lanes" and written into the owner's registers through a small warp buffer.
 //
-// Kept features are summed separately: "kept lanes" (one per (row, kept feature) pair of the
-// block) add the P side values in rank order into a small shared buffer, and the owning threads
-// take them from there before the bf16 (or fp32) output row is stored with 16-byte stores.
-//
-// Roofline: HBM-bound; per output element ~P*(H'/H*0.5 + k/H*2) bytes read + 2 (or 4) written.
-// No scratch memory.
+// Roofline: HBM-bound; per output element P*(0.5*H'/H + 2*k/H) bytes read + 2 (or 4) written.
+// No memory beyond the inputs and outputs is used.
 #pragma once
 
 #include "hq_common.cuh"
 
 namespace hq {
 
-constexpr int kDqThreads = 256;
-constexpr int kDqRows = 4;          // rows per thread per block
-constexpr int kDqKeptChunk = 64;    // kept features per pass of the kept lanes
-constexpr int kDqMaxG = 64;
+constexpr int kDqWarps = 8;
+constexpr int kDqThreads = 32 * kDqWarps;
+constexpr int kDqR = 4;       // rows per block
+constexpr int kDqD = 8;       // cp.async tiles in flight per warp
+constexpr int kDqWin = 36;    // staged words per row (>= 35)
+constexpr int kDqSliceGroups = 32;
 
-// Groups per slice for P ranks: the constants take P * G * 64 bytes (<= 32 KB).
-inline int dq_groups_for(int P) {
-  int g = kDqMaxG;
-  while (g > 8 && P * g * 64 > 32 * 1024) g >>= 1;
-  return g;
+// Dynamic shared memory of one CTA for P ranks.
+inline size_t dq_smem_bytes(int P) {
+  return (size_t)P * 4 * 32 * 16                            // constants: [P][4][32] float4
+         + (size_t)kDqWarps * kDqD * kDqR * kDqWin * 4      // staged code tiles
+         + (size_t)kDqWarps * kDqR * 32 * 4;                // kept sums
 }
 
 template <typename OutT>
@@ -72,112 +75,122 @@ template <typename OutT>
 __global__ void __launch_bounds__(kDqThreads) dequant_reduce_kernel(
     const uint32_t* __restrict__ codes, const uint16_t* __restrict__ side, int P, int T, int H,
     int k, const int32_t* __restrict__ keep_idx, const float* __restrict__ scale,
-    const uint8_t* __restrict__ zero, OutT* __restrict__ out, int G, int S, int NB,
-    long long units_per_cta) {
+    const uint8_t* __restrict__ zero, OutT* __restrict__ out, int S, int chunks, int rows_per_chunk) {
   extern __shared__ float4 s_dyn[];
-  float* s_const = reinterpret_cast<float*>(s_dyn);         // [P][G][16]: scale x8, offset x8
-  float* s_kept = s_const + (size_t)P * G * 16;             // [RL*R][kDqKeptChunk]
+  float4* s_const = s_dyn;                                                    // [P][4][32]
+  uint32_t* s_tiles = reinterpret_cast<uint32_t*>(s_const + (size_t)P * 4 * 32);
+  float* s_kept = reinterpret_cast<float*>(s_tiles + kDqWarps * kDqD * kDqR * kDqWin);
 
-  const int tid = threadIdx.x;
-  const int RL = kDqThreads / G;
-  const int gi = tid % G, lane_row = tid / G;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int Hr = H - k, Wr = Hr / 8;
-  const int rows_per_block = RL * kDqRows;
-  const long long U = (long long)S * NB;
+  const int s = blockIdx.x / chunks, chunk = blockIdx.x - s * chunks;
+  const int t_first = chunk * rows_per_chunk, t_last = min(T, t_first + rows_per_chunk);
 
-  long long u = (long long)blockIdx.x * units_per_cta;
-  const long long u_end = min(U, u + units_per_cta);
-  int cur_slice = -1;
-
-  // per-thread static layout of its group in the current slice
-  int h0 = 0, c0 = 0, n = 0, j0 = 0;
-  uint32_t kmask = 0;
+  // ---- this lane's group: layout and nibble positions ----------------------------------------
+  const int h0 = 8 * (s * kDqSliceGroups + lane);
+  const bool active = h0 < H;
+  GroupLayout L{0, 0, 0u, 0};
+  if (active) L = group_layout(keep_idx, k, H, h0);
   int nib_shift[8];
+  {
+    int j = 0;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) nib_shift[i] = 0;
-  bool active = false;
-  int ja = 0, jb = 0;
-
-  for (; u < u_end; ++u) {
-    const int s = (int)(u / NB);
-    const int b = (int)(u - (long long)s * NB);
-
-    if (s != cur_slice) {
-      __syncthreads();  // previous users of s_const are done
-      cur_slice = s;
-      const int g = s * G + gi;
-      h0 = 8 * g;
-      active = h0 < H;
-      if (active) {
-        const GroupLayout L = group_layout(keep_idx, k, H, h0);
-        c0 = L.c0;
-        n = L.n;
-        j0 = L.j0;
-        kmask = L.kmask;
-        int j = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const bool kept = (kmask >> i) & 1u;
-          nib_shift[i] = kept ? 0 : 4 * j;
-          j += kept ? 0 : 1;
-        }
-      } else {
-        c0 = n = j0 = 0;
-        kmask = 0;
-      }
-      const int ha = s * G * 8, hb = min(H, ha + G * 8);
-      ja = lower_bound_i32(keep_idx, k, ha);
-      jb = lower_bound_i32(keep_idx, k, hb);
-      if (tid == 0 && ((s == 0 && ja != 0) || (s == S - 1 && jb != k))) record_error(HQ_ERR_BAD_INDEX);
-      // constants of the slice: threads of row lane 0 fill their own group for all ranks
-      if (lane_row == 0) {
-        for (int r = 0; r < P; ++r) {
-          float* dst = s_const + ((size_t)r * G + gi) * 16;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            float sc = 0.0f, off = -8388608.0f;  // kept / inactive: contributes fma(q, 0, acc)
-            if (active && !((kmask >> i) & 1u)) {
-              const size_t p = (size_t)r * H + h0 + i;
-              sc = scale[p];
-              off = -__int_as_float(0x4B000000 | (int)zero[p]);  // -(2^23 + zero)
-            }
-            dst[i] = sc;
-            dst[8 + i] = off;
-          }
-        }
-      }
-      __syncthreads();
+    for (int i = 0; i < 8; ++i) {
+      const bool kept = (L.kmask >> i) & 1u;
+      nib_shift[i] = kept ? 0 : 4 * j;
+      j += kept ? 0 : 1;
     }
+  }
+  // words the warp stages per row: [w_first, w_end), at most 35
+  const int hs = 8 * s * kDqSliceGroups, he = min(H, hs + 8 * kDqSliceGroups);
+  const int ja = lower_bound_i32(keep_idx, k, hs), jb = lower_bound_i32(keep_idx, k, he);
+  if (threadIdx.x == 0 && ((s == 0 && ja != 0) || (s == S - 1 && jb != k))) record_error(HQ_ERR_BAD_INDEX);
+  const int Ca = min(max(hs - ja, 0), Hr), Cb = min(max(he - jb, 0), Hr);
+  const int w_first = Ca >> 3;
+  const int n_words = max(0, min(Wr, (Cb >> 3) + 2) - w_first);
+  const int my_w = (L.c0 >> 3) - w_first;  // this lane's first word inside the window
+  const int fsh = 4 * (L.c0 & 7);
+  const bool has_hi = (L.c0 >> 3) + 1 < Wr;
 
-    const int t_blk = b * rows_per_block;
-    float acc[kDqRows][8];
+  // ---- constants of the slice for all ranks (conflict-free [P][4][32] float4 layout) ---------
+  for (int idx = threadIdx.x; idx < P * 32; idx += kDqThreads) {
+    const int r = idx >> 5, g = idx & 31;
+    const int hg = 8 * (s * kDqSliceGroups + g);
+    float sc[8], off[8];
+    uint32_t km = 0;
+    if (hg < H) km = group_layout(keep_idx, k, H, hg).kmask;
 #pragma unroll
-    for (int m = 0; m < kDqRows; ++m)
+    for (int i = 0; i < 8; ++i) {
+      sc[i] = 0.0f;
+      off[i] = -8388608.0f;
+      if (hg < H && !((km >> i) & 1u)) {
+        const size_t p = (size_t)r * H + hg + i;
+        sc[i] = scale[p];
+        off[i] = -__int_as_float(0x4B000000 | (int)zero[p]);  // -(2^23 + zero)
+      }
+    }
+    float4* dst = s_const + (size_t)r * 4 * 32 + g;
+    dst[0] = make_float4(sc[0], sc[1], sc[2], sc[3]);
+    dst[32] = make_float4(sc[4], sc[5], sc[6], sc[7]);
+    dst[64] = make_float4(off[0], off[1], off[2], off[3]);
+    dst[96] = make_float4(off[4], off[5], off[6], off[7]);
+  }
+  __syncthreads();
+
+  // ---- this warp's row blocks: rows t_first + (warp + kDqWarps*bi)*kDqR + m ------------------
+  const int nblk_total = (t_last - t_first + kDqR - 1) / kDqR;
+  const int my_blocks = nblk_total > warp ? (nblk_total - warp + kDqWarps - 1) / kDqWarps : 0;
+  const int n_tiles = my_blocks * P;  // tile i = (block i / P, rank i % P)
+  uint32_t* my_tiles = s_tiles + (size_t)warp * kDqD * kDqR * kDqWin;
+  float* my_kept = s_kept + warp * kDqR * 32;
+  const uint32_t tiles_saddr = smem_addr(my_tiles);
+
+  auto block_row0 = [&](int bi) { return t_first + (warp + kDqWarps * bi) * kDqR; };
+  auto issue_tile = [&](int i) {
+    if (i < n_tiles) {
+      const int bi = i / P, r = i - bi * P;
+      const int t0 = block_row0(bi);
+      const int stage = i % kDqD;
+#pragma unroll
+      for (int m = 0; m < kDqR; ++m) {
+        const int t = t0 + m;
+        if (t < t_last) {
+          const uint32_t* src = codes + ((size_t)r * T + t) * Wr + w_first;
+          const uint32_t dst = tiles_saddr + (uint32_t)(((stage * kDqR + m) * kDqWin) * 4);
+          for (int w = lane; w < n_words; w += 32) cp_async4(dst + 4u * w, src + w);
+        }
+      }
+    }
+    cp_async_commit();  // one group per tile, empty ones included, keeps the count uniform
+  };
+
+  for (int i = 0; i < kDqD - 1; ++i) issue_tile(i);
+
+  const int nk = jb - ja;
+  int tile = 0;
+  for (int bi = 0; bi < my_blocks; ++bi) {
+    const int t0 = block_row0(bi);
+    float acc[kDqR][8];
+#pragma unroll
+    for (int m = 0; m < kDqR; ++m)
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[m][i] = 0.0f;
 
-    const int w0 = c0 >> 3, fsh = 4 * (c0 & 7);
-    const bool has_hi = (w0 + 1) < Wr;
-    if (active && n > 0) {
-      for (int r = 0; r < P; ++r) {
-        const float4* cst = reinterpret_cast<const float4*>(s_const + ((size_t)r * G + gi) * 16);
-        const float4 s0 = cst[0], s1 = cst[1], o0 = cst[2], o1 = cst[3];
-        const float sc[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-        const float off[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
-        uint32_t wlo[kDqRows], whi[kDqRows];
+    for (int r = 0; r < P; ++r, ++tile) {
+      issue_tile(tile + kDqD - 1);
+      cp_async_wait<kDqD - 1>();
+      __syncwarp();
+      const uint32_t* st = my_tiles + (size_t)(tile % kDqD) * kDqR * kDqWin;
+      const float4* cst = s_const + (size_t)r * 4 * 32 + lane;
+      const float4 s0 = cst[0], s1 = cst[32], o0 = cst[64], o1 = cst[96];
+      const float sc[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+      const float off[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+      if (active && L.n > 0) {
 #pragma unroll
-        for (int m = 0; m < kDqRows; ++m) {
-          const int t = t_blk + lane_row + m * RL;
-          wlo[m] = whi[m] = 0u;
-          if (t < T) {
-            const uint32_t* row = codes + ((size_t)r * T + t) * Wr;
-            wlo[m] = __ldg(row + w0);
-            if (has_hi) whi[m] = __ldg(row + w0 + 1);
-          }
-        }
-#pragma unroll
-        for (int m = 0; m < kDqRows; ++m) {
-          const uint32_t v = __funnelshift_r(wlo[m], whi[m], fsh);
+        for (int m = 0; m < kDqR; ++m) {
+          const uint32_t wlo = st[m * kDqWin + my_w];
+          const uint32_t whi = has_hi ? st[m * kDqWin + my_w + 1] : 0u;
+          const uint32_t v = __funnelshift_r(wlo, whi, fsh);
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const uint32_t bits = ((v >> nib_shift[i]) & 0xFu) | 0x4B000000u;
@@ -186,50 +199,51 @@ __global__ void __launch_bounds__(kDqThreads) dequant_reduce_kernel(
           }
         }
       }
+      __syncwarp();  // the stage is free for the copy issued next iteration
     }
 
-    // ---- kept features of the slice, in chunks -------------------------------------------
-    const int nk = jb - ja;
-    for (int kc = 0; kc < nk; kc += kDqKeptChunk) {
-      const int kw = min(kDqKeptChunk, nk - kc);
-      const int pairs = rows_per_block * kw;
-      for (int p = tid; p < pairs; p += kDqThreads) {
-        const int row = p / kw, jj = p - row * kw;
-        const int t = t_blk + row;
+    // ---- kept features of the warp's slice: (row, kept feature) pairs over the lanes ---------
+    for (int kc = 0; kc < nk; kc += 32) {
+      const int kw = min(32, nk - kc);
+      for (int p = lane; p < kDqR * kw; p += 32) {
+        const int m = p / kw, jj = p - m * kw;
+        const int t = t0 + m;
         float a = 0.0f;
-        if (t < T) {
-          const int j = ja + kc + jj;
-          for (int r = 0; r < P; ++r)
-            a = __fadd_rn(a, __uint_as_float((uint32_t)__ldg(side + ((size_t)r * T + t) * k + j) << 16));
+        if (t < t_last) {
+          const uint16_t* sp = side + (size_t)t * k + ja + kc + jj;
+          const size_t rank_stride = (size_t)T * k;
+#pragma unroll 8
+          for (int r = 0; r < P; ++r) a = __fadd_rn(a, __uint_as_float((uint32_t)__ldg(sp + r * rank_stride) << 16));
         }
-        s_kept[row * kDqKeptChunk + jj] = a;
+        my_kept[m * 32 + jj] = a;
       }
-      __syncthreads();
-      if (kmask) {
-        int jk = j0;  // keep_idx position of the group's next kept feature
+      __syncwarp();
+      if (L.kmask) {
+        int jk = L.j0;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          if ((kmask >> i) & 1u) {
+          if ((L.kmask >> i) & 1u) {
             const int jj = jk - ja - kc;
             if (jj >= 0 && jj < kw) {
 #pragma unroll
-              for (int m = 0; m < kDqRows; ++m) acc[m][i] = s_kept[(lane_row + m * RL) * kDqKeptChunk + jj];
+              for (int m = 0; m < kDqR; ++m) acc[m][i] = my_kept[m * 32 + jj];
             }
             ++jk;
           }
         }
       }
-      __syncthreads();
+      __syncwarp();
     }
 
     if (active) {
 #pragma unroll
-      for (int m = 0; m < kDqRows; ++m) {
-        const int t = t_blk + lane_row + m * RL;
-        if (t < T) store_row8<OutT>(out + (size_t)t * H + h0, acc[m]);
+      for (int m = 0; m < kDqR; ++m) {
+        const int t = t0 + m;
+        if (t < t_last) store_row8<OutT>(out + (size_t)t * H + h0, acc[m]);
       }
     }
   }
+  cp_async_wait<0>();
 }
 
 }  // namespace hq
