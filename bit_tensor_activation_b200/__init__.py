@@ -40,6 +40,8 @@ for _f in ("hq_calibrate", "hq_select_topk", "hq_quantize_pack", "hq_dequant_red
 _lib.hq_read_device_error.argtypes = [_vp]
 _lib.hq_status_string.argtypes = [_i32]
 _lib.hq_status_string.restype = ctypes.c_char_p
+_lib.hq_selftest_bounded_wait.argtypes = [ctypes.c_longlong, _vp]
+_lib.hq_selftest_bounded_wait.restype = _i32
 _lib.hq_wire_bytes_per_row.argtypes = [_i32, _i32]
 _lib.hq_wire_bytes_per_row.restype = ctypes.c_int64
 
@@ -47,7 +49,8 @@ HQ_OK, HQ_ERR_INVALID_ARG, HQ_ERR_MISALIGNED, HQ_ERR_CUDA, HQ_ERR_TIMEOUT, HQ_ER
 HQ_OUT_BF16, HQ_OUT_F32 = 0, 1
 
 EXPORTS = ["hq_calibrate", "hq_select_topk", "hq_quantize_pack", "hq_dequant_reduce",
-           "hq_compress_reduce", "hq_status_string", "hq_read_device_error", "hq_wire_bytes_per_row"]
+           "hq_compress_reduce", "hq_status_string", "hq_read_device_error", "hq_wire_bytes_per_row",
+           "hq_selftest_bounded_wait"]
 
 
 class HQError(RuntimeError):
@@ -156,6 +159,12 @@ def hq_compress_reduce(x, keep_idx, rest_idx, scale, inv_scale, zero, out, codes
             _ptr(codes, _CODES, (P, T, (H - k) // 8), "codes"), _ptr(side, _BF16, (P, T, k), "side"),
             _stream(stream, x.device))
     _check(_lib.hq_compress_reduce(*args), "hq_compress_reduce")
+
+
+def hq_selftest_bounded_wait(limit_cycles: int, stream=None, device=None) -> None:
+    """Launches a wait that nothing satisfies; it gives up after limit_cycles and records
+    HQ_ERR_TIMEOUT (read it with hq_read_device_error)."""
+    _check(_lib.hq_selftest_bounded_wait(int(limit_cycles), _stream(stream, device)), "hq_selftest_bounded_wait")
 
 
 def hq_read_device_error(stream=None, device=None) -> int:

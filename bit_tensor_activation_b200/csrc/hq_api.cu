@@ -4,16 +4,20 @@
 // entry point checks its arguments on the host, picks a launch shape, enqueues one kernel on the
 // caller's stream and returns; nothing is allocated and nothing waits, except
 // hq_read_device_error, which synchronises the stream it is given.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
 
 #include "hq.h"
 #include "hq_common.cuh"
+#include "hq_tma.cuh"
 #include "k_calibrate.cuh"
 #include "k_dequant.cuh"
 #include "k_fused.cuh"
 #include "k_quantize.cuh"
+#include "k_quantize_tma.cuh"
 #include "k_select.cuh"
 
 namespace {
@@ -34,8 +38,39 @@ hq_status check_shape(int P, int H, int k) {
 struct DeviceInfo {
   int sms = 0;
   int qp_blocks = 0;
+  int qt_blocks = 0;
   bool select_smem_set = false;
 };
+
+// cuTensorMapEncodeTiled, fetched once through the runtime (no link-time libcuda dependency).
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::mutex g_encode_mu;
+
+bool get_encode() {
+  std::lock_guard<std::mutex> lock(g_encode_mu);
+  if (g_encode) return true;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || fn == nullptr)
+    return false;
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return true;
+}
+
+// Row-major 2-D tensor [rows][cols] of `elem`-byte elements (row pitch cols*elem bytes, a
+// multiple of 16) read in boxes of box_rows x box_cols; out-of-range box elements read as 0.
+bool encode_2d(CUtensorMap* map, const void* base, CUtensorMapDataType type, size_t elem, uint64_t cols,
+               uint64_t rows, uint32_t box_cols, uint32_t box_rows,
+               CUtensorMapL2promotion promo = CU_TENSOR_MAP_L2_PROMOTION_L2_256B) {
+  if (!get_encode()) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * elem};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return g_encode(map, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
 
@@ -54,6 +89,13 @@ hq_status device_info(DeviceInfo** out) {
                                                       hq::kQpThreads, qp_smem) != cudaSuccess)
       return HQ_ERR_CUDA;
     if (d.qp_blocks < 1) d.qp_blocks = 1;
+    const int qt_smem = (int)(sizeof(hq::QtSmem) + 128);
+    if (cudaFuncSetAttribute(hq::quantize_pack_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             qt_smem) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.qt_blocks, hq::quantize_pack_tma_kernel,
+                                                      hq::kQtThreads, qt_smem) != cudaSuccess)
+      return HQ_ERR_CUDA;
+    if (d.qt_blocks < 1) d.qt_blocks = 1;
   }
   *out = &d;
   return HQ_OK;
@@ -79,6 +121,31 @@ hq_status launch_dequant(const uint32_t* codes, const uint16_t* side, int P, int
                          const int32_t* keep_idx, const float* scale, const uint8_t* zero, void* out,
                          cudaStream_t st, const DeviceInfo& d) {
   const int S = (H + 8 * hq::kDqSliceGroups - 1) / (8 * hq::kDqSliceGroups);
+  const int Wr = (H - k) / 8;
+  CUtensorMap map, map_side;
+  const bool tma = Wr >= 4 && Wr % 4 == 0 && aligned(codes, 16) &&
+                   encode_2d(&map, codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)Wr, (uint64_t)P * T,
+                             hq::kDtWords, hq::kDtTileRows) &&
+                   (k == 0 || encode_2d(&map_side, side, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)k,
+                                        (uint64_t)P * T, hq::kDtSideCols, hq::kDtTileRows,
+                                        CU_TENSOR_MAP_L2_PROMOTION_NONE));
+  if (k == 0) map_side = map;  // never read: no slice stages side values when k == 0
+  if (tma) {
+    const size_t smem = hq::dt_smem_bytes(P);
+    auto kern = hq::dequant_reduce_tma_kernel<OutT>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return HQ_ERR_CUDA;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, hq::kDtThreads, smem) != cudaSuccess)
+      return HQ_ERR_CUDA;
+    if (per_sm < 1) per_sm = 1;
+    int chunks, rpc;
+    slice_chunks(T, S, (long long)d.sms * per_sm, hq::kDtTileRows, &chunks, &rpc);
+    kern<<<(unsigned)(S * chunks), hq::kDtThreads, smem, st>>>(map, map_side, side, P, T, H, k, keep_idx, scale, zero,
+                                                                static_cast<OutT*>(out), S, chunks, rpc,
+                                                                hq::kWaitLimitCycles);
+    return launched();
+  }
   const size_t smem = hq::dq_smem_bytes(P);
   auto kern = hq::dequant_reduce_kernel<OutT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
@@ -98,7 +165,11 @@ template <typename OutT>
 hq_status launch_fused(const uint16_t* x, int P, int T, int H, int k, const int32_t* keep_idx,
                        const float* scale, const float* inv_scale, const uint8_t* zero, void* out,
                        cudaStream_t st, const DeviceInfo& d) {
-  const int S = (H + 8 * hq::kFuSliceGroups - 1) / (8 * hq::kFuSliceGroups);
+  const int S = (H + hq::kFuSlice - 1) / hq::kFuSlice;
+  CUtensorMap map;
+  if (!encode_2d(&map, x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)H, (uint64_t)P * T, hq::kFuSlice,
+                 hq::kFuTileRows))
+    return HQ_ERR_CUDA;
   const size_t smem = hq::fu_smem_bytes(P);
   auto kern = hq::compress_reduce_kernel<OutT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
@@ -108,10 +179,21 @@ hq_status launch_fused(const uint16_t* x, int P, int T, int H, int k, const int3
     return HQ_ERR_CUDA;
   if (per_sm < 1) per_sm = 1;
   int chunks, rpc;
-  slice_chunks(T, S, (long long)d.sms * per_sm, hq::kFuR, &chunks, &rpc);
-  kern<<<(unsigned)(S * chunks), hq::kFuThreads, smem, st>>>(x, P, T, H, k, keep_idx, scale, inv_scale,
-                                                              zero, static_cast<OutT*>(out), S, chunks, rpc);
+  slice_chunks(T, S, (long long)d.sms * per_sm, hq::kFuTileRows, &chunks, &rpc);
+  kern<<<(unsigned)(S * chunks), hq::kFuThreads, smem, st>>>(map, P, T, H, k, keep_idx, scale, inv_scale, zero,
+                                                              static_cast<OutT*>(out), S, chunks, rpc,
+                                                              hq::kWaitLimitCycles);
   return launched();
+}
+
+// Bounded-wait self-test: one thread waits on an mbarrier that nothing arrives on.
+__global__ void selftest_wait_kernel(long long limit) {
+  __shared__ uint64_t bar;
+  __shared__ int abort;
+  hq::mbar_init(&bar, 1);
+  abort = 0;
+  hq::fence_barrier_init();
+  hq::mbar_wait(&bar, 0, &abort, limit);
 }
 
 }  // namespace
@@ -170,6 +252,22 @@ hq_status hq_quantize_pack(const uint16_t* x, int P, int T, int H, int k, const 
   if (T == 0) return HQ_OK;
   DeviceInfo* d = nullptr;
   if (device_info(&d) != HQ_OK) return HQ_ERR_CUDA;
+  {
+    const int S = (H + hq::kQtSlice - 1) / hq::kQtSlice;
+    CUtensorMap map_x, map_halo;
+    if (!encode_2d(&map_x, x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)H, (uint64_t)P * T, hq::kQtSlice,
+                   hq::kQtTileRows) ||
+        !encode_2d(&map_halo, x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)H, (uint64_t)P * T, hq::kQtHalo,
+                   hq::kQtTileRows, CU_TENSOR_MAP_L2_PROMOTION_NONE))  // 32-byte rows: no 256-byte over-fetch
+      return HQ_ERR_CUDA;
+    int chunks, rpc;
+    slice_chunks(T, S, (long long)d->sms * d->qt_blocks, hq::kQtTileRows, &chunks, &rpc);
+    hq::quantize_pack_tma_kernel<<<(unsigned)(S * chunks), hq::kQtThreads, sizeof(hq::QtSmem) + 128,
+                                   (cudaStream_t)stream>>>(map_x, map_halo, x, P, T, H, k, keep_idx, rest_idx,
+                                                           inv_scale, zero, codes, side, S, chunks, rpc,
+                                                           hq::kWaitLimitCycles);
+    return launched();
+  }
   const int S = (H + 8 * hq::kQpSliceGroups - 1) / (8 * hq::kQpSliceGroups);
   const long long units = (long long)P * S * T;
   // one warp per resident warp slot, at least kQpR rows each
@@ -254,6 +352,12 @@ hq_status hq_read_device_error(void* stream) {
     return HQ_ERR_CUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess) return HQ_ERR_CUDA;
   return (hq_status)v;
+}
+
+hq_status hq_selftest_bounded_wait(long long limit_cycles, void* stream) {
+  if (limit_cycles < 0) return HQ_ERR_INVALID_ARG;
+  selftest_wait_kernel<<<1, 1, 0, (cudaStream_t)stream>>>(limit_cycles);
+  return launched();
 }
 
 int64_t hq_wire_bytes_per_row(int H, int k) {

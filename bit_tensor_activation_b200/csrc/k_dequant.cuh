@@ -4,46 +4,40 @@
 // in rank order, acc = fma(float(q_r - zero_r), scale_r, acc) for 4-bit features and
 // acc = acc + side_r for kept ones.
 //
-// Work decomposition.  A warp owns a slice of 32 groups of 8 consecutive output features (256
-// features, one group per lane) and a block of kDqR rows at a time; the 8 warps of a CTA share
-// one slice (so they share its per-(rank, feature) constants in shared memory) and split the
-// CTA's row range between them.  Nothing in the main loop synchronises more than one warp.
+// Work decomposition (both kernels below).  A CTA covers a slice of 32 groups of 8 consecutive
+// output features (256 features) and a range of rows; a warp owns the whole slice (one group per
+// lane) for kDqR rows at a time and keeps kDqR x 8 fp32 sums in registers while it walks the
+// ranks in order.  The CTA's warps share the slice's per-(rank, feature) constants in shared
+// memory.  Two ways of staging the code words:
+//   - dequant_reduce_tma_kernel (default): a producer warp loads, per (32-row block, rank), one
+//     32 x 40-word TMA tile into an 8-stage mbarrier ring; eight consumer warps take 4 rows each.
+//     Needs code rows whose byte length is a multiple of 16 ((H-k) % 32 == 0).
+//   - dequant_reduce_kernel (any shape): each warp stages its own rows with 4-byte cp.async
+//     copies, 8 tiles ahead.
 //
-// Data movement.  For every (row block, rank) the warp stages the code words its 32 groups need
-// -- at most 35 consecutive words per row -- into shared memory with 4-byte cp.async copies,
-// kDqD tiles ahead of the tile it consumes (an 8-deep pipeline per warp, ~0.6 KB per tile), so
-// the latency of HBM is covered without holding the data in registers.  cp.async.wait_group is a
-// hardware wait: there is no spin loop.
-//
-// Codes of a group: its n non-kept features occupy compact positions c0..c0+n-1, i.e. at most
-// two consecutive words; a funnel shift brings them to bits 0..4n-1 of v, and feature i of the
-// group reads nibble j_i (its rank among the group's non-kept features).  The nibble becomes a
-// float without a conversion instruction: (nibble | 0x4B000000) is the float 2^23 + q, and
-// adding the per-(rank, feature) constant -(2^23 + zero) gives q - zero exactly.  A kept feature
-// gets scale 0 and offset -2^23, which leaves its sum untouched; its sum over the side values is
-// computed by "kept lanes" and written into the owner's registers through a small warp buffer.
+// Decoding a group: its n non-kept features occupy compact positions c0..c0+n-1, i.e. at most
+// two consecutive words; a funnel shift brings them to bits 0..4n-1 of v.  Feature i's nibble
+// is turned into a float without a conversion instruction: (v & (0xF << 4p_i)) | 0x4B000000 is
+// the float 2^23 + q*16^p_i; adding the per-(rank, feature) constant -(2^23 + zero*16^p_i)
+// gives (q - zero)*16^p_i exactly, and the FMA uses scale/16^p_i, so the product is exactly
+// (q - zero)*scale.  p_i <= 4 is arranged by reading features 5..7 from a second view
+// v2 = v >> 4b.  Scales below 2^-109 could lose bits when divided by 16^4: a slice that has one
+// decodes with explicit shifts and undivided constants instead ("generic" path).  Adds and FMAs
+// go two at a time through add/fma.rn.f32x2 (per-lane IEEE, so bit-identical).  A kept feature
+// gets scale 0 (its decoded value is then multiplied by 0); its sum over the side values is
+// formed by "kept lanes" and written into the owner's registers through a small warp buffer.
 //
 // Roofline: HBM-bound; per output element P*(0.5*H'/H + 2*k/H) bytes read + 2 (or 4) written.
 // No memory beyond the inputs and outputs is used.
 #pragma once
 
 #include "hq_common.cuh"
+#include "hq_tma.cuh"
 
 namespace hq {
 
-constexpr int kDqWarps = 8;
-constexpr int kDqThreads = 32 * kDqWarps;
-constexpr int kDqR = 4;       // rows per block
-constexpr int kDqD = 8;       // cp.async tiles in flight per warp
-constexpr int kDqWin = 36;    // staged words per row (>= 35)
 constexpr int kDqSliceGroups = 32;
-
-// Dynamic shared memory of one CTA for P ranks.
-inline size_t dq_smem_bytes(int P) {
-  return (size_t)P * 4 * 32 * 16                            // constants: [P][4][32] float4
-         + (size_t)kDqWarps * kDqD * kDqR * kDqWin * 4      // staged code tiles
-         + (size_t)kDqWarps * kDqR * 32 * 4;                // kept sums
-}
+constexpr int kDqR = 4;  // rows per warp per block
 
 template <typename OutT>
 __device__ __forceinline__ void store_row8(OutT* dst, const float* v);
@@ -71,6 +65,371 @@ __device__ __forceinline__ void store_row8<float>(float* dst, const float* v) {
       make_float4(canonical_nan(v[4]), canonical_nan(v[5]), canonical_nan(v[6]), canonical_nan(v[7]));
 }
 
+// Nibble positions of a group with kept mask km: jpos[i] = rank of feature i among the group's
+// non-kept features (its nibble sits at bits 4*jpos[i] of v); pos[i] = in-place position used by
+// the fast path (features 5..7 are read from v2 = v >> 4b); returns b.
+__device__ __forceinline__ int dq_positions(uint32_t km, int* pos, int* jpos) {
+  int j = 0, b = -1;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const bool kept = (km >> i) & 1u;
+    jpos[i] = j;
+    if (i >= 5 && !kept && b < 0) b = j;
+    j += kept ? 0 : 1;
+  }
+  if (b < 0) b = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) pos[i] = (i < 5) ? jpos[i] : jpos[i] - b;
+  return b;
+}
+
+// What one lane needs to decode its group from a staged row of code words.
+struct DqLane {
+  GroupLayout L;
+  int h0;
+  bool active;
+  bool decode;       // active and at least one non-kept feature
+  bool has_hi;       // the group's second word exists
+  int my_w;          // first word of the group inside a staged row
+  int fsh;           // funnel shift bringing the group's first nibble to bit 0
+  int sh2;           // fast path: v2 = v >> sh2
+  uint32_t key[8];   // fast path: in-place nibble mask; generic path: nibble shift
+};
+
+__device__ __forceinline__ DqLane dq_lane(const int32_t* __restrict__ keep_idx, int k, int H, int s, int lane,
+                                          int w_base, bool generic) {
+  DqLane D;
+  D.h0 = 8 * (s * kDqSliceGroups + lane);
+  D.active = D.h0 < H;
+  D.L = GroupLayout{0, 0, 0u, 0};
+  if (D.active) D.L = group_layout(keep_idx, k, H, D.h0);
+  int pos[8], jpos[8];
+  const int b = dq_positions(D.L.kmask, pos, jpos);
+  D.sh2 = 4 * b;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const bool kept = (D.L.kmask >> i) & 1u;
+    D.key[i] = generic ? (uint32_t)(4 * jpos[i]) : (kept ? 0u : (0xFu << (4 * pos[i])));
+  }
+  const int Wr = (H - k) / 8;
+  D.my_w = (D.L.c0 >> 3) - w_base;
+  D.fsh = 4 * (D.L.c0 & 7);
+  D.has_hi = (D.L.c0 >> 3) + 1 < Wr;
+  D.decode = D.active && D.L.n > 0;
+  return D;
+}
+
+// Whether this thread's share of slice s has a scale below 2^-109 (the slice then needs the
+// generic path); `nthreads` threads split the slice.
+__device__ __forceinline__ bool dq_has_tiny_scale(const float* __restrict__ scale, int P, int H, int s,
+                                                  int nthreads) {
+  const int hs = 8 * s * kDqSliceGroups;
+  bool tiny = false;
+  for (int idx = threadIdx.x; idx < P * 8 * kDqSliceGroups; idx += nthreads) {
+    const int r = idx / (8 * kDqSliceGroups), h = hs + idx % (8 * kDqSliceGroups);
+    if (h < H && scale[(size_t)r * H + h] < 0x1p-109f) tiny = true;
+  }
+  return tiny;
+}
+
+// Per-(rank, group) constants of slice s in a conflict-free [P][4][32] float4 layout:
+// scale/16^p x8, -(2^23 + zero*16^p) x8 (p = 0 on the generic path).
+__device__ __forceinline__ void dq_fill_constants(float4* s_const, const int32_t* __restrict__ keep_idx,
+                                                  const float* __restrict__ scale,
+                                                  const uint8_t* __restrict__ zero, int P, int H, int k,
+                                                  int s, bool generic, int nthreads) {
+  for (int idx = threadIdx.x; idx < P * 32; idx += nthreads) {
+    const int r = idx >> 5, g = idx & 31;
+    const int hg = 8 * (s * kDqSliceGroups + g);
+    float sc[8], off[8];
+    uint32_t km = 0;
+    if (hg < H) km = group_layout(keep_idx, k, H, hg).kmask;
+    int pos[8], jpos[8];
+    dq_positions(km, pos, jpos);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      sc[i] = 0.0f;
+      off[i] = -8388608.0f;  // kept / inactive: decodes to a small value times scale 0
+      if (hg < H && !((km >> i) & 1u)) {
+        const size_t p = (size_t)r * H + hg + i;
+        const int e = generic ? 0 : 4 * pos[i];
+        sc[i] = __fmul_rn(scale[p], __int_as_float((127 - e) << 23));  // scale / 16^p, exact
+        off[i] = -__int_as_float(0x4B000000 | ((int)zero[p] << e));     // -(2^23 + zero*16^p)
+      }
+    }
+    float4* dst = s_const + (size_t)r * 4 * 32 + g;
+    dst[0] = make_float4(sc[0], sc[1], sc[2], sc[3]);
+    dst[32] = make_float4(sc[4], sc[5], sc[6], sc[7]);
+    dst[64] = make_float4(off[0], off[1], off[2], off[3]);
+    dst[96] = make_float4(off[4], off[5], off[6], off[7]);
+  }
+}
+
+// Adds one rank's contribution for kDqR staged rows (row m at st + m * stride words).
+template <bool kFast>
+__device__ __forceinline__ void dq_decode_rows(const DqLane& D, const uint32_t* __restrict__ st, int stride,
+                                               const float4* __restrict__ cst, float (&acc)[kDqR][8]) {
+  const float4 s0 = cst[0], s1 = cst[32], o0 = cst[64], o1 = cst[96];
+  const float sc[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+  const float off[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+#pragma unroll
+  for (int m = 0; m < kDqR; ++m) {
+    const uint32_t wlo = st[m * stride + D.my_w];
+    const uint32_t whi = D.has_hi ? st[m * stride + D.my_w + 1] : 0u;
+    const uint32_t v = __funnelshift_r(wlo, whi, D.fsh);
+    float q[8];
+    if (kFast) {
+      const uint32_t v2 = v >> D.sh2;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) q[i] = __uint_as_float(((i < 5 ? v : v2) & D.key[i]) | 0x4B000000u);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) q[i] = __uint_as_float(((v >> D.key[i]) & 0xFu) | 0x4B000000u);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      float d0, d1;
+      fadd2(d0, d1, q[i], q[i + 1], off[i], off[i + 1]);  // (q - zero) * 16^p, exact
+      ffma2_acc(acc[m][i], acc[m][i + 1], d0, d1, sc[i], sc[i + 1]);
+    }
+  }
+}
+
+// Owners of kept features ja+kc .. ja+kc+kw-1 take their sums from kept[m * 32 + (j - ja - kc)].
+__device__ __forceinline__ void dq_patch_kept(const DqLane& D, float (&acc)[kDqR][8], const float* kept, int ja,
+                                              int kc, int kw) {
+  if (D.L.kmask) {
+    int jk = D.L.j0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if ((D.L.kmask >> i) & 1u) {
+        const int jj = jk - ja - kc;
+        if (jj >= 0 && jj < kw) {
+#pragma unroll
+          for (int m = 0; m < kDqR; ++m) acc[m][i] = kept[m * 32 + jj];
+        }
+        ++jk;
+      }
+    }
+  }
+}
+
+template <typename OutT>
+__device__ __forceinline__ void dq_store_rows(const DqLane& D, const float (&acc)[kDqR][8], int H, int t0,
+                                              int t_last, OutT* __restrict__ out) {
+  if (D.active) {
+#pragma unroll
+    for (int m = 0; m < kDqR; ++m) {
+      const int t = t0 + m;
+      if (t < t_last) store_row8<OutT>(out + (size_t)t * H + D.h0, acc[m]);
+    }
+  }
+}
+
+// Kept features of the warp's slice for rows t0..t0+kDqR-1, read from global memory:
+// (row, kept feature) pairs over the lanes sum the P side values in rank order; owners copy them
+// into their sums; then the rows are stored.  Warp-level only (uses `kept`, kDqR x 32 floats of
+// shared memory per warp).
+template <typename OutT>
+__device__ __forceinline__ void dq_finish_block(const DqLane& D, float (&acc)[kDqR][8],
+                                                const uint16_t* __restrict__ side, float* kept, int P,
+                                                int T, int H, int k, int ja, int jb, int t0, int t_last,
+                                                OutT* __restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  const int nk = jb - ja;
+  for (int kc = 0; kc < nk; kc += 32) {
+    const int kw = min(32, nk - kc);
+    for (int p = lane; p < kDqR * kw; p += 32) {
+      const int m = p / kw, jj = p - m * kw;
+      const int t = t0 + m;
+      float a = 0.0f;
+      if (t < t_last) {
+        const uint16_t* sp = side + (size_t)t * k + ja + kc + jj;
+        const size_t rank_stride = (size_t)T * k;
+#pragma unroll 8
+        for (int r = 0; r < P; ++r)
+          a = __fadd_rn(a, __uint_as_float((uint32_t)__ldg(sp + r * rank_stride) << 16));
+      }
+      kept[m * 32 + jj] = a;
+    }
+    __syncwarp();
+    dq_patch_kept(D, acc, kept, ja, kc, kw);
+    __syncwarp();
+  }
+  dq_store_rows<OutT>(D, acc, H, t0, t_last, out);
+}
+
+// Slice bookkeeping shared by both kernels.
+struct DqSlice {
+  int hs, he, ja, jb, Ca, Cb, w_first, n_words;
+};
+__device__ __forceinline__ DqSlice dq_slice(const int32_t* __restrict__ keep_idx, int H, int k, int s, int S) {
+  DqSlice q;
+  const int Hr = H - k, Wr = Hr / 8;
+  q.hs = 8 * s * kDqSliceGroups;
+  q.he = min(H, q.hs + 8 * kDqSliceGroups);
+  q.ja = lower_bound_i32(keep_idx, k, q.hs);
+  q.jb = lower_bound_i32(keep_idx, k, q.he);
+  if (threadIdx.x == 0 && ((s == 0 && q.ja != 0) || (s == S - 1 && q.jb != k))) record_error(HQ_ERR_BAD_INDEX);
+  q.Ca = min(max(q.hs - q.ja, 0), Hr);
+  q.Cb = min(max(q.he - q.jb, 0), Hr);
+  q.w_first = q.Ca >> 3;
+  q.n_words = max(0, min(Wr, (q.Cb >> 3) + 2) - q.w_first);  // words the slice needs per row, <= 35
+  return q;
+}
+
+// ======================================================================== TMA kernel (default)
+constexpr int kDtWarps = 8;                      // consumer warps
+constexpr int kDtThreads = 32 * (kDtWarps + 1);  // + one producer warp
+constexpr int kDtTileRows = kDtWarps * kDqR;     // 32
+constexpr int kDtWords = 40;                     // staged words per row (box inner dim)
+constexpr int kDtStages = 8;
+constexpr unsigned kDtTileBytes = kDtTileRows * kDtWords * 4;
+constexpr int kDtSideCols = 32;                  // side box width (bf16): kept features staged per slice
+constexpr int kDtMaxStagedKept = 24;             // slices with more kept features read them from HBM
+constexpr unsigned kDtSideBytes = kDtTileRows * kDtSideCols * 2;
+
+struct DtSmem {
+  alignas(128) uint32_t tile[kDtStages][kDtTileRows][kDtWords];
+  alignas(128) uint16_t side[kDtStages][kDtTileRows][kDtSideCols];
+  float kept[kDtWarps][kDqR * 32];
+  TmaRing<kDtStages> ring;
+  int abort;
+  // followed by the constants: float4 [P][4][32]
+};
+
+inline size_t dt_smem_bytes(int P) { return sizeof(DtSmem) + 128 + (size_t)P * 4 * 32 * 16; }
+
+template <typename OutT>
+__global__ void __launch_bounds__(kDtThreads, 2) dequant_reduce_tma_kernel(
+    const __grid_constant__ CUtensorMap tmap_codes, const __grid_constant__ CUtensorMap tmap_side,
+    const uint16_t* __restrict__ side, int P, int T, int H,
+    int k, const int32_t* __restrict__ keep_idx, const float* __restrict__ scale,
+    const uint8_t* __restrict__ zero, OutT* __restrict__ out, int S, int chunks, int rows_per_chunk,
+    long long wait_limit) {
+  extern __shared__ __align__(128) unsigned char s_raw[];
+  DtSmem& sm = *reinterpret_cast<DtSmem*>(s_raw);
+  float4* s_const = reinterpret_cast<float4*>(s_raw + ((sizeof(DtSmem) + 127) & ~size_t(127)));
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int s = blockIdx.x / chunks, chunk = blockIdx.x - s * chunks;
+  const int t_first = chunk * rows_per_chunk, t_last = min(T, t_first + rows_per_chunk);
+  const int nblk = (t_last - t_first + kDtTileRows - 1) / kDtTileRows;
+  const int n_tiles = nblk * P;  // tile i = (block i / P, rank i % P)
+
+  const DqSlice q = dq_slice(keep_idx, H, k, s, S);
+  const int w_a = q.w_first & ~3;  // 16-byte aligned x coordinate of the box
+  const int nk = q.jb - q.ja;
+  const int j_a = q.ja & ~7;       // 16-byte aligned x coordinate of the side box
+  const bool stage_side = nk > 0 && nk <= kDtMaxStagedKept && q.jb <= j_a + kDtSideCols;
+  if (threadIdx.x == 0) {
+    sm.ring.init(kDtWarps);
+    sm.abort = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  volatile int* abort = &sm.abort;
+
+  if (warp == kDtWarps) {  // ------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensor_map(&tmap_codes);
+      if (stage_side) prefetch_tensor_map(&tmap_side);
+      int issued = 0, bi = 0, r = 0;
+      for (int i = 0; i < n_tiles; ++i) {
+        if (!sm.ring.acquire(i, abort, wait_limit)) break;
+        const int st = i % kDtStages;
+        const int row = r * T + t_first + bi * kDtTileRows;
+        mbar_arrive_expect_tx(&sm.ring.full[st], kDtTileBytes + (stage_side ? kDtSideBytes : 0u));
+        tma_load_2d(&sm.tile[st][0][0], &tmap_codes, w_a, row, &sm.ring.full[st]);
+        if (stage_side) tma_load_2d(&sm.side[st][0][0], &tmap_side, j_a, row, &sm.ring.full[st]);
+        ++issued;
+        if (++r == P) {
+          r = 0;
+          ++bi;
+        }
+      }
+      if (*abort) sm.ring.drain(issued, wait_limit);
+    }
+    return;
+  }
+
+  // ---------------------------------------------------------------------- consumers
+  // (the producer is already loading while the consumers set up the slice's constants)
+  constexpr int kConsumers = 32 * kDtWarps;
+  const bool generic = named_barrier_or(kConsumers, dq_has_tiny_scale(scale, P, H, s, kConsumers));
+  dq_fill_constants(s_const, keep_idx, scale, zero, P, H, k, s, generic, kConsumers);
+  const DqLane D = dq_lane(keep_idx, k, H, s, lane, w_a, generic);
+  named_barrier_sync(kConsumers);
+  float* kept = sm.kept[warp];
+  // staged kept sums: pair p = lane + 32c (c < n_slots) is (row p & 3, kept feature p >> 2);
+  // koff[c] = its element offset inside a stage's side tile
+  const int n_pairs = stage_side ? kDqR * nk : 0;
+  const int n_slots = (n_pairs + 31) >> 5;
+  int koff[3];
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    const int p = lane + 32 * c;
+    koff[c] = (p < n_pairs) ? (warp * kDqR + (p & 3)) * kDtSideCols + (q.ja - j_a + (p >> 2)) : -1;
+  }
+  int i = 0;
+  for (int bi = 0; bi < nblk && !*abort; ++bi) {
+    const int t0 = t_first + bi * kDtTileRows + warp * kDqR;
+    float acc[kDqR][8];
+#pragma unroll
+    for (int m = 0; m < kDqR; ++m)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[m][e] = 0.0f;
+    float kacc[3] = {0.0f, 0.0f, 0.0f};
+    bool ok = true;
+    for (int r = 0; r < P; ++r, ++i) {
+      if (!sm.ring.wait_full(i, abort, wait_limit)) {
+        ok = false;
+        break;
+      }
+      const int st_i = i % kDtStages;
+      const uint32_t* st = &sm.tile[st_i][warp * kDqR][0];
+      const float4* cst = s_const + (size_t)r * 4 * 32 + lane;
+      if (D.decode) {
+        if (generic) dq_decode_rows<false>(D, st, kDtWords, cst, acc);
+        else dq_decode_rows<true>(D, st, kDtWords, cst, acc);
+      }
+      const uint16_t* sside = &sm.side[st_i][0][0];
+#pragma unroll
+      for (int c = 0; c < 3; ++c) {
+        if (c < n_slots && koff[c] >= 0) kacc[c] = __fadd_rn(kacc[c], __uint_as_float((uint32_t)sside[koff[c]] << 16));
+      }
+      __syncwarp();
+      if (lane == 0) sm.ring.release(i);
+    }
+    if (!ok) break;
+    if (stage_side) {
+#pragma unroll
+      for (int c = 0; c < 3; ++c) {
+        const int p = lane + 32 * c;
+        if (p < n_pairs) kept[(p & 3) * 32 + (p >> 2)] = kacc[c];
+      }
+      __syncwarp();
+      dq_patch_kept(D, acc, kept, q.ja, 0, nk);
+      __syncwarp();
+      dq_store_rows<OutT>(D, acc, H, t0, t_last, out);
+    } else {
+      dq_finish_block<OutT>(D, acc, side, kept, P, T, H, k, q.ja, q.jb, t0, t_last, out);
+    }
+  }
+}
+
+// =============================================================== cp.async kernel (any shape)
+constexpr int kDqWarps = 8;
+constexpr int kDqThreads = 32 * kDqWarps;
+constexpr int kDqD = 8;       // cp.async tiles in flight per warp
+constexpr int kDqWin = 36;    // staged words per row (>= 35)
+
+// Dynamic shared memory of one CTA for P ranks.
+inline size_t dq_smem_bytes(int P) {
+  return (size_t)P * 4 * 32 * 16                            // constants: [P][4][32] float4
+         + (size_t)kDqWarps * kDqD * kDqR * kDqWin * 4      // staged code tiles
+         + (size_t)kDqWarps * kDqR * 32 * 4;                // kept sums
+}
+
 template <typename OutT>
 __global__ void __launch_bounds__(kDqThreads) dequant_reduce_kernel(
     const uint32_t* __restrict__ codes, const uint16_t* __restrict__ side, int P, int T, int H,
@@ -82,166 +441,70 @@ __global__ void __launch_bounds__(kDqThreads) dequant_reduce_kernel(
   float* s_kept = reinterpret_cast<float*>(s_tiles + kDqWarps * kDqD * kDqR * kDqWin);
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int Hr = H - k, Wr = Hr / 8;
+  const int Wr = (H - k) / 8;
   const int s = blockIdx.x / chunks, chunk = blockIdx.x - s * chunks;
   const int t_first = chunk * rows_per_chunk, t_last = min(T, t_first + rows_per_chunk);
 
-  // ---- this lane's group: layout and nibble positions ----------------------------------------
-  const int h0 = 8 * (s * kDqSliceGroups + lane);
-  const bool active = h0 < H;
-  GroupLayout L{0, 0, 0u, 0};
-  if (active) L = group_layout(keep_idx, k, H, h0);
-  int nib_shift[8];
-  {
-    int j = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const bool kept = (L.kmask >> i) & 1u;
-      nib_shift[i] = kept ? 0 : 4 * j;
-      j += kept ? 0 : 1;
-    }
-  }
-  // words the warp stages per row: [w_first, w_end), at most 35
-  const int hs = 8 * s * kDqSliceGroups, he = min(H, hs + 8 * kDqSliceGroups);
-  const int ja = lower_bound_i32(keep_idx, k, hs), jb = lower_bound_i32(keep_idx, k, he);
-  if (threadIdx.x == 0 && ((s == 0 && ja != 0) || (s == S - 1 && jb != k))) record_error(HQ_ERR_BAD_INDEX);
-  const int Ca = min(max(hs - ja, 0), Hr), Cb = min(max(he - jb, 0), Hr);
-  const int w_first = Ca >> 3;
-  const int n_words = max(0, min(Wr, (Cb >> 3) + 2) - w_first);
-  const int my_w = (L.c0 >> 3) - w_first;  // this lane's first word inside the window
-  const int fsh = 4 * (L.c0 & 7);
-  const bool has_hi = (L.c0 >> 3) + 1 < Wr;
-
-  // ---- constants of the slice for all ranks (conflict-free [P][4][32] float4 layout) ---------
-  for (int idx = threadIdx.x; idx < P * 32; idx += kDqThreads) {
-    const int r = idx >> 5, g = idx & 31;
-    const int hg = 8 * (s * kDqSliceGroups + g);
-    float sc[8], off[8];
-    uint32_t km = 0;
-    if (hg < H) km = group_layout(keep_idx, k, H, hg).kmask;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      sc[i] = 0.0f;
-      off[i] = -8388608.0f;
-      if (hg < H && !((km >> i) & 1u)) {
-        const size_t p = (size_t)r * H + hg + i;
-        sc[i] = scale[p];
-        off[i] = -__int_as_float(0x4B000000 | (int)zero[p]);  // -(2^23 + zero)
-      }
-    }
-    float4* dst = s_const + (size_t)r * 4 * 32 + g;
-    dst[0] = make_float4(sc[0], sc[1], sc[2], sc[3]);
-    dst[32] = make_float4(sc[4], sc[5], sc[6], sc[7]);
-    dst[64] = make_float4(off[0], off[1], off[2], off[3]);
-    dst[96] = make_float4(off[4], off[5], off[6], off[7]);
-  }
+  const DqSlice q = dq_slice(keep_idx, H, k, s, S);
+  const bool generic = __syncthreads_or(dq_has_tiny_scale(scale, P, H, s, kDqThreads)) != 0;
+  const DqLane D = dq_lane(keep_idx, k, H, s, lane, q.w_first, generic);
+  dq_fill_constants(s_const, keep_idx, scale, zero, P, H, k, s, generic, kDqThreads);
   __syncthreads();
 
-  // ---- this warp's row blocks: rows t_first + (warp + kDqWarps*bi)*kDqR + m ------------------
+  // this warp's row blocks: rows t_first + (warp + kDqWarps*bi)*kDqR + m
   const int nblk_total = (t_last - t_first + kDqR - 1) / kDqR;
   const int my_blocks = nblk_total > warp ? (nblk_total - warp + kDqWarps - 1) / kDqWarps : 0;
   const int n_tiles = my_blocks * P;  // tile i = (block i / P, rank i % P)
   uint32_t* my_tiles = s_tiles + (size_t)warp * kDqD * kDqR * kDqWin;
   float* my_kept = s_kept + warp * kDqR * 32;
   const uint32_t tiles_saddr = smem_addr(my_tiles);
+  const size_t rank_words = (size_t)T * Wr;
 
-  auto block_row0 = [&](int bi) { return t_first + (warp + kDqWarps * bi) * kDqR; };
-  auto issue_tile = [&](int i) {
-    if (i < n_tiles) {
-      const int bi = i / P, r = i - bi * P;
-      const int t0 = block_row0(bi);
-      const int stage = i % kDqD;
+  int i_next = 0, ib = 0, ir = 0;
+  auto issue_next = [&]() {
+    if (i_next < n_tiles) {
+      const int t0 = t_first + (warp + kDqWarps * ib) * kDqR;
+      const uint32_t* src = codes + (size_t)ir * rank_words + (size_t)t0 * Wr + q.w_first;
+      const uint32_t dst = tiles_saddr + (uint32_t)(((i_next % kDqD) * kDqR * kDqWin) * 4);
 #pragma unroll
       for (int m = 0; m < kDqR; ++m) {
-        const int t = t0 + m;
-        if (t < t_last) {
-          const uint32_t* src = codes + ((size_t)r * T + t) * Wr + w_first;
-          const uint32_t dst = tiles_saddr + (uint32_t)(((stage * kDqR + m) * kDqWin) * 4);
-          for (int w = lane; w < n_words; w += 32) cp_async4(dst + 4u * w, src + w);
+        if (t0 + m < t_last) {
+          if (lane < q.n_words) cp_async4(dst + 4u * (m * kDqWin + lane), src + (size_t)m * Wr + lane);
+          if (lane + 32 < q.n_words)
+            cp_async4(dst + 4u * (m * kDqWin + lane + 32), src + (size_t)m * Wr + lane + 32);
         }
       }
+      if (++ir == P) {
+        ir = 0;
+        ++ib;
+      }
+      ++i_next;
     }
     cp_async_commit();  // one group per tile, empty ones included, keeps the count uniform
   };
+  for (int i = 0; i < kDqD - 1; ++i) issue_next();
 
-  for (int i = 0; i < kDqD - 1; ++i) issue_tile(i);
-
-  const int nk = jb - ja;
   int tile = 0;
   for (int bi = 0; bi < my_blocks; ++bi) {
-    const int t0 = block_row0(bi);
+    const int t0 = t_first + (warp + kDqWarps * bi) * kDqR;
     float acc[kDqR][8];
 #pragma unroll
     for (int m = 0; m < kDqR; ++m)
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[m][i] = 0.0f;
-
+      for (int e = 0; e < 8; ++e) acc[m][e] = 0.0f;
     for (int r = 0; r < P; ++r, ++tile) {
-      issue_tile(tile + kDqD - 1);
+      issue_next();
       cp_async_wait<kDqD - 1>();
       __syncwarp();
       const uint32_t* st = my_tiles + (size_t)(tile % kDqD) * kDqR * kDqWin;
       const float4* cst = s_const + (size_t)r * 4 * 32 + lane;
-      const float4 s0 = cst[0], s1 = cst[32], o0 = cst[64], o1 = cst[96];
-      const float sc[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-      const float off[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
-      if (active && L.n > 0) {
-#pragma unroll
-        for (int m = 0; m < kDqR; ++m) {
-          const uint32_t wlo = st[m * kDqWin + my_w];
-          const uint32_t whi = has_hi ? st[m * kDqWin + my_w + 1] : 0u;
-          const uint32_t v = __funnelshift_r(wlo, whi, fsh);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const uint32_t bits = ((v >> nib_shift[i]) & 0xFu) | 0x4B000000u;
-            const float d = __fadd_rn(__uint_as_float(bits), off[i]);
-            acc[m][i] = __fmaf_rn(d, sc[i], acc[m][i]);
-          }
-        }
+      if (D.decode) {
+        if (generic) dq_decode_rows<false>(D, st, kDqWin, cst, acc);
+        else dq_decode_rows<true>(D, st, kDqWin, cst, acc);
       }
       __syncwarp();  // the stage is free for the copy issued next iteration
     }
-
-    // ---- kept features of the warp's slice: (row, kept feature) pairs over the lanes ---------
-    for (int kc = 0; kc < nk; kc += 32) {
-      const int kw = min(32, nk - kc);
-      for (int p = lane; p < kDqR * kw; p += 32) {
-        const int m = p / kw, jj = p - m * kw;
-        const int t = t0 + m;
-        float a = 0.0f;
-        if (t < t_last) {
-          const uint16_t* sp = side + (size_t)t * k + ja + kc + jj;
-          const size_t rank_stride = (size_t)T * k;
-#pragma unroll 8
-          for (int r = 0; r < P; ++r) a = __fadd_rn(a, __uint_as_float((uint32_t)__ldg(sp + r * rank_stride) << 16));
-        }
-        my_kept[m * 32 + jj] = a;
-      }
-      __syncwarp();
-      if (L.kmask) {
-        int jk = L.j0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          if ((L.kmask >> i) & 1u) {
-            const int jj = jk - ja - kc;
-            if (jj >= 0 && jj < kw) {
-#pragma unroll
-              for (int m = 0; m < kDqR; ++m) acc[m][i] = my_kept[m * 32 + jj];
-            }
-            ++jk;
-          }
-        }
-      }
-      __syncwarp();
-    }
-
-    if (active) {
-#pragma unroll
-      for (int m = 0; m < kDqR; ++m) {
-        const int t = t0 + m;
-        if (t < t_last) store_row8<OutT>(out + (size_t)t * H + h0, acc[m]);
-      }
-    }
+    dq_finish_block<OutT>(D, acc, side, my_kept, P, T, H, k, q.ja, q.jb, t0, t_last, out);
   }
   cp_async_wait<0>();
 }

@@ -9,47 +9,90 @@
 // float(c) is formed without a conversion instruction: the bits c + 0x4B400000 are the float
 // 1.5*2^23 + c, from which 1.5*2^23 is subtracted exactly.
 //
-// Work decomposition as in dequant-reduce: the 8 warps of a CTA share one slice of 256 features
-// (one group of 8 per lane) and its per-(rank, feature) constants in shared memory, and split
-// the CTA's row range in blocks of kFuR rows.  A warp walks the ranks in order; each lane stages
-// its own 16 bytes of the kFuR rows of upcoming ranks into shared memory with cp.async, kFuD - 1
-// tiles ahead, and reads back only what it copied (its own wait_group is the only sync needed).
+// Work decomposition as in dequant-reduce: a CTA covers a slice of 256 features and a range of
+// rows; its per-(rank, feature) constants live in shared memory.  Warp 8 is the producer: one
+// lane loads, per (32-row block, rank), the 32 x 256 bf16 tile (16 KB) with one TMA instruction
+// into a 3-stage mbarrier ring.  Warps 0..7 consume 4 rows each (lane l: features 8l..8l+7),
+// walking the ranks in order with 4 x 8 fp32 sums in registers.
 //
 // Roofline: HBM-bound, P*2 bytes read + 2 (or 4) bytes written per output element.
+// No memory beyond the inputs and outputs is used.
 #pragma once
 
 #include "hq_common.cuh"
+#include "hq_tma.cuh"
 #include "k_dequant.cuh"
 
 namespace hq {
 
-constexpr int kFuWarps = 8;
-constexpr int kFuThreads = 32 * kFuWarps;
-constexpr int kFuR = 4;
-constexpr int kFuD = 3;  // tiles staged per warp
-constexpr int kFuSliceGroups = 32;
+constexpr int kFuWarps = 8;                      // consumer warps
+constexpr int kFuThreads = 32 * (kFuWarps + 1);  // + one producer warp
+constexpr int kFuR = 4;                          // rows per consumer warp per block
+constexpr int kFuTileRows = kFuWarps * kFuR;     // 32
+constexpr int kFuSlice = 256;
+constexpr int kFuStages = 3;
+constexpr unsigned kFuTileBytes = kFuTileRows * kFuSlice * 2;
 
-inline size_t fu_smem_bytes(int P) {
-  return (size_t)P * 5 * 32 * 16 + (size_t)kFuWarps * kFuD * kFuR * 32 * 16;
-}
+struct FuSmem {
+  alignas(128) uint16_t tile[kFuStages][kFuTileRows][kFuSlice];
+  TmaRing<kFuStages> ring;
+  int abort;
+  // followed by the constants: float4 [P][5][32]
+};
+
+inline size_t fu_smem_bytes(int P) { return sizeof(FuSmem) + 128 + (size_t)P * 5 * 32 * 16; }
 
 template <typename OutT>
-__global__ void __launch_bounds__(kFuThreads) compress_reduce_kernel(
-    const uint16_t* __restrict__ x, int P, int T, int H, int k, const int32_t* __restrict__ keep_idx,
-    const float* __restrict__ scale, const float* __restrict__ inv_scale,
-    const uint8_t* __restrict__ zero, OutT* __restrict__ out, int S, int chunks, int rows_per_chunk) {
-  extern __shared__ float4 s_dyn[];
-  float4* s_const = s_dyn;  // [P][5][32]: inv 0-3, inv 4-7, scale 0-3, scale 4-7, (zero bytes, kmask)
-
+__global__ void __launch_bounds__(kFuThreads, 2) compress_reduce_kernel(
+    const __grid_constant__ CUtensorMap tmap_x, int P, int T, int H, int k,
+    const int32_t* __restrict__ keep_idx, const float* __restrict__ scale,
+    const float* __restrict__ inv_scale, const uint8_t* __restrict__ zero, OutT* __restrict__ out, int S,
+    int chunks, int rows_per_chunk, long long wait_limit) {
+  extern __shared__ __align__(128) unsigned char s_raw[];
+  FuSmem& sm = *reinterpret_cast<FuSmem*>(s_raw);
+  float4* s_const = reinterpret_cast<float4*>(s_raw + ((sizeof(FuSmem) + 127) & ~size_t(127)));
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int s = blockIdx.x / chunks, chunk = blockIdx.x - s * chunks;
   const int t_first = chunk * rows_per_chunk, t_last = min(T, t_first + rows_per_chunk);
-  const int h0 = 8 * (s * kFuSliceGroups + lane);
-  const bool active = h0 < H;
+  const int nblk = (t_last - t_first + kFuTileRows - 1) / kFuTileRows;
+  const int n_tiles = nblk * P;  // tile i = (block i / P, rank i % P)
+  const int hs = s * kFuSlice;
 
-  for (int idx = threadIdx.x; idx < P * 32; idx += kFuThreads) {
+  if (threadIdx.x == 0) {
+    sm.ring.init(kFuWarps);
+    sm.abort = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  volatile int* abort = &sm.abort;
+  constexpr int kConsumers = 32 * kFuWarps;
+
+  if (warp == kFuWarps) {  // ------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensor_map(&tmap_x);
+      int issued = 0, bi = 0, r = 0;
+      for (int i = 0; i < n_tiles; ++i) {
+        if (!sm.ring.acquire(i, abort, wait_limit)) break;
+        const int st = i % kFuStages;
+        mbar_arrive_expect_tx(&sm.ring.full[st], kFuTileBytes);
+        tma_load_2d(&sm.tile[st][0][0], &tmap_x, hs, r * T + t_first + bi * kFuTileRows, &sm.ring.full[st]);
+        ++issued;
+        if (++r == P) {
+          r = 0;
+          ++bi;
+        }
+      }
+      if (*abort) sm.ring.drain(issued, wait_limit);
+    }
+    return;
+  }
+
+  // ---------------------------------------------------------------------- consumers
+  // constants [P][5][32]: inv 0-3, inv 4-7, scale 0-3, scale 4-7 (1 for kept), (zero bytes, kmask),
+  // filled while the producer is already loading
+  for (int idx = threadIdx.x; idx < P * 32; idx += kConsumers) {
     const int r = idx >> 5, g = idx & 31;
-    const int hg = 8 * (s * kFuSliceGroups + g);
+    const int hg = hs + 8 * g;
     float iv[8], sc[8];
     uint32_t zlo = 0, zhi = 0, km = 0;
     if (hg < H) {
@@ -74,74 +117,64 @@ __global__ void __launch_bounds__(kFuThreads) compress_reduce_kernel(
     dst[96] = make_float4(sc[4], sc[5], sc[6], sc[7]);
     dst[128] = make_float4(__uint_as_float(zlo), __uint_as_float(zhi), __uint_as_float(km), 0.0f);
   }
-  __syncthreads();
-  if (!active) return;
-
+  named_barrier_sync(kConsumers);
+  const int h0 = hs + 8 * lane;
+  const bool active = h0 < H;
   const uint32_t kmask = __float_as_uint(s_const[128 + lane].z);
-  const int nblk_total = (t_last - t_first + kFuR - 1) / kFuR;
-  const int my_blocks = nblk_total > warp ? (nblk_total - warp + kFuWarps - 1) / kFuWarps : 0;
-  const int n_tiles = my_blocks * P;  // tile i = (block i / P, rank i % P)
-  uint4* my_rows = reinterpret_cast<uint4*>(s_const + (size_t)P * 5 * 32) + (size_t)warp * kFuD * kFuR * 32;
-  const uint16_t* xl = x + h0;
-
-  auto block_row0 = [&](int bi) { return t_first + (warp + kFuWarps * bi) * kFuR; };
-  auto issue = [&](int i) {
-    if (i < n_tiles) {
-      const int bi = i / P, r = i - bi * P;
-      const int t0 = block_row0(bi);
-      const int stage = i % kFuD;
-#pragma unroll
-      for (int m = 0; m < kFuR; ++m)
-        if (t0 + m < t_last)
-          cp_async16(smem_addr(my_rows + (stage * kFuR + m) * 32 + lane), xl + ((size_t)r * T + t0 + m) * H);
-    }
-    cp_async_commit();
-  };
-  for (int i = 0; i < kFuD - 1; ++i) issue(i);
-
-  int tile = 0;
-  for (int bi = 0; bi < my_blocks; ++bi) {
-    const int t0 = block_row0(bi);
-    const int nrows = min(kFuR, t_last - t0);
+  int i = 0;
+  for (int bi = 0; bi < nblk && !*abort; ++bi) {
+    const int t0 = t_first + bi * kFuTileRows + warp * kFuR;
     float acc[kFuR][8];
 #pragma unroll
     for (int m = 0; m < kFuR; ++m)
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[m][i] = 0.0f;
-
-    for (int r = 0; r < P; ++r, ++tile) {
-      issue(tile + kFuD - 1);
-      cp_async_wait<kFuD - 1>();
-      const uint4* st = my_rows + (tile % kFuD) * kFuR * 32 + lane;
-      const float4* cst = s_const + (size_t)r * 5 * 32 + lane;
-      const float4 i0 = cst[0], i1 = cst[32], s0 = cst[64], s1 = cst[96], zz = cst[128];
-      const float inv[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
-      const float sc[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-      const uint32_t zlo = __float_as_uint(zz.x), zhi = __float_as_uint(zz.y);
-      int lo[8];
+      for (int e = 0; e < 8; ++e) acc[m][e] = 0.0f;
+    bool ok = true;
+    for (int r = 0; r < P; ++r, ++i) {
+      if (!sm.ring.wait_full(i, abort, wait_limit)) {
+        ok = false;
+        break;
+      }
+      if (active) {
+        const float4* cst = s_const + (size_t)r * 5 * 32 + lane;
+        const float4 i0 = cst[0], i1 = cst[32], s0 = cst[64], s1 = cst[96], zz = cst[128];
+        const float inv[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
+        const float sc[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+        const uint32_t zlo = __float_as_uint(zz.x), zhi = __float_as_uint(zz.y);
+        int lo[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) lo[i] = -(int)(((i < 4 ? zlo : zhi) >> (8 * (i & 3))) & 0xFFu);
+        for (int e = 0; e < 8; ++e) lo[e] = -(int)(((e < 4 ? zlo : zhi) >> (8 * (e & 3))) & 0xFFu);
 #pragma unroll
-      for (int m = 0; m < kFuR; ++m) {
-        if (m < nrows) {
-          const uint4 xv = st[m * 32];
+        for (int m = 0; m < kFuR; ++m) {
+          const uint4 xv = reinterpret_cast<const uint4*>(&sm.tile[i % kFuStages][warp * kFuR + m][0])[lane];
+          const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float f = bf16_at(xv, i);
-            int c = __float2int_rn(__fmul_rn(f, inv[i]));  // saturating; NaN -> 0
-            c = min(max(c, lo[i]), lo[i] + 15);
-            const float d = __fadd_rn(__int_as_float(c + 0x4B400000), -12582912.0f);
-            const float v = ((kmask >> i) & 1u) ? f : d;
-            acc[m][i] = __fmaf_rn(v, sc[i], acc[m][i]);
+          for (int e = 0; e < 8; e += 2) {
+            const float f0 = __uint_as_float(w[e / 2] << 16), f1 = __uint_as_float(w[e / 2] & 0xFFFF0000u);
+            float a0, a1;
+            fmul2(a0, a1, f0, f1, inv[e], inv[e + 1]);
+            int c0 = __float2int_rn(a0), c1 = __float2int_rn(a1);  // saturating; NaN -> 0
+            c0 = min(max(c0, lo[e]), lo[e] + 15);
+            c1 = min(max(c1, lo[e + 1]), lo[e + 1] + 15);
+            float d0, d1;
+            fadd2(d0, d1, __int_as_float(c0 + 0x4B400000), __int_as_float(c1 + 0x4B400000), -12582912.0f,
+                  -12582912.0f);
+            const float v0 = ((kmask >> e) & 1u) ? f0 : d0;
+            const float v1 = ((kmask >> (e + 1)) & 1u) ? f1 : d1;
+            ffma2_acc(acc[m][e], acc[m][e + 1], v0, v1, sc[e], sc[e + 1]);
           }
         }
       }
+      __syncwarp();
+      if (lane == 0) sm.ring.release(i);
     }
+    if (!ok) break;
+    if (active) {
 #pragma unroll
-    for (int m = 0; m < kFuR; ++m)
-      if (m < nrows) store_row8<OutT>(out + (size_t)(t0 + m) * H + h0, acc[m]);
+      for (int m = 0; m < kFuR; ++m)
+        if (t0 + m < t_last) store_row8<OutT>(out + (size_t)(t0 + m) * H + h0, acc[m]);
+    }
   }
-  cp_async_wait<0>();
 }
 
 }  // namespace hq

@@ -40,12 +40,12 @@ constexpr int kQpThreads = 32 * kQpWarps;
 constexpr int kQpR = 4;              // rows per tile
 constexpr int kQpD = 3;              // tiles staged per warp (kQpD - 1 in flight while computing)
 constexpr int kQpSliceGroups = 32;   // groups per warp slice
-constexpr int kQpBufWords = 36;      // >= 33 owned words per row
+constexpr int kQpBufWords = 36;      // >= 33 owned words + 2 guard slots per row
 
 struct QpWarpSmem {
   uint4 rows[kQpD][kQpR][32];        // each lane's 16 bytes of each staged row
-  uint32_t halo[kQpD][kQpR][8];      // the 4-byte word holding each halo lane's feature
-  uint32_t buf[kQpR][kQpBufWords];   // compact words being assembled
+  uint32_t halo[kQpD][kQpR][8];      // the 4-byte word holding each halo feature
+  uint32_t buf[kQpR][kQpBufWords];   // slot 1 + (word - Wb); slot 0 and slot nw + 1 are guards
 };
 
 __global__ void __launch_bounds__(kQpThreads) quantize_pack_kernel(
@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(kQpThreads) quantize_pack_kernel(
     const int h0 = 8 * g;
     GroupLayout L{0, 0, 0u, 0};
     float inv[8];
-    int lo[8];
+    int lo[8], hi[8];
     uint32_t mul[8], zbase = 0;
     if (active) L = group_layout(keep_idx, k, H, h0);
     {
@@ -93,6 +93,7 @@ __global__ void __launch_bounds__(kQpThreads) quantize_pack_kernel(
           inv[i] = inv_scale[p];
         }
         lo[i] = -z;
+        hi[i] = 15 - z;
         mul[i] = (active && !kept) ? (1u << (4 * j)) : 0u;
         j += kept ? 0 : 1;
         zbase += (uint32_t)z * mul[i];
@@ -107,96 +108,108 @@ __global__ void __launch_bounds__(kQpThreads) quantize_pack_kernel(
     const int Wb = (Ca + 7) >> 3, We = (Cb + 7) >> 3;  // owned words [Wb, We)
     const int nw = max(We - Wb, 0);                    // <= 33
     const int nhalo = (We > Wb) ? (8 * We - Cb) : 0;   // 0..7 codes from the next slice
+    const int slot = (L.c0 >> 3) - Wb + 1;             // buffer slot of the group's first word
+    const int sh = 4 * (L.c0 & 7);
 
-    // halo lane: one non-kept feature after the slice
-    const bool is_halo = lane < nhalo;
+    // halo work of a tile: lane p < nhalo*kQpR takes halo feature p % nhalo of row p / nhalo
+    const bool is_halo = lane < nhalo * kQpR;
+    const int h_row = is_halo ? lane / nhalo : 0, h_idx = is_halo ? lane - h_row * nhalo : 0;
     float h_inv = 0.0f;
     int h_col = 0, h_lo = 0, h_z = 0, h_shift = 0;
     if (is_halo) {
-      h_col = checked_col(rest_idx, Cb + lane, H);
+      h_col = checked_col(rest_idx, Cb + h_idx, H);
       const size_t p = (size_t)r * H + h_col;
       h_z = zero[p];
       h_inv = inv_scale[p];
       h_lo = -h_z;
-      h_shift = 4 * ((Cb + lane) & 7);
+      h_shift = 4 * ((Cb + h_idx) & 7);
     }
+    // kept work of a tile: pair p = jj * kQpR + m (rounds of 32 pairs)
     const int nk = jb - ja;
-    const int w0 = (L.c0 >> 3) - Wb, sh = 4 * (L.c0 & 7);
+    const int npairs = nk * kQpR;
+
     const uint16_t* xr = x + ((size_t)r * T) * H;
+    uint32_t* crow = codes + ((size_t)r * T) * Wr + Wb;
+    uint16_t* srow = side + ((size_t)r * T) * k;
     const int n_tiles = (t_stop - t_begin + kQpR - 1) / kQpR;
 
-    auto issue = [&](int i) {
-      if (i < n_tiles) {
-        const int stage = i % kQpD;
+    int i_next = 0;
+    auto issue_next = [&]() {
+      if (i_next < n_tiles) {
+        const int stage = i_next % kQpD;
+        const int t0 = t_begin + i_next * kQpR;
+        const uint16_t* src = xr + (size_t)t0 * H;
 #pragma unroll
-        for (int m = 0; m < kQpR; ++m) {
-          const int t = t_begin + i * kQpR + m;
-          if (t < t_stop) {
-            if (active) cp_async16(smem_addr(&W.rows[stage][m][lane]), xr + (size_t)t * H + h0);
-            if (is_halo) cp_async4(smem_addr(&W.halo[stage][m][lane]), xr + (size_t)t * H + (h_col & ~1));
-          }
-        }
+        for (int m = 0; m < kQpR; ++m)
+          if (active && t0 + m < t_stop) cp_async16(smem_addr(&W.rows[stage][m][lane]), src + (size_t)m * H + h0);
+        if (is_halo && t0 + h_row < t_stop)
+          cp_async4(smem_addr(&W.halo[stage][h_row][h_idx]), src + (size_t)h_row * H + (h_col & ~1));
+        ++i_next;
       }
       cp_async_commit();
     };
-    for (int i = 0; i < kQpD - 1; ++i) issue(i);
+    for (int i = 0; i < kQpD - 1; ++i) issue_next();
 
     for (int i = 0; i < n_tiles; ++i) {
-      issue(i + kQpD - 1);
+      issue_next();
       cp_async_wait<kQpD - 1>();
-      __syncwarp();  // the kept-value shuffles below read other lanes' registers, not their smem
+      __syncwarp();
       const int stage = i % kQpD;
-      const int t = t_begin + i * kQpR;
-      const int nrows = min(kQpR, t_stop - t);
+      const int t0 = t_begin + i * kQpR;
+      const int nrows = min(kQpR, t_stop - t0);
+      // codes of the lane's group, one word V per row, OR-ed into two slots
+      if (active && L.n > 0) {
 #pragma unroll
-      for (int m = 0; m < kQpR; ++m) {
-        if (m >= nrows) break;
-        const uint4 v = W.rows[stage][m][lane];
-        if (active && L.n > 0) {
+        for (int m = 0; m < kQpR; ++m) {
+          const uint4 v = W.rows[stage][m][lane];
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
           uint32_t V = zbase;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float a = __fmul_rn(bf16_at(v, e), inv[e]);
-            int c = __float2int_rn(a);  // saturating; NaN -> 0
-            c = min(max(c, lo[e]), lo[e] + 15);
-            V += (uint32_t)c * mul[e];
+          for (int e = 0; e < 8; e += 2) {
+            float a0, a1;
+            fmul2(a0, a1, __uint_as_float(w[e / 2] << 16), __uint_as_float(w[e / 2] & 0xFFFF0000u),
+                  inv[e], inv[e + 1]);
+            int c0 = __float2int_rn(a0), c1 = __float2int_rn(a1);  // saturating; NaN -> 0
+            c0 = min(max(c0, lo[e]), hi[e]);
+            c1 = min(max(c1, lo[e + 1]), hi[e + 1]);
+            V += (uint32_t)c0 * mul[e] + (uint32_t)c1 * mul[e + 1];
           }
-          const uint32_t lo_part = V << sh;
-          const uint32_t hi_part = sh ? (V >> (32 - sh)) : 0u;
-          if (lo_part && w0 >= 0 && w0 < nw) atomicOr(&W.buf[m][w0], lo_part);
-          if (hi_part && w0 + 1 >= 0 && w0 + 1 < nw) atomicOr(&W.buf[m][w0 + 1], hi_part);
+          atomicOr(&W.buf[m][slot], V << sh);
+          atomicOr(&W.buf[m][slot + 1], sh ? (V >> (32 - sh)) : 0u);
         }
-        if (is_halo) {
-          const uint32_t hw = W.halo[stage][m][lane];
-          const uint32_t hb16 = (h_col & 1) ? (hw & 0xFFFF0000u) : (hw << 16);
-          int c = __float2int_rn(__fmul_rn(__uint_as_float(hb16), h_inv));
-          c = min(max(c, h_lo), h_lo + 15) + h_z;
-          if (c) atomicOr(&W.buf[m][nw - 1], (uint32_t)c << h_shift);
-        }
-        // kept values, one per lane (rounds of 32), from the owner lane's staged row
-        for (int kc = 0; kc < nk; kc += 32) {
-          const int j = ja + kc + lane;
-          const bool mine = j < jb;
-          const int col = mine ? checked_col(keep_idx, j, H) : ha;
-          const int src = min(max((col - ha) >> 3, 0), 31), e = col & 7;
-          const uint32_t a0 = __shfl_sync(0xFFFFFFFFu, v.x, src);
-          const uint32_t a1 = __shfl_sync(0xFFFFFFFFu, v.y, src);
-          const uint32_t a2 = __shfl_sync(0xFFFFFFFFu, v.z, src);
-          const uint32_t a3 = __shfl_sync(0xFFFFFFFFu, v.w, src);
-          const uint32_t w = (e < 2) ? a0 : (e < 4) ? a1 : (e < 6) ? a2 : a3;
-          if (mine) side[((size_t)r * T + t + m) * k + j] = (uint16_t)((e & 1) ? (w >> 16) : (w & 0xFFFFu));
+      }
+      if (is_halo && h_row < nrows) {
+        const uint32_t hw = W.halo[stage][h_row][h_idx];
+        const uint32_t hb16 = (h_col & 1) ? (hw & 0xFFFF0000u) : (hw << 16);
+        int c = __float2int_rn(__fmul_rn(__uint_as_float(hb16), h_inv));
+        c = min(max(c, h_lo), h_lo + 15) + h_z;
+        atomicOr(&W.buf[h_row][nw], (uint32_t)c << h_shift);
+      }
+      // kept values straight from the staged rows
+      for (int p = lane; p < npairs; p += 32) {
+        const int jj = p / kQpR, m = p - jj * kQpR;
+        if (m < nrows) {
+          const int j = ja + jj;
+          const int col = checked_col(keep_idx, j, H);
+          const int src = min(max((col - ha) >> 3, 0), 31);
+          const uint16_t* rowp = reinterpret_cast<const uint16_t*>(&W.rows[stage][m][src]);
+          srow[(size_t)(t0 + m) * k + j] = rowp[col & 7];
         }
       }
       __syncwarp();
-      // owned words out, buffer cleared
+      // owned words out (slots 1..nw).  Each lane clears exactly the slots it read (slots
+      // 1..kQpBufWords-1 in all; slot 0 only ever collects nibbles of the previous slice's word
+      // and is never read), so every read precedes its clear in that lane's program order.
 #pragma unroll
       for (int m = 0; m < kQpR; ++m) {
-        if (m < nrows) {
-          uint32_t* dst = codes + ((size_t)r * T + t + m) * Wr + Wb;
-          for (int q = lane; q < nw; q += 32) {
-            dst[q] = W.buf[m][q];
-            W.buf[m][q] = 0u;
-          }
+        uint32_t* dst = crow + (size_t)(t0 + m) * Wr;
+        const uint32_t a = W.buf[m][lane + 1];
+        if (m < nrows && lane < nw) dst[lane] = a;
+        W.buf[m][lane + 1] = 0u;
+        if (lane + 33 < kQpBufWords) {
+          const uint32_t b = W.buf[m][lane + 33];
+          if (m < nrows && lane + 32 < nw) dst[lane + 32] = b;
+          W.buf[m][lane + 33] = 0u;
         }
       }
       __syncwarp();

@@ -142,6 +142,15 @@ const char* hq_status_string(hq_status s);
  */
 hq_status hq_read_device_error(void* stream);
 
+/*
+ * Self-test of the bounded waits used by the TMA pipelines (no counterpart on the page; it
+ * exists so that failure detection can be tested without faulting or hanging a GPU): launches
+ * one thread that waits on a shared-memory mbarrier nothing ever arrives on, giving up after
+ * `limit_cycles` clock cycles.  It records HQ_ERR_TIMEOUT in the device error word (read it
+ * with hq_read_device_error) and returns; the context stays usable.
+ */
+hq_status hq_selftest_bounded_wait(long long limit_cycles, void* stream);
+
 /* Bytes of the two wire buffers per rank and row: 4-bit part (H-k)/2, BF16 part 2k. */
 int64_t hq_wire_bytes_per_row(int H, int k);
 

@@ -129,6 +129,32 @@ def test_special_input_values_bit_exact():
     compare_all(cfg, cal, x)
 
 
+def test_tiny_scales_bit_exact():
+    """Scales below 2^-109 (partial sums of magnitude ~1e-35): the dequant kernel decodes such
+    slices with explicit shifts instead of pre-divided scales, still bit-exact."""
+    o = oracle.get()
+    P, T, H, k = 3, 20, 1024, 16
+    rng = np.random.default_rng(21)
+    vals = (rng.standard_normal((P, T, H)) * 1e-35).astype(np.float32)
+    vals[:, :, 300:700] *= 1e30          # ordinary magnitudes in some slices
+    from pins import f32_to_bf16_torch
+    x = f32_to_bf16_torch(vals.ravel()).reshape(P, T, H)
+    emin, emax = o.calibrate(x, 0.9, True)
+    sel = o.select_topk(emin, emax, k)
+    assert (sel["scale"] < 2.0 ** -109).any() and (sel["scale"] > 1e-10).any()
+    prm = params_to_dev(sel)
+    codes_r, side_r = o.quantize_pack(x, sel["keep_idx"], sel["rest_idx"], sel["inv_scale"], sel["zero"])
+    out_r = o.dequant_reduce(codes_r, side_r, H, sel["keep_idx"], sel["rest_idx"], sel["scale"], sel["zero"], out_f32=True)
+    xd = to_dev_u16(x)
+    codes, side = gpu_quantize(xd, prm)
+    out = gpu_dequant(codes, side, prm, H, out_f32=True)
+    fused, _, _ = gpu_fused(xd, prm, out_f32=True)
+    assert_no_device_error()
+    assert np.array_equal(u32(codes), codes_r)
+    assert np.array_equal(f32bits(out), f32bits(out_r))
+    assert np.array_equal(f32bits(fused), f32bits(out_r))
+
+
 def test_empty_rows_are_no_ops():
     prm = params_to_dev(oracle.get().select_topk(-np.ones((2, 64), np.float32), np.ones((2, 64), np.float32), 8))
     x = torch.empty((2, 0, 64), dtype=torch.int16, device=DEV)
@@ -137,6 +163,18 @@ def test_empty_rows_are_no_ops():
     fused, _, _ = gpu_fused(x, prm)
     assert out.numel() == 0 and fused.numel() == 0
     assert_no_device_error()
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    """A pipeline wait that nothing satisfies gives up after its limit, records HQ_ERR_TIMEOUT,
+    and the context keeps working (no trap, no hang)."""
+    assert hq.hq_read_device_error() == hq.HQ_OK
+    hq.hq_selftest_bounded_wait(2_000_000)  # ~1 ms
+    assert hq.hq_read_device_error() == hq.HQ_ERR_TIMEOUT
+    assert hq.hq_read_device_error() == hq.HQ_OK
+    cfg = synth.CONFIGS["pr1"]
+    cs, _ = synth.colscale(cfg)
+    compare_all(cfg, _batches(cfg, cs), synth.fill_cpu(cfg, synth.EVAL, 0, cs=cs))
 
 
 def test_bad_index_is_recorded_not_dereferenced():
