@@ -180,8 +180,9 @@ __device__ __forceinline__ void dq_decode_rows(const DqLane& D, const uint32_t* 
     float q[8];
     if (kFast) {
       const uint32_t v2 = v >> D.sh2;
+      const uint32_t magic = 0x4B000000u;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) q[i] = __uint_as_float(((i < 5 ? v : v2) & D.key[i]) | 0x4B000000u);
+      for (int i = 0; i < 8; ++i) q[i] = __uint_as_float(and_or(i < 5 ? v : v2, D.key[i], magic));
     } else {
 #pragma unroll
       for (int i = 0; i < 8; ++i) q[i] = __uint_as_float(((v >> D.key[i]) & 0xFu) | 0x4B000000u);
@@ -363,12 +364,14 @@ __global__ void __launch_bounds__(kDtThreads, 2) dequant_reduce_tma_kernel(
   // staged kept sums: pair p = lane + 32c (c < n_slots) is (row p & 3, kept feature p >> 2);
   // koff[c] = its element offset inside a stage's side tile
   const int n_pairs = stage_side ? kDqR * nk : 0;
-  const int n_slots = (n_pairs + 31) >> 5;
+  const int n_slots = (n_pairs + 31) >> 5;  // the same in every lane
+  // A lane without a pair in a slot reads element 0 of the stage into an accumulator it never
+  // uses, so the slot loop has no per-lane branch.
   int koff[3];
 #pragma unroll
   for (int c = 0; c < 3; ++c) {
     const int p = lane + 32 * c;
-    koff[c] = (p < n_pairs) ? (warp * kDqR + (p & 3)) * kDtSideCols + (q.ja - j_a + (p >> 2)) : -1;
+    koff[c] = (p < n_pairs) ? (warp * kDqR + (p & 3)) * kDtSideCols + (q.ja - j_a + (p >> 2)) : 0;
   }
   int i = 0;
   for (int bi = 0; bi < nblk && !*abort; ++bi) {
@@ -393,10 +396,9 @@ __global__ void __launch_bounds__(kDtThreads, 2) dequant_reduce_tma_kernel(
         else dq_decode_rows<true>(D, st, kDtWords, cst, acc);
       }
       const uint16_t* sside = &sm.side[st_i][0][0];
-#pragma unroll
-      for (int c = 0; c < 3; ++c) {
-        if (c < n_slots && koff[c] >= 0) kacc[c] = __fadd_rn(kacc[c], __uint_as_float((uint32_t)sside[koff[c]] << 16));
-      }
+      if (n_slots > 0) kacc[0] = __fadd_rn(kacc[0], __uint_as_float((uint32_t)sside[koff[0]] << 16));
+      if (n_slots > 1) kacc[1] = __fadd_rn(kacc[1], __uint_as_float((uint32_t)sside[koff[1]] << 16));
+      if (n_slots > 2) kacc[2] = __fadd_rn(kacc[2], __uint_as_float((uint32_t)sside[koff[2]] << 16));
       __syncwarp();
       if (lane == 0) sm.ring.release(i);
     }
