@@ -66,30 +66,38 @@ __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
 }
 
-// Packed fp32 pairs (sm_100): each lane of add/fma.rn.f32x2 is one correctly rounded IEEE
-// operation, so results are bit-identical to the scalar __fadd_rn / __fmaf_rn; one instruction
-// does two of them.
+// Packed fp32 pairs (sm_100 f32x2 instructions): each lane of __fadd2_rn / __fmul2_rn /
+// __ffma2_rn is one correctly rounded IEEE operation, so results are bit-identical to the scalar
+// __fadd_rn / __fmul_rn / __fmaf_rn; one instruction does two of them.
 __device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
-  asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+  const float2 r = __fadd2_rn(make_float2(a0, a1), make_float2(b0, b1));
+  d0 = r.x;
+  d1 = r.y;
 }
 __device__ __forceinline__ void fmul2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
-  asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+  const float2 r = __fmul2_rn(make_float2(a0, a1), make_float2(b0, b1));
+  d0 = r.x;
+  d1 = r.y;
 }
 // (d0, d1) = (a0*b0 + d0, a1*b1 + d1), each with one rounding.
 __device__ __forceinline__ void ffma2_acc(float& d0, float& d1, float a0, float a1, float b0, float b1) {
-  asm("{\n\t.reg .b64 ra, rb, rc;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-      "mov.b64 rc, {%0, %1};\n\tfma.rn.f32x2 rc, ra, rb, rc;\n\tmov.b64 {%0, %1}, rc;\n\t}"
-      : "+f"(d0), "+f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+  const float2 r = __ffma2_rn(make_float2(a0, a1), make_float2(b0, b1), make_float2(d0, d1));
+  d0 = r.x;
+  d1 = r.y;
 }
 
 // (a & b) | c in one LOP3.
 __device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {
   uint32_t d;
   asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// (a & M) | c in one LOP3 with M as its immediate operand (c stays in a register).
+template <uint32_t M>
+__device__ __forceinline__ uint32_t and_or_imm(uint32_t a, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "n"(M), "r"(c));
   return d;
 }
 

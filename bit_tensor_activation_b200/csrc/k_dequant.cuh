@@ -89,7 +89,6 @@ struct DqLane {
   int h0;
   bool active;
   bool decode;       // active and at least one non-kept feature
-  bool has_hi;       // the group's second word exists
   int my_w;          // first word of the group inside a staged row
   int fsh;           // funnel shift bringing the group's first nibble to bit 0
   int sh2;           // fast path: v2 = v >> sh2
@@ -114,7 +113,6 @@ __device__ __forceinline__ DqLane dq_lane(const int32_t* __restrict__ keep_idx, 
   const int Wr = (H - k) / 8;
   D.my_w = (D.L.c0 >> 3) - w_base;
   D.fsh = 4 * (D.L.c0 & 7);
-  D.has_hi = (D.L.c0 >> 3) + 1 < Wr;
   D.decode = D.active && D.L.n > 0;
   return D;
 }
@@ -165,17 +163,20 @@ __device__ __forceinline__ void dq_fill_constants(float4* s_const, const int32_t
   }
 }
 
-// Adds one rank's contribution for kDqR staged rows (row m at st + m * stride words).
-template <bool kFast>
+// Adds one rank's contribution for R staged rows (row m at st + m * stride words).
+template <bool kFast, int R>
 __device__ __forceinline__ void dq_decode_rows(const DqLane& D, const uint32_t* __restrict__ st, int stride,
-                                               const float4* __restrict__ cst, float (&acc)[kDqR][8]) {
+                                               const float4* __restrict__ cst, float (&acc)[R][8]) {
   const float4 s0 = cst[0], s1 = cst[32], o0 = cst[64], o1 = cst[96];
   const float sc[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
   const float off[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
 #pragma unroll
-  for (int m = 0; m < kDqR; ++m) {
+  for (int m = 0; m < R; ++m) {
     const uint32_t wlo = st[m * stride + D.my_w];
-    const uint32_t whi = D.has_hi ? st[m * stride + D.my_w + 1] : 0u;
+    // The next word is always inside the staged row (zero past the last code word of a row, or
+    // unused words of the staging window); its bits only reach v above the group's nibbles
+    // when the group fits in wlo.
+    const uint32_t whi = st[m * stride + D.my_w + 1];
     const uint32_t v = __funnelshift_r(wlo, whi, D.fsh);
     float q[8];
     if (kFast) {
@@ -197,7 +198,8 @@ __device__ __forceinline__ void dq_decode_rows(const DqLane& D, const uint32_t* 
 }
 
 // Owners of kept features ja+kc .. ja+kc+kw-1 take their sums from kept[m * 32 + (j - ja - kc)].
-__device__ __forceinline__ void dq_patch_kept(const DqLane& D, float (&acc)[kDqR][8], const float* kept, int ja,
+template <int R>
+__device__ __forceinline__ void dq_patch_kept(const DqLane& D, float (&acc)[R][8], const float* kept, int ja,
                                               int kc, int kw) {
   if (D.L.kmask) {
     int jk = D.L.j0;
@@ -207,7 +209,7 @@ __device__ __forceinline__ void dq_patch_kept(const DqLane& D, float (&acc)[kDqR
         const int jj = jk - ja - kc;
         if (jj >= 0 && jj < kw) {
 #pragma unroll
-          for (int m = 0; m < kDqR; ++m) acc[m][i] = kept[m * 32 + jj];
+          for (int m = 0; m < R; ++m) acc[m][i] = kept[m * 32 + jj];
         }
         ++jk;
       }
@@ -215,24 +217,24 @@ __device__ __forceinline__ void dq_patch_kept(const DqLane& D, float (&acc)[kDqR
   }
 }
 
-template <typename OutT>
-__device__ __forceinline__ void dq_store_rows(const DqLane& D, const float (&acc)[kDqR][8], int H, int t0,
+template <typename OutT, int R>
+__device__ __forceinline__ void dq_store_rows(const DqLane& D, const float (&acc)[R][8], int H, int t0,
                                               int t_last, OutT* __restrict__ out) {
   if (D.active) {
 #pragma unroll
-    for (int m = 0; m < kDqR; ++m) {
+    for (int m = 0; m < R; ++m) {
       const int t = t0 + m;
       if (t < t_last) store_row8<OutT>(out + (size_t)t * H + D.h0, acc[m]);
     }
   }
 }
 
-// Kept features of the warp's slice for rows t0..t0+kDqR-1, read from global memory:
+// Kept features of the warp's slice for rows t0..t0+R-1, read from global memory:
 // (row, kept feature) pairs over the lanes sum the P side values in rank order; owners copy them
-// into their sums; then the rows are stored.  Warp-level only (uses `kept`, kDqR x 32 floats of
+// into their sums; then the rows are stored.  Warp-level only (uses `kept`, R x 32 floats of
 // shared memory per warp).
-template <typename OutT>
-__device__ __forceinline__ void dq_finish_block(const DqLane& D, float (&acc)[kDqR][8],
+template <typename OutT, int R>
+__device__ __forceinline__ void dq_finish_block(const DqLane& D, float (&acc)[R][8],
                                                 const uint16_t* __restrict__ side, float* kept, int P,
                                                 int T, int H, int k, int ja, int jb, int t0, int t_last,
                                                 OutT* __restrict__ out) {
@@ -240,7 +242,7 @@ __device__ __forceinline__ void dq_finish_block(const DqLane& D, float (&acc)[kD
   const int nk = jb - ja;
   for (int kc = 0; kc < nk; kc += 32) {
     const int kw = min(32, nk - kc);
-    for (int p = lane; p < kDqR * kw; p += 32) {
+    for (int p = lane; p < R * kw; p += 32) {
       const int m = p / kw, jj = p - m * kw;
       const int t = t0 + m;
       float a = 0.0f;
@@ -254,10 +256,10 @@ __device__ __forceinline__ void dq_finish_block(const DqLane& D, float (&acc)[kD
       kept[m * 32 + jj] = a;
     }
     __syncwarp();
-    dq_patch_kept(D, acc, kept, ja, kc, kw);
+    dq_patch_kept<R>(D, acc, kept, ja, kc, kw);
     __syncwarp();
   }
-  dq_store_rows<OutT>(D, acc, H, t0, t_last, out);
+  dq_store_rows<OutT, R>(D, acc, H, t0, t_last, out);
 }
 
 // Slice bookkeeping shared by both kernels.
@@ -280,20 +282,27 @@ __device__ __forceinline__ DqSlice dq_slice(const int32_t* __restrict__ keep_idx
 }
 
 // ======================================================================== TMA kernel (default)
+// A ring slot holds the code tiles (and side tiles) of kDtG consecutive ranks for one block of
+// rows, so a consumer warp waits and releases once per kDtG ranks, and the rank loop inside a
+// slot has no synchronisation in it.
 constexpr int kDtWarps = 8;                      // consumer warps
 constexpr int kDtThreads = 32 * (kDtWarps + 1);  // + one producer warp
-constexpr int kDtTileRows = kDtWarps * kDqR;     // 32
+constexpr int kDtR = 4;                          // rows per consumer warp per block
+constexpr int kDtMinBlocks = 2;                  // CTAs per SM the register budget is set for
+constexpr int kDtTileRows = kDtWarps * kDtR;     // 32
 constexpr int kDtWords = 40;                     // staged words per row (box inner dim)
-constexpr int kDtStages = 8;
+constexpr int kDtG = 4;                          // ranks per ring slot
+constexpr int kDtStages = 3;
 constexpr unsigned kDtTileBytes = kDtTileRows * kDtWords * 4;
 constexpr int kDtSideCols = 32;                  // side box width (bf16): kept features staged per slice
-constexpr int kDtMaxStagedKept = 24;             // slices with more kept features read them from HBM
+constexpr int kDtKeptSlots = 3;                  // (row, kept feature) pairs per lane
+constexpr int kDtMaxStagedKept = 32 * kDtKeptSlots / kDtR;  // slices with more read them from HBM
 constexpr unsigned kDtSideBytes = kDtTileRows * kDtSideCols * 2;
 
 struct DtSmem {
-  alignas(128) uint32_t tile[kDtStages][kDtTileRows][kDtWords];
-  alignas(128) uint16_t side[kDtStages][kDtTileRows][kDtSideCols];
-  float kept[kDtWarps][kDqR * 32];
+  alignas(128) uint32_t tile[kDtStages][kDtG][kDtTileRows][kDtWords];
+  alignas(128) uint16_t side[kDtStages][kDtG][kDtTileRows][kDtSideCols];
+  float kept[kDtWarps][kDtR * 32];
   TmaRing<kDtStages> ring;
   int abort;
   // followed by the constants: float4 [P][4][32]
@@ -301,8 +310,26 @@ struct DtSmem {
 
 inline size_t dt_smem_bytes(int P) { return sizeof(DtSmem) + 128 + (size_t)P * 4 * 32 * 16; }
 
+// The nr ranks of one ring slot, in rank order: 4-bit features of the warp's rows into acc
+// (cst = this lane's constants of the slot's first rank), the first NS kept-pair slots into
+// kacc.
+template <bool kFast, int NS>
+__device__ __forceinline__ void dt_slot(const DqLane& D, const DtSmem& sm, int st_i, int warp, int nr,
+                                        const float4* __restrict__ cst, const int (&koff)[kDtKeptSlots],
+                                        float (&acc)[kDtR][8], float (&kacc)[kDtKeptSlots]) {
+#pragma unroll
+  for (int j = 0; j < kDtG; ++j) {
+    if (j < nr) {
+      if (D.decode) dq_decode_rows<kFast, kDtR>(D, &sm.tile[st_i][j][warp * kDtR][0], kDtWords, cst + j * 4 * 32, acc);
+      const uint16_t* sside = &sm.side[st_i][j][0][0];
+#pragma unroll
+      for (int c = 0; c < NS; ++c) kacc[c] = __fadd_rn(kacc[c], __uint_as_float((uint32_t)sside[koff[c]] << 16));
+    }
+  }
+}
+
 template <typename OutT>
-__global__ void __launch_bounds__(kDtThreads, 2) dequant_reduce_tma_kernel(
+__global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_kernel(
     const __grid_constant__ CUtensorMap tmap_codes, const __grid_constant__ CUtensorMap tmap_side,
     const uint16_t* __restrict__ side, int P, int T, int H,
     int k, const int32_t* __restrict__ keep_idx, const float* __restrict__ scale,
@@ -315,7 +342,8 @@ __global__ void __launch_bounds__(kDtThreads, 2) dequant_reduce_tma_kernel(
   const int s = blockIdx.x / chunks, chunk = blockIdx.x - s * chunks;
   const int t_first = chunk * rows_per_chunk, t_last = min(T, t_first + rows_per_chunk);
   const int nblk = (t_last - t_first + kDtTileRows - 1) / kDtTileRows;
-  const int n_tiles = nblk * P;  // tile i = (block i / P, rank i % P)
+  const int n_groups = (P + kDtG - 1) / kDtG;  // ring slots per block
+  const int n_slots_total = nblk * n_groups;     // slot i = (block i / n_groups, rank group i % n_groups)
 
   const DqSlice q = dq_slice(keep_idx, H, k, s, S);
   const int w_a = q.w_first & ~3;  // 16-byte aligned x coordinate of the box
@@ -334,17 +362,20 @@ __global__ void __launch_bounds__(kDtThreads, 2) dequant_reduce_tma_kernel(
     if (lane == 0) {
       prefetch_tensor_map(&tmap_codes);
       if (stage_side) prefetch_tensor_map(&tmap_side);
-      int issued = 0, bi = 0, r = 0;
-      for (int i = 0; i < n_tiles; ++i) {
+      int issued = 0, bi = 0, g = 0;
+      for (int i = 0; i < n_slots_total; ++i) {
         if (!sm.ring.acquire(i, abort, wait_limit)) break;
         const int st = i % kDtStages;
-        const int row = r * T + t_first + bi * kDtTileRows;
-        mbar_arrive_expect_tx(&sm.ring.full[st], kDtTileBytes + (stage_side ? kDtSideBytes : 0u));
-        tma_load_2d(&sm.tile[st][0][0], &tmap_codes, w_a, row, &sm.ring.full[st]);
-        if (stage_side) tma_load_2d(&sm.side[st][0][0], &tmap_side, j_a, row, &sm.ring.full[st]);
+        const int r0 = g * kDtG, nr = min(kDtG, P - r0);
+        mbar_arrive_expect_tx(&sm.ring.full[st], (unsigned)nr * (kDtTileBytes + (stage_side ? kDtSideBytes : 0u)));
+        for (int j = 0; j < nr; ++j) {
+          const int row = (r0 + j) * T + t_first + bi * kDtTileRows;
+          tma_load_2d(&sm.tile[st][j][0][0], &tmap_codes, w_a, row, &sm.ring.full[st]);
+          if (stage_side) tma_load_2d(&sm.side[st][j][0][0], &tmap_side, j_a, row, &sm.ring.full[st]);
+        }
         ++issued;
-        if (++r == P) {
-          r = 0;
+        if (++g == n_groups) {
+          g = 0;
           ++bi;
         }
       }
@@ -361,60 +392,68 @@ __global__ void __launch_bounds__(kDtThreads, 2) dequant_reduce_tma_kernel(
   const DqLane D = dq_lane(keep_idx, k, H, s, lane, w_a, generic);
   named_barrier_sync(kConsumers);
   float* kept = sm.kept[warp];
-  // staged kept sums: pair p = lane + 32c (c < n_slots) is (row p & 3, kept feature p >> 2);
-  // koff[c] = its element offset inside a stage's side tile
-  const int n_pairs = stage_side ? kDqR * nk : 0;
-  const int n_slots = (n_pairs + 31) >> 5;  // the same in every lane
-  // A lane without a pair in a slot reads element 0 of the stage into an accumulator it never
-  // uses, so the slot loop has no per-lane branch.
-  int koff[3];
+  // staged kept sums: pair p = lane + 32c (c < n_slots) is (row p % kDtR, kept feature p / kDtR);
+  // koff[c] = its element offset inside a rank's side tile.  n_slots is the same in every lane;
+  // a lane without a pair in a slot reads element 0 of the tile into a sum it never uses, so
+  // the slot loop has no per-lane branch.
+  const int n_pairs = stage_side ? kDtR * nk : 0;
+  const int n_slots = (n_pairs + 31) >> 5;
+  int koff[kDtKeptSlots];
 #pragma unroll
-  for (int c = 0; c < 3; ++c) {
+  for (int c = 0; c < kDtKeptSlots; ++c) {
     const int p = lane + 32 * c;
-    koff[c] = (p < n_pairs) ? (warp * kDqR + (p & 3)) * kDtSideCols + (q.ja - j_a + (p >> 2)) : 0;
+    koff[c] = (p < n_pairs) ? (warp * kDtR + p % kDtR) * kDtSideCols + (q.ja - j_a + p / kDtR) : 0;
   }
-  int i = 0;
+  int st_i = 0;
+  unsigned phase = 0;
   for (int bi = 0; bi < nblk && !*abort; ++bi) {
-    const int t0 = t_first + bi * kDtTileRows + warp * kDqR;
-    float acc[kDqR][8];
+    const int t0 = t_first + bi * kDtTileRows + warp * kDtR;
+    float acc[kDtR][8];
 #pragma unroll
-    for (int m = 0; m < kDqR; ++m)
+    for (int m = 0; m < kDtR; ++m)
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[m][e] = 0.0f;
-    float kacc[3] = {0.0f, 0.0f, 0.0f};
+    float kacc[kDtKeptSlots];
+#pragma unroll
+    for (int c = 0; c < kDtKeptSlots; ++c) kacc[c] = 0.0f;
     bool ok = true;
-    for (int r = 0; r < P; ++r, ++i) {
-      if (!sm.ring.wait_full(i, abort, wait_limit)) {
+    for (int g = 0; g < n_groups; ++g) {
+      if (!mbar_wait(&sm.ring.full[st_i], phase, abort, wait_limit)) {
         ok = false;
         break;
       }
-      const int st_i = i % kDtStages;
-      const uint32_t* st = &sm.tile[st_i][warp * kDqR][0];
-      const float4* cst = s_const + (size_t)r * 4 * 32 + lane;
-      if (D.decode) {
-        if (generic) dq_decode_rows<false>(D, st, kDtWords, cst, acc);
-        else dq_decode_rows<true>(D, st, kDtWords, cst, acc);
+      const int nr = min(kDtG, P - g * kDtG);
+      const float4* cst = s_const + (size_t)g * kDtG * 4 * 32 + lane;
+      if (generic) {
+        dt_slot<false, kDtKeptSlots>(D, sm, st_i, warp, nr, cst, koff, acc, kacc);
+      } else {
+        switch (n_slots) {  // the same in every lane of the CTA
+          case 0: dt_slot<true, 0>(D, sm, st_i, warp, nr, cst, koff, acc, kacc); break;
+          case 1: dt_slot<true, 1>(D, sm, st_i, warp, nr, cst, koff, acc, kacc); break;
+          case 2: dt_slot<true, 2>(D, sm, st_i, warp, nr, cst, koff, acc, kacc); break;
+          default: dt_slot<true, kDtKeptSlots>(D, sm, st_i, warp, nr, cst, koff, acc, kacc); break;
+        }
       }
-      const uint16_t* sside = &sm.side[st_i][0][0];
-      if (n_slots > 0) kacc[0] = __fadd_rn(kacc[0], __uint_as_float((uint32_t)sside[koff[0]] << 16));
-      if (n_slots > 1) kacc[1] = __fadd_rn(kacc[1], __uint_as_float((uint32_t)sside[koff[1]] << 16));
-      if (n_slots > 2) kacc[2] = __fadd_rn(kacc[2], __uint_as_float((uint32_t)sside[koff[2]] << 16));
       __syncwarp();
-      if (lane == 0) sm.ring.release(i);
+      if (lane == 0) mbar_arrive(&sm.ring.empty[st_i]);
+      if (++st_i == kDtStages) {
+        st_i = 0;
+        phase ^= 1u;
+      }
     }
     if (!ok) break;
     if (stage_side) {
 #pragma unroll
-      for (int c = 0; c < 3; ++c) {
+      for (int c = 0; c < kDtKeptSlots; ++c) {
         const int p = lane + 32 * c;
-        if (p < n_pairs) kept[(p & 3) * 32 + (p >> 2)] = kacc[c];
+        if (p < n_pairs) kept[(p % kDtR) * 32 + p / kDtR] = kacc[c];
       }
       __syncwarp();
-      dq_patch_kept(D, acc, kept, q.ja, 0, nk);
+      dq_patch_kept<kDtR>(D, acc, kept, q.ja, 0, nk);
       __syncwarp();
-      dq_store_rows<OutT>(D, acc, H, t0, t_last, out);
+      dq_store_rows<OutT, kDtR>(D, acc, H, t0, t_last, out);
     } else {
-      dq_finish_block<OutT>(D, acc, side, kept, P, T, H, k, q.ja, q.jb, t0, t_last, out);
+      dq_finish_block<OutT, kDtR>(D, acc, side, kept, P, T, H, k, q.ja, q.jb, t0, t_last, out);
     }
   }
 }
@@ -501,12 +540,12 @@ __global__ void __launch_bounds__(kDqThreads) dequant_reduce_kernel(
       const uint32_t* st = my_tiles + (size_t)(tile % kDqD) * kDqR * kDqWin;
       const float4* cst = s_const + (size_t)r * 4 * 32 + lane;
       if (D.decode) {
-        if (generic) dq_decode_rows<false>(D, st, kDqWin, cst, acc);
-        else dq_decode_rows<true>(D, st, kDqWin, cst, acc);
+        if (generic) dq_decode_rows<false, kDqR>(D, st, kDqWin, cst, acc);
+        else dq_decode_rows<true, kDqR>(D, st, kDqWin, cst, acc);
       }
       __syncwarp();  // the stage is free for the copy issued next iteration
     }
-    dq_finish_block<OutT>(D, acc, side, my_kept, P, T, H, k, q.ja, q.jb, t0, t_last, out);
+    dq_finish_block<OutT, kDqR>(D, acc, side, my_kept, P, T, H, k, q.ja, q.jb, t0, t_last, out);
   }
   cp_async_wait<0>();
 }
