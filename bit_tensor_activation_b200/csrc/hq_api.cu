@@ -17,7 +17,6 @@
 #include "k_dequant.cuh"
 #include "k_fused.cuh"
 #include "k_quantize.cuh"
-#include "k_quantize_tma.cuh"
 #include "k_select.cuh"
 
 namespace {
@@ -37,7 +36,6 @@ hq_status check_shape(int P, int H, int k) {
 // Launch-shape facts cached per device: SM count and resident CTAs per SM of each kernel.
 struct DeviceInfo {
   int sms = 0;
-  int qp_blocks = 0;
   int qt_blocks = 0;
   bool select_smem_set = false;
 };
@@ -82,13 +80,6 @@ hq_status device_info(DeviceInfo** out) {
   if (d.sms == 0) {
     if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return HQ_ERR_CUDA;
-    const int qp_smem = (int)(hq::kQpWarps * sizeof(hq::QpWarpSmem));
-    if (cudaFuncSetAttribute(hq::quantize_pack_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             qp_smem) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.qp_blocks, hq::quantize_pack_kernel,
-                                                      hq::kQpThreads, qp_smem) != cudaSuccess)
-      return HQ_ERR_CUDA;
-    if (d.qp_blocks < 1) d.qp_blocks = 1;
     const int qt_smem = (int)(sizeof(hq::QtSmem) + 128);
     if (cudaFuncSetAttribute(hq::quantize_pack_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              qt_smem) != cudaSuccess ||
@@ -252,31 +243,19 @@ hq_status hq_quantize_pack(const uint16_t* x, int P, int T, int H, int k, const 
   if (T == 0) return HQ_OK;
   DeviceInfo* d = nullptr;
   if (device_info(&d) != HQ_OK) return HQ_ERR_CUDA;
-  {
-    const int S = (H + hq::kQtSlice - 1) / hq::kQtSlice;
-    CUtensorMap map_x, map_halo;
-    if (!encode_2d(&map_x, x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)H, (uint64_t)P * T, hq::kQtSlice,
-                   hq::kQtTileRows) ||
-        !encode_2d(&map_halo, x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)H, (uint64_t)P * T, hq::kQtHalo,
-                   hq::kQtTileRows, CU_TENSOR_MAP_L2_PROMOTION_NONE))  // 32-byte rows: no 256-byte over-fetch
-      return HQ_ERR_CUDA;
-    int chunks, rpc;
-    slice_chunks(T, S, (long long)d->sms * d->qt_blocks, hq::kQtTileRows, &chunks, &rpc);
-    hq::quantize_pack_tma_kernel<<<(unsigned)(S * chunks), hq::kQtThreads, sizeof(hq::QtSmem) + 128,
-                                   (cudaStream_t)stream>>>(map_x, map_halo, x, P, T, H, k, keep_idx, rest_idx,
-                                                           inv_scale, zero, codes, side, S, chunks, rpc,
-                                                           hq::kWaitLimitCycles);
-    return launched();
-  }
-  const int S = (H + 8 * hq::kQpSliceGroups - 1) / (8 * hq::kQpSliceGroups);
-  const long long units = (long long)P * S * T;
-  // one warp per resident warp slot, at least kQpR rows each
-  long long warps = (long long)d->sms * d->qp_blocks * hq::kQpWarps;
-  long long per = ceil_div(units, warps);
-  if (per < hq::kQpR) per = hq::kQpR;
-  const unsigned grid = (unsigned)ceil_div(ceil_div(units, per), hq::kQpWarps);
-  hq::quantize_pack_kernel<<<grid, hq::kQpThreads, hq::kQpWarps * sizeof(hq::QpWarpSmem), (cudaStream_t)stream>>>(
-      x, P, T, H, k, keep_idx, rest_idx, inv_scale, zero, codes, side, S, per);
+  const int S = (H + hq::kQtSlice - 1) / hq::kQtSlice;
+  CUtensorMap map_x, map_halo;
+  if (!encode_2d(&map_x, x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)H, (uint64_t)P * T, hq::kQtSlice,
+                 hq::kQtTileRows) ||
+      !encode_2d(&map_halo, x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)H, (uint64_t)P * T, hq::kQtHalo,
+                 hq::kQtTileRows, CU_TENSOR_MAP_L2_PROMOTION_NONE))  // 32-byte rows: no 256-byte over-fetch
+    return HQ_ERR_CUDA;
+  int chunks, rpc;
+  slice_chunks(T, S, (long long)d->sms * d->qt_blocks, hq::kQtTileRows, &chunks, &rpc);
+  hq::quantize_pack_tma_kernel<<<(unsigned)(S * chunks), hq::kQtThreads, sizeof(hq::QtSmem) + 128,
+                                 (cudaStream_t)stream>>>(map_x, map_halo, x, P, T, H, k, keep_idx, rest_idx,
+                                                         inv_scale, zero, codes, side, S, chunks, rpc,
+                                                         hq::kWaitLimitCycles);
   return launched();
 }
 

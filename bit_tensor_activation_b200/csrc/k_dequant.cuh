@@ -110,7 +110,6 @@ __device__ __forceinline__ DqLane dq_lane(const int32_t* __restrict__ keep_idx, 
     const bool kept = (D.L.kmask >> i) & 1u;
     D.key[i] = generic ? (uint32_t)(4 * jpos[i]) : (kept ? 0u : (0xFu << (4 * pos[i])));
   }
-  const int Wr = (H - k) / 8;
   D.my_w = (D.L.c0 >> 3) - w_base;
   D.fsh = 4 * (D.L.c0 & 7);
   D.decode = D.active && D.L.n > 0;

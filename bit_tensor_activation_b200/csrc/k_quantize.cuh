@@ -4,218 +4,314 @@
 // become 4-bit codes q = clamp(rint(x*inv_scale)+zero, 0, 15) packed 8 per uint32 in rest_idx
 // order.
 //
-// Work decomposition.  A warp owns a slice of 32 groups of 8 consecutive features (256 features,
-// one group per lane).  A work unit is one row of one rank restricted to one slice; units are
-// laid out rank-major, then slice, then row, and every warp of a persistent grid takes one
-// contiguous run of them, so it changes (rank, slice) rarely and keeps its features' parameters
-// in registers in between.  Warps never wait for one another.
+// Work decomposition.  A CTA owns one slice of 256 features and one chunk of rows, and walks the
+// ranks (outer) and the chunk's 32-row blocks (inner); a work unit is one (rank, row block).  The
+// grid is one wave of slices x chunks, so the CTAs of the S slices of a chunk write the same rows
+// of codes and side at about the same time: the 32-byte sectors those rows share at slice
+// boundaries are completed in L2 before eviction instead of costing a read-modify-write in HBM
+// each time.  In a CTA, warp 8 is the producer: one lane issues, per unit, a TMA load of the
+// 32 x 256 bf16 tile (16 KB) plus, when the slice has halo features and they lie within 32
+// columns, a 32 x 32 tile holding them (a second tensor map with that box), into a 4-stage ring.
+// Warps 0..7 are consumers; warp w quantizes rows 4w..4w+3 of each tile, lane l the 8 features
+// 8l..8l+7 (parameters in registers, reloaded only when the unit's rank changes).
 //
-// Data movement.  Each lane stages its own 16 bytes of kQpR rows per tile into shared memory
-// with cp.async, kQpD - 1 tiles ahead of the tile it computes; a lane only reads what it copied,
-// so its own cp.async.wait_group (a hardware wait) is the only synchronisation the data needs.
-//
-// Per lane: inv_scale, the clamp bound -zero and a nibble multiplier 16^j (0 for a kept feature,
-// j = the feature's rank among the group's non-kept ones) for its 8 features.  The group's code
-// word is V = sum_i (zero_i + clamp_i) * 16^j_i: every nibble stays in [0,15], so the sum is the
-// packed word of the group's n non-kept codes.  Its compact position c0 is in general not a
-// multiple of 8, so V is split across two words and OR-ed into a per-warp word buffer in shared
-// memory.
+// Packing.  Per lane: inv_scale, the clamp bounds -zero and 15-zero and a nibble multiplier 16^j
+// (0 for a kept feature, j = the feature's rank among the group's non-kept ones) for its 8
+// features.  The group's code word is V = sum_i (zero_i + clamp_i) * 16^j_i: every nibble stays
+// in [0,15], so the sum is the packed word of the group's n non-kept codes.  Its compact position
+// c0 is in general not a multiple of 8, so V is split across two words and OR-ed into a per-warp
+// word buffer in shared memory, from which whole words are stored with coalesced 32-bit stores.
 //
 // Ownership of compact words: a slice owns the words whose first nibble one of its groups
 // produces; it drops nibbles that fall into the previous slice's last word and completes its own
-// last word from the next <= 7 non-kept features of the next slice ("halo", read through
-// rest_idx, one lane each).  So every codes word is written by exactly one warp with plain
-// coalesced stores.  Kept values are taken from the owner lane's staged row with shuffles.
+// last word from the next <= 7 non-kept features of the next slice (the "halo", read through
+// rest_idx, one lane each).  So every codes word is written by exactly one CTA.  Kept values are
+// copied from the staged tile to the side buffer.
 //
 // Roofline: HBM-bound; 2 bytes read + 0.5 byte written per non-kept element, 2 + 2 per kept one.
 // No memory beyond the inputs and outputs is used.
 #pragma once
 
 #include "hq_common.cuh"
+#include "hq_tma.cuh"
 
 namespace hq {
 
-constexpr int kQpWarps = 8;
-constexpr int kQpThreads = 32 * kQpWarps;
-constexpr int kQpR = 4;              // rows per tile
-constexpr int kQpD = 3;              // tiles staged per warp (kQpD - 1 in flight while computing)
-constexpr int kQpSliceGroups = 32;   // groups per warp slice
-constexpr int kQpBufWords = 36;      // >= 33 owned words + 2 guard slots per row
+constexpr int kQtWarps = 8;                             // consumer warps
+constexpr int kQtThreads = 32 * (kQtWarps + 1);         // + one producer warp
+constexpr int kQtRowsPerWarp = 4;
+constexpr int kQtTileRows = kQtWarps * kQtRowsPerWarp;  // 32
+constexpr int kQtStages = 4;
+constexpr int kQtSlice = 256;                           // features per slice (box inner dim)
+constexpr int kQtHalo = 32;                             // halo box width (features)
+constexpr int kQtBufWords = 36;                         // >= 33 owned words + 2 guard slots per row
+constexpr unsigned kQtTileBytes = kQtTileRows * kQtSlice * 2;
+constexpr unsigned kQtHaloBytes = kQtTileRows * kQtHalo * 2;
 
-struct QpWarpSmem {
-  uint4 rows[kQpD][kQpR][32];        // each lane's 16 bytes of each staged row
-  uint32_t halo[kQpD][kQpR][8];      // the 4-byte word holding each halo feature
-  uint32_t buf[kQpR][kQpBufWords];   // slot 1 + (word - Wb); slot 0 and slot nw + 1 are guards
+struct QtSmem {
+  alignas(128) uint16_t tile[kQtStages][kQtTileRows][kQtSlice];
+  alignas(128) uint16_t halo[kQtStages][kQtTileRows][kQtHalo];
+  uint32_t buf[kQtWarps][kQtRowsPerWarp][kQtBufWords];
+  TmaRing<kQtStages> ring;
+  int abort;
 };
 
-__global__ void __launch_bounds__(kQpThreads) quantize_pack_kernel(
-    const uint16_t* __restrict__ x, int P, int T, int H, int k, const int32_t* __restrict__ keep_idx,
-    const int32_t* __restrict__ rest_idx, const float* __restrict__ inv_scale,
-    const uint8_t* __restrict__ zero, uint32_t* __restrict__ codes, uint16_t* __restrict__ side,
-    int S, long long units_per_warp) {
-  extern __shared__ float4 s_dyn[];
+// Slice facts shared by the producer and the consumers.
+struct QtSlice {
+  int ha, hb, ja, jb, Ca, Cb, Wb, We, nw, nhalo;
+  int halo_c0;   // first column of the halo box (a multiple of 8)
+  bool halo_box; // every halo feature lies in [halo_c0, halo_c0 + kQtHalo)
+};
+
+__device__ __forceinline__ QtSlice qt_slice(const int32_t* __restrict__ keep_idx,
+                                            const int32_t* __restrict__ rest_idx, int H, int k, int s) {
+  QtSlice q;
+  const int Hr = H - k;
+  q.ha = s * kQtSlice;
+  q.hb = min(H, q.ha + kQtSlice);
+  q.ja = lower_bound_i32(keep_idx, k, q.ha);
+  q.jb = lower_bound_i32(keep_idx, k, q.hb);
+  q.Ca = min(max(q.ha - q.ja, 0), Hr);
+  q.Cb = min(max(q.hb - q.jb, 0), Hr);
+  q.Wb = (q.Ca + 7) >> 3;
+  q.We = (q.Cb + 7) >> 3;
+  q.nw = max(q.We - q.Wb, 0);
+  q.nhalo = (q.We > q.Wb) ? (8 * q.We - q.Cb) : 0;
+  q.halo_c0 = 0;
+  q.halo_box = true;
+  if (q.nhalo > 0) {
+    const int first = checked_col(rest_idx, q.Cb, H);
+    const int last = checked_col(rest_idx, q.Cb + q.nhalo - 1, H);
+    q.halo_c0 = first & ~7;
+    q.halo_box = last < q.halo_c0 + kQtHalo;
+  }
+  return q;
+}
+
+__global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
+    const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_halo,
+    const uint16_t* __restrict__ x, int P, int T, int H,
+    int k, const int32_t* __restrict__ keep_idx, const int32_t* __restrict__ rest_idx,
+    const float* __restrict__ inv_scale, const uint8_t* __restrict__ zero, uint32_t* __restrict__ codes,
+    uint16_t* __restrict__ side, int S, int chunks, int rows_per_chunk, long long wait_limit) {
+  extern __shared__ __align__(128) unsigned char s_raw[];
+  QtSmem& sm = *reinterpret_cast<QtSmem*>(s_raw);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  QpWarpSmem& W = reinterpret_cast<QpWarpSmem*>(s_dyn)[warp];
+  const int s = blockIdx.x / chunks, chunk = blockIdx.x - s * chunks;
+  const int t_first = chunk * rows_per_chunk, t_last = min(T, t_first + rows_per_chunk);
+  const int NBc = (t_last - t_first + kQtTileRows - 1) / kQtTileRows;  // row blocks of the chunk
+  const int n_units = NBc * P;                                         // unit i = (rank i / NBc, block i % NBc)
+
+  if (threadIdx.x == 0) {
+    sm.ring.init(kQtWarps);
+    sm.abort = 0;
+    fence_barrier_init();
+  }
+  for (int i = threadIdx.x; i < kQtWarps * kQtRowsPerWarp * kQtBufWords; i += kQtThreads)
+    (&sm.buf[0][0][0])[i] = 0u;
+  __syncthreads();
+  volatile int* abort = &sm.abort;
+
+  // ---------------------------------------------------------------- producer warp
+  if (warp == kQtWarps) {
+    if (lane == 0) {
+      prefetch_tensor_map(&tmap_x);
+      prefetch_tensor_map(&tmap_halo);
+      int issued = 0;
+      const QtSlice q = qt_slice(keep_idx, rest_idx, H, k, s);
+      int r = 0, b = 0;  // unit i = (rank r, row block b), advanced incrementally
+      for (int i = 0; i < n_units; ++i) {
+        if (i > 0 && ++b == NBc) {
+          b = 0;
+          ++r;
+        }
+        if (!sm.ring.acquire(i, abort, wait_limit)) break;
+        const int st = i % kQtStages;
+        const int row = r * T + t_first + b * kQtTileRows;
+        const bool halo = q.nhalo > 0 && q.halo_box;
+        mbar_arrive_expect_tx(&sm.ring.full[st], kQtTileBytes + (halo ? kQtHaloBytes : 0u));
+        tma_load_2d(&sm.tile[st][0][0], &tmap_x, q.ha, row, &sm.ring.full[st]);
+        if (halo) tma_load_2d(&sm.halo[st][0][0], &tmap_halo, q.halo_c0, row, &sm.ring.full[st]);
+        ++issued;
+      }
+      if (*abort) sm.ring.drain(issued, wait_limit);
+    }
+    return;
+  }
+
+  // ---------------------------------------------------------------- consumer warps
   const int Hr = H - k, Wr = Hr / 8, NG = H / 8;
-  const long long U = (long long)P * S * T;
+  int r = 0, b = 0;
+  bool fresh = true;  // rank changed: reload this lane's parameters
+  const QtSlice q = qt_slice(keep_idx, rest_idx, H, k, s);
+  if (threadIdx.x == 0 && ((s == 0 && q.ja != 0) || (s == S - 1 && q.jb != k))) record_error(HQ_ERR_BAD_INDEX);
+  GroupLayout L{0, 0, 0u, 0};
+  bool active = false;
+  float inv[8];
+  int lo[8], hi[8];
+  uint32_t mul[8], zbase = 0;
+  int slot = 0, sh = 0;
+  bool is_halo = false;
+  int h_row = 0, h_col = 0, h_lo = 0, h_z = 0, h_shift = 0, h_off = 0;
+  float h_inv = 0.0f;
+  // kept copies of this lane: pair p = lane + 32c (c < 3) is (row p & 3, kept feature p >> 2);
+  // k_off = tile element offset (-1: no pair), k_side = side element offset within the unit
+  bool k_generic = false;
+  int k_off[3] = {-1, -1, -1}, k_side[3] = {0, 0, 0};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    inv[i] = 0.0f;
+    lo[i] = hi[i] = 0;
+    mul[i] = 0u;
+  }
+  uint32_t(*buf)[kQtBufWords] = sm.buf[warp];
 
-  for (int i = lane; i < kQpR * kQpBufWords; i += 32) (&W.buf[0][0])[i] = 0u;
-  __syncwarp();
-
-  long long u = ((long long)blockIdx.x * kQpWarps + warp) * units_per_warp;
-  const long long u_end = min(U, u + units_per_warp);
-
-  while (u < u_end) {
-    const long long rs = u / T;
-    const int t_begin = (int)(u - rs * T);
-    const int t_stop = (int)min((long long)T, (long long)t_begin + (u_end - u));
-    const int r = (int)(rs / S), s = (int)(rs - (long long)r * S);
-
-    // ---- this lane's group: parameters in registers ----------------------------------------
-    const int g = s * kQpSliceGroups + lane;
-    const bool active = g < NG;
-    const int h0 = 8 * g;
-    GroupLayout L{0, 0, 0u, 0};
-    float inv[8];
-    int lo[8], hi[8];
-    uint32_t mul[8], zbase = 0;
-    if (active) L = group_layout(keep_idx, k, H, h0);
-    {
+  for (int i = 0; i < n_units; ++i) {
+    if (i > 0 && ++b == NBc) {
+      b = 0;
+      fresh = true;
+      ++r;
+    }
+    if (fresh) {  // new rank: this lane's parameters
+      fresh = false;
+      const int g = s * (kQtSlice / 8) + lane;
+      active = g < NG;
+      L = GroupLayout{0, 0, 0u, 0};
+      if (active) L = group_layout(keep_idx, k, H, 8 * g);
+      zbase = 0;
       int j = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const bool kept = (L.kmask >> i) & 1u;
+      for (int e = 0; e < 8; ++e) {
+        const bool kept = (L.kmask >> e) & 1u;
         int z = 0;
-        inv[i] = 0.0f;
+        inv[e] = 0.0f;
         if (active) {
-          const size_t p = (size_t)r * H + h0 + i;
+          const size_t p = (size_t)r * H + 8 * g + e;
           z = zero[p];
-          inv[i] = inv_scale[p];
+          inv[e] = inv_scale[p];
         }
-        lo[i] = -z;
-        hi[i] = 15 - z;
-        mul[i] = (active && !kept) ? (1u << (4 * j)) : 0u;
+        lo[e] = -z;
+        hi[e] = 15 - z;
+        mul[e] = (active && !kept) ? (1u << (4 * j)) : 0u;
         j += kept ? 0 : 1;
-        zbase += (uint32_t)z * mul[i];
+        zbase += (uint32_t)z * mul[e];
       }
-    }
-
-    // ---- slice ownership (the same values in every lane) ------------------------------------
-    const int ha = 8 * s * kQpSliceGroups, hb = min(H, ha + 8 * kQpSliceGroups);
-    const int ja = lower_bound_i32(keep_idx, k, ha), jb = lower_bound_i32(keep_idx, k, hb);
-    if (lane == 0 && ((s == 0 && ja != 0) || (s == S - 1 && jb != k))) record_error(HQ_ERR_BAD_INDEX);
-    const int Ca = min(max(ha - ja, 0), Hr), Cb = min(max(hb - jb, 0), Hr);
-    const int Wb = (Ca + 7) >> 3, We = (Cb + 7) >> 3;  // owned words [Wb, We)
-    const int nw = max(We - Wb, 0);                    // <= 33
-    const int nhalo = (We > Wb) ? (8 * We - Cb) : 0;   // 0..7 codes from the next slice
-    const int slot = (L.c0 >> 3) - Wb + 1;             // buffer slot of the group's first word
-    const int sh = 4 * (L.c0 & 7);
-
-    // halo work of a tile: lane p < nhalo*kQpR takes halo feature p % nhalo of row p / nhalo
-    const bool is_halo = lane < nhalo * kQpR;
-    const int h_row = is_halo ? lane / nhalo : 0, h_idx = is_halo ? lane - h_row * nhalo : 0;
-    float h_inv = 0.0f;
-    int h_col = 0, h_lo = 0, h_z = 0, h_shift = 0;
-    if (is_halo) {
-      h_col = checked_col(rest_idx, Cb + h_idx, H);
-      const size_t p = (size_t)r * H + h_col;
-      h_z = zero[p];
-      h_inv = inv_scale[p];
-      h_lo = -h_z;
-      h_shift = 4 * ((Cb + h_idx) & 7);
-    }
-    // kept work of a tile: pair p = jj * kQpR + m (rounds of 32 pairs)
-    const int nk = jb - ja;
-    const int npairs = nk * kQpR;
-
-    const uint16_t* xr = x + ((size_t)r * T) * H;
-    uint32_t* crow = codes + ((size_t)r * T) * Wr + Wb;
-    uint16_t* srow = side + ((size_t)r * T) * k;
-    const int n_tiles = (t_stop - t_begin + kQpR - 1) / kQpR;
-
-    int i_next = 0;
-    auto issue_next = [&]() {
-      if (i_next < n_tiles) {
-        const int stage = i_next % kQpD;
-        const int t0 = t_begin + i_next * kQpR;
-        const uint16_t* src = xr + (size_t)t0 * H;
-#pragma unroll
-        for (int m = 0; m < kQpR; ++m)
-          if (active && t0 + m < t_stop) cp_async16(smem_addr(&W.rows[stage][m][lane]), src + (size_t)m * H + h0);
-        if (is_halo && t0 + h_row < t_stop)
-          cp_async4(smem_addr(&W.halo[stage][h_row][h_idx]), src + (size_t)h_row * H + (h_col & ~1));
-        ++i_next;
+      slot = (L.c0 >> 3) - q.Wb + 1;
+      sh = 4 * (L.c0 & 7);
+      // halo work of a tile: lane p < nhalo*4 takes halo feature p % nhalo of row p / nhalo
+      is_halo = lane < q.nhalo * kQtRowsPerWarp;
+      h_row = is_halo ? lane / q.nhalo : 0;
+      const int h_idx = is_halo ? lane - h_row * q.nhalo : 0;
+      if (is_halo) {
+        h_col = checked_col(rest_idx, q.Cb + h_idx, H);
+        const size_t p = (size_t)r * H + h_col;
+        h_z = zero[p];
+        h_inv = inv_scale[p];
+        h_lo = -h_z;
+        h_shift = 4 * ((q.Cb + h_idx) & 7);
+        h_off = (warp * kQtRowsPerWarp + h_row) * kQtHalo + (h_col - q.halo_c0);
       }
-      cp_async_commit();
-    };
-    for (int i = 0; i < kQpD - 1; ++i) issue_next();
-
-    for (int i = 0; i < n_tiles; ++i) {
-      issue_next();
-      cp_async_wait<kQpD - 1>();
-      __syncwarp();
-      const int stage = i % kQpD;
-      const int t0 = t_begin + i * kQpR;
-      const int nrows = min(kQpR, t_stop - t0);
-      // codes of the lane's group, one word V per row, OR-ed into two slots
-      if (active && L.n > 0) {
+      const int nk = q.jb - q.ja;
+      k_generic = nk * kQtRowsPerWarp > 96;
 #pragma unroll
-        for (int m = 0; m < kQpR; ++m) {
-          const uint4 v = W.rows[stage][m][lane];
-          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-          uint32_t V = zbase;
-#pragma unroll
-          for (int e = 0; e < 8; e += 2) {
-            float a0, a1;
-            fmul2(a0, a1, __uint_as_float(w[e / 2] << 16), __uint_as_float(w[e / 2] & 0xFFFF0000u),
-                  inv[e], inv[e + 1]);
-            int c0 = __float2int_rn(a0), c1 = __float2int_rn(a1);  // saturating; NaN -> 0
-            c0 = min(max(c0, lo[e]), hi[e]);
-            c1 = min(max(c1, lo[e + 1]), hi[e + 1]);
-            V += (uint32_t)c0 * mul[e] + (uint32_t)c1 * mul[e + 1];
-          }
-          atomicOr(&W.buf[m][slot], V << sh);
-          atomicOr(&W.buf[m][slot + 1], sh ? (V >> (32 - sh)) : 0u);
+      for (int c = 0; c < 3; ++c) {
+        const int p = lane + 32 * c;
+        k_off[c] = -1;
+        if (!k_generic && p < nk * kQtRowsPerWarp) {
+          const int m = p & 3, jj = p >> 2;
+          const int col = checked_col(keep_idx, q.ja + jj, H);
+          k_off[c] = (warp * kQtRowsPerWarp + m) * kQtSlice + min(max(col - q.ha, 0), kQtSlice - 1);
+          k_side[c] = m * k + q.ja + jj;
         }
       }
-      if (is_halo && h_row < nrows) {
-        const uint32_t hw = W.halo[stage][h_row][h_idx];
-        const uint32_t hb16 = (h_col & 1) ? (hw & 0xFFFF0000u) : (hw << 16);
-        int c = __float2int_rn(__fmul_rn(__uint_as_float(hb16), h_inv));
-        c = min(max(c, h_lo), h_lo + 15) + h_z;
-        atomicOr(&W.buf[h_row][nw], (uint32_t)c << h_shift);
+    }
+    if (!sm.ring.wait_full(i, abort, wait_limit)) break;
+    const int st = i % kQtStages;
+    const int t_base = t_first + b * kQtTileRows + warp * kQtRowsPerWarp;  // this warp's first row
+    const int nrows = max(0, min(kQtRowsPerWarp, t_last - t_base));
+    const uint16_t* tile = &sm.tile[st][0][0];
+
+    if (active && L.n > 0) {
+#pragma unroll
+      for (int m = 0; m < kQtRowsPerWarp; ++m) {
+        const uint4 v = reinterpret_cast<const uint4*>(tile + (warp * kQtRowsPerWarp + m) * kQtSlice)[lane];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t V = zbase;
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+          float a0, a1;
+          fmul2(a0, a1, __uint_as_float(w[e / 2] << 16), __uint_as_float(w[e / 2] & 0xFFFF0000u), inv[e],
+                inv[e + 1]);
+          int c0 = __float2int_rn(a0), c1 = __float2int_rn(a1);  // saturating; NaN -> 0
+          c0 = min(max(c0, lo[e]), hi[e]);
+          c1 = min(max(c1, lo[e + 1]), hi[e + 1]);
+          V += (uint32_t)c0 * mul[e] + (uint32_t)c1 * mul[e + 1];
+        }
+        atomicOr(&buf[m][slot], V << sh);
+        atomicOr(&buf[m][slot + 1], sh ? (V >> (32 - sh)) : 0u);
       }
-      // kept values straight from the staged rows
-      for (int p = lane; p < npairs; p += 32) {
-        const int jj = p / kQpR, m = p - jj * kQpR;
+    }
+    if (is_halo && h_row < nrows) {
+      uint32_t hb16;
+      if (q.halo_box) {
+        hb16 = (uint32_t)(&sm.halo[st][0][0])[h_off] << 16;
+      } else {  // halo features spread further than the box: read them directly
+        hb16 = (uint32_t)x[((size_t)r * T + t_base + h_row) * H + h_col] << 16;
+      }
+      int c = __float2int_rn(__fmul_rn(__uint_as_float(hb16), h_inv));
+      c = min(max(c, h_lo), h_lo + 15) + h_z;
+      atomicOr(&buf[h_row][q.nw], (uint32_t)c << h_shift);
+    }
+    // kept values straight from the staged tile
+    uint16_t* srow = side + ((size_t)r * T + t_base) * k;
+    if (!k_generic) {
+#pragma unroll
+      for (int c = 0; c < 3; ++c)
+        if (k_off[c] >= 0 && (lane & 3) < nrows) srow[k_side[c]] = tile[k_off[c]];
+    } else {
+      const int nk = q.jb - q.ja;
+      for (int p = lane; p < nk * kQtRowsPerWarp; p += 32) {
+        const int jj = p >> 2, m = p & 3;
         if (m < nrows) {
-          const int j = ja + jj;
-          const int col = checked_col(keep_idx, j, H);
-          const int src = min(max((col - ha) >> 3, 0), 31);
-          const uint16_t* rowp = reinterpret_cast<const uint16_t*>(&W.rows[stage][m][src]);
-          srow[(size_t)(t0 + m) * k + j] = rowp[col & 7];
+          const int col = checked_col(keep_idx, q.ja + jj, H);
+          srow[(size_t)m * k + q.ja + jj] =
+              tile[(warp * kQtRowsPerWarp + m) * kQtSlice + min(max(col - q.ha, 0), kQtSlice - 1)];
         }
       }
-      __syncwarp();
-      // owned words out (slots 1..nw).  Each lane clears exactly the slots it read (slots
-      // 1..kQpBufWords-1 in all; slot 0 only ever collects nibbles of the previous slice's word
-      // and is never read), so every read precedes its clear in that lane's program order.
-#pragma unroll
-      for (int m = 0; m < kQpR; ++m) {
-        uint32_t* dst = crow + (size_t)(t0 + m) * Wr;
-        const uint32_t a = W.buf[m][lane + 1];
-        if (m < nrows && lane < nw) dst[lane] = a;
-        W.buf[m][lane + 1] = 0u;
-        if (lane + 33 < kQpBufWords) {
-          const uint32_t b = W.buf[m][lane + 33];
-          if (m < nrows && lane + 32 < nw) dst[lane + 32] = b;
-          W.buf[m][lane + 33] = 0u;
-        }
-      }
-      __syncwarp();
     }
-    cp_async_wait<0>();
-    u += t_stop - t_begin;
+    __syncwarp();
+    if (lane == 0) sm.ring.release(i);
+    // owned words out (slots 1..nw); each lane clears exactly the slots it read
+    uint32_t* crow = codes + ((size_t)r * T + t_base) * Wr + q.Wb + lane;
+    const bool w1 = lane < q.nw;
+    if (nrows == kQtRowsPerWarp) {
+#pragma unroll
+      for (int m = 0; m < kQtRowsPerWarp; ++m) {
+        const uint32_t a = buf[m][lane + 1];
+        buf[m][lane + 1] = 0u;
+        if (w1) crow[m * Wr] = a;
+      }
+    } else {
+#pragma unroll
+      for (int m = 0; m < kQtRowsPerWarp; ++m) {
+        const uint32_t a = buf[m][lane + 1];
+        buf[m][lane + 1] = 0u;
+        if (w1 && m < nrows) crow[m * Wr] = a;
+      }
+    }
+    // Slots above 32 only ever hold nonzero bits when the slice owns 33 words (a hi part or a
+    // halo code goes at most to slot nw); otherwise they only receive zero ORs.
+    if (q.nw > 32) {
+      if (lane + 33 < kQtBufWords) {
+#pragma unroll
+        for (int m = 0; m < kQtRowsPerWarp; ++m) {
+          const uint32_t c = buf[m][lane + 33];
+          buf[m][lane + 33] = 0u;
+          if (m < nrows && lane + 32 < q.nw) crow[m * Wr + 32] = c;
+        }
+      }
+    }
+    __syncwarp();
   }
 }
 

@@ -382,7 +382,8 @@ def irwin_hall_stats(o, P=4, H=1024, T=256, k=0, seed=1234):
 
 
 def pin_irwin_hall(o):
-    """Page 4, "Combating Quantization Errors with Tensor Parallelism": quantizing the partial sums
+    """Page "Revolutionizing LLM Inference: The Power of Efficient Low-Bit Communication", section
+    "Combating Quantization Errors with Tensor Parallelism": quantizing the partial sums
     before synchronisation gives a summed error distributed as a sum of P independent uniform
     errors (Irwin-Hall).  Its variance must be sum_r scale_r^2 / 12 within 5%, its mean ~0, and
     for P = 2 its shape the triangular Irwin-Hall(2) law."""

@@ -56,16 +56,25 @@ def test_mid_shapes_bit_exact(cfg):
     compare_all(cfg, _batches(cfg, cs), synth.fill_cpu(cfg, synth.EVAL, 0, cs=cs))
 
 
-def test_clustered_kept_features_bit_exact():
+# (P, T, H, k, runs of kept features): code rows of 182 words (staged with cp.async) and of 384
+# words (staged with TMA; slices with more kept features than the staged side tile holds sum
+# them from HBM).
+CLUSTERED = [
+    (3, 40, 2560, 1104, np.r_[0:8, 100:1100, 1500:1580, 2544:2560]),
+    (3, 70, 4096, 1024, np.r_[0:40, 256:900, 1024:1031, 2000:2300, 4063:4096]),
+]
+
+
+@pytest.mark.parametrize("P,T,H,k,big", CLUSTERED, ids=["cp_async", "tma"])
+def test_clustered_kept_features_bit_exact(P, T, H, k, big):
     """Kept features in long runs (whole groups and slices kept) stress the compact layout."""
     o = oracle.get()
     rng = np.random.default_rng(3)
-    P, T, H, k = 3, 40, 2560, 1104
+    assert len(big) <= k
     x = synth.fill_cpu(synth.CONFIGS["decode"].with_(P=P, T=T, H=H, n_out=4), synth.EVAL, 0,
                        cs=np.ones(H))
     emin = -np.ones((P, H), np.float32)
     emax = np.ones((P, H), np.float32)
-    big = np.r_[0:8, 100:1100, 1500:1580, 2544:2560]  # runs across groups and 1024-feature slices
     emax[:, big] = 50.0
     emin[:, big] = -50.0
     emax += rng.uniform(0, 0.01, (P, H)).astype(np.float32)
