@@ -260,10 +260,21 @@ def run_reference(args, cfg, world, rank):
 # ---------------------------------------------------------------------------------------------
 # the CUDA path
 # ---------------------------------------------------------------------------------------------
-def kernel_source_hash() -> str:
+# The source files each kernel is compiled from (its own header plus what it includes).
+KERNEL_SOURCES = {
+    "calibrate": ["k_calibrate.cuh", "hq_common.cuh"],
+    "select": ["k_select.cuh", "hq_common.cuh"],
+    "quantize_pack": ["k_quantize.cuh", "hq_common.cuh", "hq_tma.cuh"],
+    "dequant_reduce": ["k_dequant.cuh", "hq_common.cuh", "hq_tma.cuh"],
+    "compress_reduce": ["k_fused.cuh", "k_dequant.cuh", "hq_common.cuh", "hq_tma.cuh"],
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    """Hash of the sources of one kernel and of the launch code in hq_api.cu."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "bit_tensor_activation_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in sorted(KERNEL_SOURCES[kernel]) + ["hq_api.cu"]:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
@@ -276,7 +287,7 @@ def ncu_traffic(kernel: str, workload: str):
         with open(path) as f:
             d = json.load(f)
         e = d.get(f"{kernel}@{workload}")
-        if e and e.get("source_hash") == kernel_source_hash():
+        if e and e.get("source_hash") == kernel_source_hash(kernel):
             return e["bytes_per_launch"]
     except Exception:
         pass

@@ -244,16 +244,14 @@ hq_status hq_quantize_pack(const uint16_t* x, int P, int T, int H, int k, const 
   DeviceInfo* d = nullptr;
   if (device_info(&d) != HQ_OK) return HQ_ERR_CUDA;
   const int S = (H + hq::kQtSlice - 1) / hq::kQtSlice;
-  CUtensorMap map_x, map_halo;
-  if (!encode_2d(&map_x, x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)H, (uint64_t)P * T, hq::kQtSlice,
-                 hq::kQtTileRows) ||
-      !encode_2d(&map_halo, x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)H, (uint64_t)P * T, hq::kQtHalo,
-                 hq::kQtTileRows, CU_TENSOR_MAP_L2_PROMOTION_NONE))  // 32-byte rows: no 256-byte over-fetch
+  CUtensorMap map_x;  // x as 32-bit pairs of bf16: the box is 132 pairs = 264 features wide
+  if (!encode_2d(&map_x, x, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)H / 2, (uint64_t)P * T, hq::kQtBoxU32,
+                 hq::kQtTileRows))
     return HQ_ERR_CUDA;
   int chunks, rpc;
   slice_chunks(T, S, (long long)d->sms * d->qt_blocks, hq::kQtTileRows, &chunks, &rpc);
   hq::quantize_pack_tma_kernel<<<(unsigned)(S * chunks), hq::kQtThreads, sizeof(hq::QtSmem) + 128,
-                                 (cudaStream_t)stream>>>(map_x, map_halo, x, P, T, H, k, keep_idx, rest_idx,
+                                 (cudaStream_t)stream>>>(map_x, x, P, T, H, k, keep_idx, rest_idx,
                                                          inv_scale, zero, codes, side, S, chunks, rpc,
                                                          hq::kWaitLimitCycles);
   return launched();

@@ -9,11 +9,11 @@
 // grid is one wave of slices x chunks, so the CTAs of the S slices of a chunk write the same rows
 // of codes and side at about the same time: the 32-byte sectors those rows share at slice
 // boundaries are completed in L2 before eviction instead of costing a read-modify-write in HBM
-// each time.  In a CTA, warp 8 is the producer: one lane issues, per unit, a TMA load of the
-// 32 x 256 bf16 tile (16 KB) plus, when the slice has halo features and they lie within 32
-// columns, a 32 x 32 tile holding them (a second tensor map with that box), into a 4-stage ring.
-// Warps 0..7 are consumers; warp w quantizes rows 4w..4w+3 of each tile, lane l the 8 features
-// 8l..8l+7 (parameters in registers, reloaded only when the unit's rank changes).
+// each time.  In a CTA, warp 8 is the producer: one lane issues, per unit, one TMA load of a
+// 64-row tile of the slice's 256 features and the 8 after them (a box of 132 32-bit elements, so
+// the halo features below are staged too in the common case), into a 3-stage ring.  Warps 0..7
+// are consumers; warp w quantizes rows 8w..8w+7 of each tile, lane l the 8 features 8l..8l+7
+// (parameters in registers, reloaded only when the unit's rank changes).
 //
 // Packing.  Per lane: inv_scale, the clamp bounds -zero and 15-zero and a nibble multiplier 16^j
 // (0 for a kept feature, j = the feature's rank among the group's non-kept ones) for its 8
@@ -25,8 +25,9 @@
 // Ownership of compact words: a slice owns the words whose first nibble one of its groups
 // produces; it drops nibbles that fall into the previous slice's last word and completes its own
 // last word from the next <= 7 non-kept features of the next slice (the "halo", read through
-// rest_idx, one lane each).  So every codes word is written by exactly one CTA.  Kept values are
-// copied from the staged tile to the side buffer.
+// rest_idx, spread over the lanes as (row, feature) pairs; read from the staged tile when they lie
+// within its 8 extra columns, else from global memory).  So every codes word is written by
+// exactly one CTA.  Kept values are copied from the staged tile to the side buffer.
 //
 // Roofline: HBM-bound; 2 bytes read + 0.5 byte written per non-kept element, 2 + 2 per kept one.
 // No memory beyond the inputs and outputs is used.
@@ -39,18 +40,20 @@ namespace hq {
 
 constexpr int kQtWarps = 8;                             // consumer warps
 constexpr int kQtThreads = 32 * (kQtWarps + 1);         // + one producer warp
-constexpr int kQtRowsPerWarp = 4;
-constexpr int kQtTileRows = kQtWarps * kQtRowsPerWarp;  // 32
-constexpr int kQtStages = 4;
-constexpr int kQtSlice = 256;                           // features per slice (box inner dim)
-constexpr int kQtHalo = 32;                             // halo box width (features)
+constexpr int kQtRowsPerWarp = 8;
+constexpr int kQtTileRows = kQtWarps * kQtRowsPerWarp;  // 64
+constexpr int kQtStages = 3;
+constexpr int kQtSlice = 256;                           // features per slice
+constexpr int kQtBoxCols = kQtSlice + 8;                // staged features per row: the slice and 8 beyond
+constexpr int kQtBoxU32 = kQtBoxCols / 2;               // box inner dim in 32-bit elements (<= 256)
 constexpr int kQtBufWords = 36;                         // >= 33 owned words + 2 guard slots per row
-constexpr unsigned kQtTileBytes = kQtTileRows * kQtSlice * 2;
-constexpr unsigned kQtHaloBytes = kQtTileRows * kQtHalo * 2;
+constexpr int kQtHaloSlots = 2;                         // (row, halo feature) pairs per lane
+constexpr int kQtKeptSlots = 4;                         // (row, kept feature) pairs per lane
+constexpr int kQtMaxFastKept = 32 * kQtKeptSlots / kQtRowsPerWarp;  // slices with more copy in a loop
+constexpr unsigned kQtTileBytes = kQtTileRows * kQtBoxCols * 2;
 
 struct QtSmem {
-  alignas(128) uint16_t tile[kQtStages][kQtTileRows][kQtSlice];
-  alignas(128) uint16_t halo[kQtStages][kQtTileRows][kQtHalo];
+  alignas(128) uint16_t tile[kQtStages][kQtTileRows][kQtBoxCols];
   uint32_t buf[kQtWarps][kQtRowsPerWarp][kQtBufWords];
   TmaRing<kQtStages> ring;
   int abort;
@@ -59,8 +62,7 @@ struct QtSmem {
 // Slice facts shared by the producer and the consumers.
 struct QtSlice {
   int ha, hb, ja, jb, Ca, Cb, Wb, We, nw, nhalo;
-  int halo_c0;   // first column of the halo box (a multiple of 8)
-  bool halo_box; // every halo feature lies in [halo_c0, halo_c0 + kQtHalo)
+  bool halo_staged;  // every halo feature lies in the staged columns [ha, ha + kQtBoxCols)
 };
 
 __device__ __forceinline__ QtSlice qt_slice(const int32_t* __restrict__ keep_idx,
@@ -77,20 +79,12 @@ __device__ __forceinline__ QtSlice qt_slice(const int32_t* __restrict__ keep_idx
   q.We = (q.Cb + 7) >> 3;
   q.nw = max(q.We - q.Wb, 0);
   q.nhalo = (q.We > q.Wb) ? (8 * q.We - q.Cb) : 0;
-  q.halo_c0 = 0;
-  q.halo_box = true;
-  if (q.nhalo > 0) {
-    const int first = checked_col(rest_idx, q.Cb, H);
-    const int last = checked_col(rest_idx, q.Cb + q.nhalo - 1, H);
-    q.halo_c0 = first & ~7;
-    q.halo_box = last < q.halo_c0 + kQtHalo;
-  }
+  q.halo_staged = q.nhalo == 0 || checked_col(rest_idx, q.Cb + q.nhalo - 1, H) < q.ha + kQtBoxCols;
   return q;
 }
 
 __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
-    const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_halo,
-    const uint16_t* __restrict__ x, int P, int T, int H,
+    const __grid_constant__ CUtensorMap tmap_x, const uint16_t* __restrict__ x, int P, int T, int H,
     int k, const int32_t* __restrict__ keep_idx, const int32_t* __restrict__ rest_idx,
     const float* __restrict__ inv_scale, const uint8_t* __restrict__ zero, uint32_t* __restrict__ codes,
     uint16_t* __restrict__ side, int S, int chunks, int rows_per_chunk, long long wait_limit) {
@@ -116,9 +110,7 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
   if (warp == kQtWarps) {
     if (lane == 0) {
       prefetch_tensor_map(&tmap_x);
-      prefetch_tensor_map(&tmap_halo);
       int issued = 0;
-      const QtSlice q = qt_slice(keep_idx, rest_idx, H, k, s);
       int r = 0, b = 0;  // unit i = (rank r, row block b), advanced incrementally
       for (int i = 0; i < n_units; ++i) {
         if (i > 0 && ++b == NBc) {
@@ -128,10 +120,8 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
         if (!sm.ring.acquire(i, abort, wait_limit)) break;
         const int st = i % kQtStages;
         const int row = r * T + t_first + b * kQtTileRows;
-        const bool halo = q.nhalo > 0 && q.halo_box;
-        mbar_arrive_expect_tx(&sm.ring.full[st], kQtTileBytes + (halo ? kQtHaloBytes : 0u));
-        tma_load_2d(&sm.tile[st][0][0], &tmap_x, q.ha, row, &sm.ring.full[st]);
-        if (halo) tma_load_2d(&sm.halo[st][0][0], &tmap_halo, q.halo_c0, row, &sm.ring.full[st]);
+        mbar_arrive_expect_tx(&sm.ring.full[st], kQtTileBytes);
+        tma_load_2d(&sm.tile[st][0][0], &tmap_x, (s * kQtSlice) / 2, row, &sm.ring.full[st]);
         ++issued;
       }
       if (*abort) sm.ring.drain(issued, wait_limit);
@@ -151,18 +141,36 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
   int lo[8], hi[8];
   uint32_t mul[8], zbase = 0;
   int slot = 0, sh = 0;
-  bool is_halo = false;
-  int h_row = 0, h_col = 0, h_lo = 0, h_z = 0, h_shift = 0, h_off = 0;
-  float h_inv = 0.0f;
-  // kept copies of this lane: pair p = lane + 32c (c < 3) is (row p & 3, kept feature p >> 2);
-  // k_off = tile element offset (-1: no pair), k_side = side element offset within the unit
-  bool k_generic = false;
-  int k_off[3] = {-1, -1, -1}, k_side[3] = {0, 0, 0};
+  // halo work: pair p = lane + 32c (c < kQtHaloSlots) is (row p / nhalo, halo feature p % nhalo);
+  // h_pack = row | shift << 4 | zero << 9 | (column - ha) << 13 (row 8: no pair)
+  uint32_t h_pack[kQtHaloSlots];
+  float h_inv[kQtHaloSlots];
+  // kept copies: pair p = lane + 32c (c < kQtKeptSlots) is (row lane % 8, kept feature
+  // lane / 8 + 4c), present while lane / 8 + 4c < nk; byte c of k_cols = its column - ha, its
+  // side element (within the unit) is k_side0 + 4c
+  const int nk = q.jb - q.ja;
+  const bool k_generic = nk > kQtMaxFastKept;
+  const int k_m = lane % kQtRowsPerWarp, k_j = lane / kQtRowsPerWarp;
+  const int k_row_off = (warp * kQtRowsPerWarp + k_m) * kQtBoxCols;
+  const int k_side0 = k_m * k + q.ja + k_j;
+  uint32_t k_cols = 0;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    inv[i] = 0.0f;
-    lo[i] = hi[i] = 0;
-    mul[i] = 0u;
+  for (int c = 0; c < kQtKeptSlots; ++c) {
+    if (!k_generic && k_j + 4 * c < nk) {
+      const int col = checked_col(keep_idx, q.ja + k_j + 4 * c, H);
+      k_cols |= (uint32_t)min(max(col - q.ha, 0), kQtSlice - 1) << (8 * c);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    inv[e] = 0.0f;
+    lo[e] = hi[e] = 0;
+    mul[e] = 0u;
+  }
+#pragma unroll
+  for (int c = 0; c < kQtHaloSlots; ++c) {
+    h_pack[c] = kQtRowsPerWarp;  // no pair
+    h_inv[c] = 0.0f;
   }
   uint32_t(*buf)[kQtBufWords] = sm.buf[warp];
 
@@ -198,30 +206,17 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
       }
       slot = (L.c0 >> 3) - q.Wb + 1;
       sh = 4 * (L.c0 & 7);
-      // halo work of a tile: lane p < nhalo*4 takes halo feature p % nhalo of row p / nhalo
-      is_halo = lane < q.nhalo * kQtRowsPerWarp;
-      h_row = is_halo ? lane / q.nhalo : 0;
-      const int h_idx = is_halo ? lane - h_row * q.nhalo : 0;
-      if (is_halo) {
-        h_col = checked_col(rest_idx, q.Cb + h_idx, H);
-        const size_t p = (size_t)r * H + h_col;
-        h_z = zero[p];
-        h_inv = inv_scale[p];
-        h_lo = -h_z;
-        h_shift = 4 * ((q.Cb + h_idx) & 7);
-        h_off = (warp * kQtRowsPerWarp + h_row) * kQtHalo + (h_col - q.halo_c0);
-      }
-      const int nk = q.jb - q.ja;
-      k_generic = nk * kQtRowsPerWarp > 96;
 #pragma unroll
-      for (int c = 0; c < 3; ++c) {
+      for (int c = 0; c < kQtHaloSlots; ++c) {
         const int p = lane + 32 * c;
-        k_off[c] = -1;
-        if (!k_generic && p < nk * kQtRowsPerWarp) {
-          const int m = p & 3, jj = p >> 2;
-          const int col = checked_col(keep_idx, q.ja + jj, H);
-          k_off[c] = (warp * kQtRowsPerWarp + m) * kQtSlice + min(max(col - q.ha, 0), kQtSlice - 1);
-          k_side[c] = m * k + q.ja + jj;
+        h_pack[c] = kQtRowsPerWarp;
+        if (p < q.nhalo * kQtRowsPerWarp) {
+          const int row = p / q.nhalo, idx = p - row * q.nhalo;
+          const int col = checked_col(rest_idx, q.Cb + idx, H);
+          const size_t pp = (size_t)r * H + col;
+          h_inv[c] = inv_scale[pp];
+          h_pack[c] = (uint32_t)row | (uint32_t)(4 * ((q.Cb + idx) & 7)) << 4 | (uint32_t)zero[pp] << 9 |
+                      (uint32_t)(col - q.ha) << 13;
         }
       }
     }
@@ -234,7 +229,7 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
     if (active && L.n > 0) {
 #pragma unroll
       for (int m = 0; m < kQtRowsPerWarp; ++m) {
-        const uint4 v = reinterpret_cast<const uint4*>(tile + (warp * kQtRowsPerWarp + m) * kQtSlice)[lane];
+        const uint4 v = reinterpret_cast<const uint4*>(tile + (warp * kQtRowsPerWarp + m) * kQtBoxCols)[lane];
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
         uint32_t V = zbase;
 #pragma unroll
@@ -251,31 +246,36 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
         atomicOr(&buf[m][slot + 1], sh ? (V >> (32 - sh)) : 0u);
       }
     }
-    if (is_halo && h_row < nrows) {
-      uint32_t hb16;
-      if (q.halo_box) {
-        hb16 = (uint32_t)(&sm.halo[st][0][0])[h_off] << 16;
-      } else {  // halo features spread further than the box: read them directly
-        hb16 = (uint32_t)x[((size_t)r * T + t_base + h_row) * H + h_col] << 16;
+    // halo codes: features of the next slice completing this slice's last word
+#pragma unroll
+    for (int c = 0; c < kQtHaloSlots; ++c) {
+      const int h_row = h_pack[c] & 15u;
+      if (h_row < nrows) {
+        const int h_shift = (h_pack[c] >> 4) & 31u, h_z = (h_pack[c] >> 9) & 15u, h_off = h_pack[c] >> 13;
+        uint32_t hb16;
+        if (q.halo_staged) {
+          hb16 = (uint32_t)tile[(warp * kQtRowsPerWarp + h_row) * kQtBoxCols + h_off] << 16;
+        } else {  // halo features spread beyond the staged columns: read them directly
+          hb16 = (uint32_t)x[((size_t)r * T + t_base + h_row) * H + q.ha + h_off] << 16;
+        }
+        int cc = __float2int_rn(__fmul_rn(__uint_as_float(hb16), h_inv[c]));
+        cc = min(max(cc, -h_z), 15 - h_z) + h_z;
+        atomicOr(&buf[h_row][q.nw], (uint32_t)cc << h_shift);
       }
-      int c = __float2int_rn(__fmul_rn(__uint_as_float(hb16), h_inv));
-      c = min(max(c, h_lo), h_lo + 15) + h_z;
-      atomicOr(&buf[h_row][q.nw], (uint32_t)c << h_shift);
     }
     // kept values straight from the staged tile
     uint16_t* srow = side + ((size_t)r * T + t_base) * k;
     if (!k_generic) {
 #pragma unroll
-      for (int c = 0; c < 3; ++c)
-        if (k_off[c] >= 0 && (lane & 3) < nrows) srow[k_side[c]] = tile[k_off[c]];
+      for (int c = 0; c < kQtKeptSlots; ++c)
+        if (k_j + 4 * c < nk && k_m < nrows) srow[k_side0 + 4 * c] = tile[k_row_off + ((k_cols >> (8 * c)) & 255u)];
     } else {
-      const int nk = q.jb - q.ja;
       for (int p = lane; p < nk * kQtRowsPerWarp; p += 32) {
-        const int jj = p >> 2, m = p & 3;
+        const int jj = p / kQtRowsPerWarp, m = p % kQtRowsPerWarp;
         if (m < nrows) {
           const int col = checked_col(keep_idx, q.ja + jj, H);
           srow[(size_t)m * k + q.ja + jj] =
-              tile[(warp * kQtRowsPerWarp + m) * kQtSlice + min(max(col - q.ha, 0), kQtSlice - 1)];
+              tile[(warp * kQtRowsPerWarp + m) * kQtBoxCols + min(max(col - q.ha, 0), kQtSlice - 1)];
         }
       }
     }
@@ -289,14 +289,14 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
       for (int m = 0; m < kQtRowsPerWarp; ++m) {
         const uint32_t a = buf[m][lane + 1];
         buf[m][lane + 1] = 0u;
-        if (w1) crow[m * Wr] = a;
+        if (w1) crow[(size_t)m * Wr] = a;
       }
     } else {
 #pragma unroll
       for (int m = 0; m < kQtRowsPerWarp; ++m) {
         const uint32_t a = buf[m][lane + 1];
         buf[m][lane + 1] = 0u;
-        if (w1 && m < nrows) crow[m * Wr] = a;
+        if (w1 && m < nrows) crow[(size_t)m * Wr] = a;
       }
     }
     // Slots above 32 only ever hold nonzero bits when the slice owns 33 words (a hi part or a
@@ -307,7 +307,7 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
         for (int m = 0; m < kQtRowsPerWarp; ++m) {
           const uint32_t c = buf[m][lane + 33];
           buf[m][lane + 33] = 0u;
-          if (m < nrows && lane + 32 < q.nw) crow[m * Wr + 32] = c;
+          if (m < nrows && lane + 32 < q.nw) crow[(size_t)m * Wr + 32] = c;
         }
       }
     }
