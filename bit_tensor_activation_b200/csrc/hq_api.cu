@@ -248,11 +248,14 @@ hq_status hq_quantize_pack(const uint16_t* x, int P, int T, int H, int k, const 
   if (!encode_2d(&map_x, x, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)H / 2, (uint64_t)P * T, hq::kQtBoxU32,
                  hq::kQtTileRows))
     return HQ_ERR_CUDA;
-  int chunks, rpc;
-  slice_chunks(T, S, (long long)d->sms * d->qt_blocks, hq::kQtTileRows, &chunks, &rpc);
-  hq::quantize_pack_tma_kernel<<<(unsigned)(S * chunks), hq::kQtThreads, sizeof(hq::QtSmem) + 128,
+  // J CTAs per slice, one wave; each takes a balanced contiguous range of (rank, 64-row block) units
+  const long long units = (long long)P * ceil_div(T, hq::kQtTileRows);
+  long long J = (long long)d->sms * d->qt_blocks / S;
+  if (J < 1) J = 1;
+  if (J > units) J = units;
+  hq::quantize_pack_tma_kernel<<<(unsigned)(S * J), hq::kQtThreads, sizeof(hq::QtSmem) + 128,
                                  (cudaStream_t)stream>>>(map_x, x, P, T, H, k, keep_idx, rest_idx,
-                                                         inv_scale, zero, codes, side, S, chunks, rpc,
+                                                         inv_scale, zero, codes, side, S, (int)J,
                                                          hq::kWaitLimitCycles);
   return launched();
 }

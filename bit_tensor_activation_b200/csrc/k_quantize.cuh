@@ -4,12 +4,13 @@
 // become 4-bit codes q = clamp(rint(x*inv_scale)+zero, 0, 15) packed 8 per uint32 in rest_idx
 // order.
 //
-// Work decomposition.  A CTA owns one slice of 256 features and one chunk of rows, and walks the
-// ranks (outer) and the chunk's 32-row blocks (inner); a work unit is one (rank, row block).  The
-// grid is one wave of slices x chunks, so the CTAs of the S slices of a chunk write the same rows
-// of codes and side at about the same time: the 32-byte sectors those rows share at slice
-// boundaries are completed in L2 before eviction instead of costing a read-modify-write in HBM
-// each time.  In a CTA, warp 8 is the producer: one lane issues, per unit, one TMA load of a
+// Work decomposition.  A slice is 256 features; a work unit is one (rank, 64-row block) of a
+// slice, numbered rank-major, u = rank * NB + block.  The grid is one wave of S slices x J CTAs:
+// CTA j of every slice takes the same contiguous range of units [j*U/J, (j+1)*U/J) (U = P*NB), so
+// the ranges differ by at most one unit and a CTA changes rank at most a few times.  The CTAs of
+// the S slices that share j write the same rows of codes and side at about the same time: the
+// 32-byte sectors those rows share at slice boundaries are completed in L2 before eviction
+// instead of costing a read-modify-write in HBM each time.  In a CTA, warp 8 is the producer: one lane issues, per unit, one TMA load of a
 // 64-row tile of the slice's 256 features and the 8 after them (a box of 132 32-bit elements, so
 // the halo features below are staged too in the common case), into a 3-stage ring.  Warps 0..7
 // are consumers; warp w quantizes rows 8w..8w+7 of each tile, lane l the 8 features 8l..8l+7
@@ -87,14 +88,15 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
     const __grid_constant__ CUtensorMap tmap_x, const uint16_t* __restrict__ x, int P, int T, int H,
     int k, const int32_t* __restrict__ keep_idx, const int32_t* __restrict__ rest_idx,
     const float* __restrict__ inv_scale, const uint8_t* __restrict__ zero, uint32_t* __restrict__ codes,
-    uint16_t* __restrict__ side, int S, int chunks, int rows_per_chunk, long long wait_limit) {
+    uint16_t* __restrict__ side, int S, int J, long long wait_limit) {
   extern __shared__ __align__(128) unsigned char s_raw[];
   QtSmem& sm = *reinterpret_cast<QtSmem*>(s_raw);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int s = blockIdx.x / chunks, chunk = blockIdx.x - s * chunks;
-  const int t_first = chunk * rows_per_chunk, t_last = min(T, t_first + rows_per_chunk);
-  const int NBc = (t_last - t_first + kQtTileRows - 1) / kQtTileRows;  // row blocks of the chunk
-  const int n_units = NBc * P;                                         // unit i = (rank i / NBc, block i % NBc)
+  const int s = blockIdx.x / J, j = blockIdx.x - s * J;
+  const int NB = (T + kQtTileRows - 1) / kQtTileRows;  // 64-row blocks per rank
+  const long long U = (long long)P * NB;
+  const int u0 = (int)(U * j / J), u1 = (int)(U * (j + 1) / J);
+  const int n_units = u1 - u0;  // unit u0 + i = (rank (u0+i) / NB, block (u0+i) % NB)
 
   if (threadIdx.x == 0) {
     sm.ring.init(kQtWarps);
@@ -111,15 +113,15 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
     if (lane == 0) {
       prefetch_tensor_map(&tmap_x);
       int issued = 0;
-      int r = 0, b = 0;  // unit i = (rank r, row block b), advanced incrementally
+      int r = u0 / NB, b = u0 - (u0 / NB) * NB;  // unit (rank r, row block b), advanced incrementally
       for (int i = 0; i < n_units; ++i) {
-        if (i > 0 && ++b == NBc) {
+        if (i > 0 && ++b == NB) {
           b = 0;
           ++r;
         }
         if (!sm.ring.acquire(i, abort, wait_limit)) break;
         const int st = i % kQtStages;
-        const int row = r * T + t_first + b * kQtTileRows;
+        const int row = r * T + b * kQtTileRows;
         mbar_arrive_expect_tx(&sm.ring.full[st], kQtTileBytes);
         tma_load_2d(&sm.tile[st][0][0], &tmap_x, (s * kQtSlice) / 2, row, &sm.ring.full[st]);
         ++issued;
@@ -131,7 +133,7 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
 
   // ---------------------------------------------------------------- consumer warps
   const int Hr = H - k, Wr = Hr / 8, NG = H / 8;
-  int r = 0, b = 0;
+  int r = u0 / NB, b = u0 - (u0 / NB) * NB;
   bool fresh = true;  // rank changed: reload this lane's parameters
   const QtSlice q = qt_slice(keep_idx, rest_idx, H, k, s);
   if (threadIdx.x == 0 && ((s == 0 && q.ja != 0) || (s == S - 1 && q.jb != k))) record_error(HQ_ERR_BAD_INDEX);
@@ -175,7 +177,7 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
   uint32_t(*buf)[kQtBufWords] = sm.buf[warp];
 
   for (int i = 0; i < n_units; ++i) {
-    if (i > 0 && ++b == NBc) {
+    if (i > 0 && ++b == NB) {
       b = 0;
       fresh = true;
       ++r;
@@ -222,8 +224,8 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
     }
     if (!sm.ring.wait_full(i, abort, wait_limit)) break;
     const int st = i % kQtStages;
-    const int t_base = t_first + b * kQtTileRows + warp * kQtRowsPerWarp;  // this warp's first row
-    const int nrows = max(0, min(kQtRowsPerWarp, t_last - t_base));
+    const int t_base = b * kQtTileRows + warp * kQtRowsPerWarp;  // this warp's first row
+    const int nrows = max(0, min(kQtRowsPerWarp, T - t_base));
     const uint16_t* tile = &sm.tile[st][0][0];
 
     if (active && L.n > 0) {
