@@ -225,8 +225,12 @@ hq_status hq_select_topk(const float* ema_min, const float* ema_max, int P, int 
       d->select_smem_set = true;
     }
   }
-  hq::select_topk_kernel<<<1, hq::kSelThreads, smem, (cudaStream_t)stream>>>(
+  // parameters and keys over the whole GPU, then the selection in one CTA (same stream)
+  const unsigned pgrid = (unsigned)ceil_div(H, hq::kSelParamThreads);
+  hq::select_params_kernel<<<pgrid, hq::kSelParamThreads, 0, (cudaStream_t)stream>>>(
       ema_min, ema_max, P, H, k, keep_idx, rest_idx, scale, inv_scale, zero);
+  if (cudaGetLastError() != cudaSuccess) return HQ_ERR_CUDA;
+  hq::select_topk_kernel<<<1, hq::kSelThreads, smem, (cudaStream_t)stream>>>(H, k, keep_idx, rest_idx);
   return launched();
 }
 

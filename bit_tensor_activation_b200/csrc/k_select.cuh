@@ -2,18 +2,19 @@
 // Power of Efficient Low-Bit Communication", section "The Hybrid Quantization Algorithm", bullet
 // "Selection of High Precision Features"), with the 4-bit grid of bullet "Calibration".
 //
-// One CTA of 1024 threads does the whole selection, so no memory beyond the inputs and outputs
-// is needed:
-//   1. per rank and feature: lo = min(ema_min,0), hi = max(ema_max,0), scale = (hi-lo)/15,
-//      inv_scale = 1/scale, zero = clamp(rint(-lo*inv_scale),0,15) (degenerate scale -> 1, 0),
-//      and the feature's score = sum over ranks of (hi-lo) in rank order; the score's fp32 bits
-//      (non-negative, so their unsigned order is the numeric order; NaN ranks as +inf) are kept
-//      in shared memory;
-//   2. radix select, 8 bits per pass from the top, finds the k-th largest score tau and how many
-//      features equal to tau are still to be taken;
-//   3. a block-wide ordered scan takes every feature above tau plus the lowest-indexed features
-//      equal to tau, and writes keep_idx / rest_idx ascending.
-// H <= 32768 (the scores fill up to 128 KB of shared memory).
+// Two kernels, no memory beyond the inputs and outputs:
+//   1. select_params_kernel, one thread per feature over the whole GPU: for each rank in order,
+//      lo = min(ema_min,0), hi = max(ema_max,0), scale = (hi-lo)/15, inv_scale = 1/scale,
+//      zero = clamp(rint(-lo*inv_scale),0,15) (degenerate scale -> 1, 0), and the feature's score
+//      = sum over ranks of (hi-lo) in rank order.  The score's fp32 bits (non-negative, so their
+//      unsigned order is the numeric order; NaN ranks as +inf) are parked in the index outputs:
+//      slot h of the H slots rest_idx[0..H-k) followed by keep_idx[0..k).
+//   2. select_topk_kernel, one CTA of 1024 threads: reads the H keys into shared memory, then a
+//      radix select, 8 bits per pass from the top, finds the k-th largest key tau and how many
+//      features equal to tau are still to be taken, and a block-wide ordered scan takes every
+//      feature above tau plus the lowest-indexed features equal to tau and writes keep_idx /
+//      rest_idx ascending over the parked keys.
+// H <= 32768 (the keys fill up to 128 KB of shared memory).
 #pragma once
 
 #include <float.h>
@@ -53,20 +54,13 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int& tot
   return r;
 }
 
-__global__ void __launch_bounds__(kSelThreads) select_topk_kernel(
+constexpr int kSelParamThreads = 256;
+
+__global__ void __launch_bounds__(kSelParamThreads) select_params_kernel(
     const float* __restrict__ ema_min, const float* __restrict__ ema_max, int P, int H, int k,
     int32_t* __restrict__ keep_idx, int32_t* __restrict__ rest_idx, float* __restrict__ scale,
     float* __restrict__ inv_scale, uint8_t* __restrict__ zero) {
-  extern __shared__ uint32_t s_key[];  // [H]
-  __shared__ int s_hist[256];
-  __shared__ int s_warp[32];
-  __shared__ uint32_t s_prefix;
-  __shared__ int s_remaining;
-
-  const int tid = threadIdx.x;
-
-  // ---- 1. parameters and scores ------------------------------------------------------------
-  for (int h = tid; h < H; h += kSelThreads) {
+  for (int h = blockIdx.x * blockDim.x + threadIdx.x; h < H; h += gridDim.x * blockDim.x) {
     float score = 0.0f;
     for (int r = 0; r < P; ++r) {
       const size_t i = (size_t)r * H + h;
@@ -89,8 +83,25 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(
       zero[i] = (uint8_t)(int)zf;
       score = __fadd_rn(score, range);
     }
-    s_key[h] = (score != score) ? 0x7F800000u : __float_as_uint(score);
+    const uint32_t key = (score != score) ? 0x7F800000u : __float_as_uint(score);
+    if (h < H - k) rest_idx[h] = (int32_t)key;
+    else keep_idx[h - (H - k)] = (int32_t)key;
   }
+}
+
+__global__ void __launch_bounds__(kSelThreads) select_topk_kernel(int H, int k, int32_t* __restrict__ keep_idx,
+                                                                  int32_t* __restrict__ rest_idx) {
+  extern __shared__ uint32_t s_key[];  // [H]
+  __shared__ int s_hist[256];
+  __shared__ int s_warp[32];
+  __shared__ uint32_t s_prefix;
+  __shared__ int s_remaining;
+
+  const int tid = threadIdx.x;
+
+  // ---- 1. the parked keys -------------------------------------------------------------------
+  for (int h = tid; h < H; h += kSelThreads)
+    s_key[h] = (uint32_t)((h < H - k) ? rest_idx[h] : keep_idx[h - (H - k)]);
   __syncthreads();
 
   // ---- 2. radix select of the k-th largest key ---------------------------------------------

@@ -86,6 +86,8 @@ hq_status hq_calibrate(const uint16_t* x, int P, int T, int H, float beta, int f
  *   keep_idx int32 [k]    the kept features, ascending
  *   rest_idx int32 [H-k]  all other features, ascending
  *   scale, inv_scale float [P][H], zero uint8 [P][H]  (computed for kept features too)
+ * Two kernels on `stream`; between them keep_idx and rest_idx hold the scores (the library uses
+ * no other memory), so they must not be read until the stream has passed the call.
  */
 hq_status hq_select_topk(const float* ema_min, const float* ema_max, int P, int H, int k,
                          int32_t* keep_idx, int32_t* rest_idx, float* scale, float* inv_scale,
