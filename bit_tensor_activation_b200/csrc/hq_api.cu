@@ -250,7 +250,7 @@ hq_status hq_quantize_pack(const uint16_t* x, int P, int T, int H, int k, const 
   const int S = (H + hq::kQtSlice - 1) / hq::kQtSlice;
   CUtensorMap map_x;  // x as 32-bit pairs of bf16: the box is 132 pairs = 264 features wide
   if (!encode_2d(&map_x, x, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)H / 2, (uint64_t)P * T, hq::kQtBoxU32,
-                 hq::kQtTileRows))
+                 hq::kQtTileRows, CU_TENSOR_MAP_L2_PROMOTION_NONE))  // 528-byte rows: no 256-byte over-fetch
     return HQ_ERR_CUDA;
   // J CTAs per slice, one wave; each takes a balanced contiguous range of (rank, 64-row block) units
   const long long units = (long long)P * ceil_div(T, hq::kQtTileRows);
