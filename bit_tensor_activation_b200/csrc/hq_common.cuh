@@ -145,6 +145,62 @@ __device__ __forceinline__ GroupLayout group_layout(const int32_t* __restrict__ 
   return L;
 }
 
+// The kept features of a feature range [lo, hi), for a whole CTA at once: ja = #{keep_idx < lo}
+// and jb = #{keep_idx < hi} (the lower bounds when keep_idx is ascending) from one coalesced pass
+// over keep_idx by all blockDim.x threads, and keep_idx[ja .. ja + min(jb-ja, cap)) copied to
+// list.  Every thread of the CTA must call it (it holds __syncthreads); all get ja and jb.
+struct SliceKept {
+  int ja, jb;
+};
+__device__ __forceinline__ SliceKept cta_slice_kept(const int32_t* __restrict__ keep_idx, int k, int lo, int hi,
+                                                    int* s_cnt, int* list, int cap) {
+  int a = 0, b = 0;
+  for (int i = threadIdx.x; i < k; i += blockDim.x) {
+    const int v = __ldg(keep_idx + i);
+    a += v < lo;
+    b += v < hi;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    a += __shfl_down_sync(0xFFFFFFFFu, a, off);
+    b += __shfl_down_sync(0xFFFFFFFFu, b, off);
+  }
+  if (threadIdx.x == 0) s_cnt[0] = s_cnt[1] = 0;
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) {
+    atomicAdd(&s_cnt[0], a);
+    atomicAdd(&s_cnt[1], b);
+  }
+  __syncthreads();
+  const SliceKept r{s_cnt[0], s_cnt[1]};
+  const int n = min(r.jb - r.ja, cap);
+  for (int i = threadIdx.x; i < n; i += blockDim.x) list[i] = __ldg(keep_idx + r.ja + i);
+  __syncthreads();
+  return r;
+}
+
+// group_layout() for a group inside a range whose kept features are list[0..n) (= keep_idx[ja..),
+// ascending), without touching global memory.
+__device__ __forceinline__ GroupLayout group_layout_list(const int* list, int n, int ja, int H, int k, int h0) {
+  GroupLayout L;
+  int below = 0;
+  uint32_t km = 0;
+  for (int i = 0; i < n; ++i) {
+    const int d = list[i] - h0;
+    below += d < 0;
+    if (d >= 0 && d < 8) km |= 1u << d;
+  }
+  L.j0 = ja + below;
+  L.kmask = km;
+  L.n = 8 - __popc(km);
+  L.c0 = h0 - L.j0;
+  if (L.c0 < 0 || L.c0 > H - k) {
+    record_error(HQ_ERR_BAD_INDEX);
+    L.c0 = min(max(L.c0, 0), H - k);
+  }
+  return L;
+}
+
 // Column index read from keep_idx / rest_idx, clamped into [0, H) with the error recorded.
 __device__ __forceinline__ int checked_col(const int32_t* __restrict__ idx, int j, int H) {
   int h = __ldg(idx + j);

@@ -95,13 +95,14 @@ struct DqLane {
   uint32_t key[8];   // fast path: in-place nibble mask; generic path: nibble shift
 };
 
-__device__ __forceinline__ DqLane dq_lane(const int32_t* __restrict__ keep_idx, int k, int H, int s, int lane,
-                                          int w_base, bool generic) {
+// max_w: the last staged word a lane may start at (its second word must be staged too); an
+// inconsistent index could only move the start, and is clamped.
+__device__ __forceinline__ DqLane dq_lane_layout(const GroupLayout& L, int h0, int H, int w_base, int max_w,
+                                                 bool generic) {
   DqLane D;
-  D.h0 = 8 * (s * kDqSliceGroups + lane);
-  D.active = D.h0 < H;
-  D.L = GroupLayout{0, 0, 0u, 0};
-  if (D.active) D.L = group_layout(keep_idx, k, H, D.h0);
+  D.h0 = h0;
+  D.active = h0 < H;
+  D.L = D.active ? L : GroupLayout{0, 0, 0u, 0};
   int pos[8], jpos[8];
   const int b = dq_positions(D.L.kmask, pos, jpos);
   D.sh2 = 4 * b;
@@ -110,10 +111,17 @@ __device__ __forceinline__ DqLane dq_lane(const int32_t* __restrict__ keep_idx, 
     const bool kept = (D.L.kmask >> i) & 1u;
     D.key[i] = generic ? (uint32_t)(4 * jpos[i]) : (kept ? 0u : (0xFu << (4 * pos[i])));
   }
-  D.my_w = (D.L.c0 >> 3) - w_base;
+  D.my_w = min(max((D.L.c0 >> 3) - w_base, 0), max_w);
   D.fsh = 4 * (D.L.c0 & 7);
   D.decode = D.active && D.L.n > 0;
   return D;
+}
+
+__device__ __forceinline__ DqLane dq_lane(const int32_t* __restrict__ keep_idx, int k, int H, int s, int lane,
+                                          int w_base, int max_w, bool generic) {
+  const int h0 = 8 * (s * kDqSliceGroups + lane);
+  const GroupLayout L = h0 < H ? group_layout(keep_idx, k, H, h0) : GroupLayout{0, 0, 0u, 0};
+  return dq_lane_layout(L, h0, H, w_base, max_w, generic);
 }
 
 // Whether this thread's share of slice s has a scale below 2^-109 (the slice then needs the
@@ -131,8 +139,9 @@ __device__ __forceinline__ bool dq_has_tiny_scale(const float* __restrict__ scal
 
 // Per-(rank, group) constants of slice s in a conflict-free [P][4][32] float4 layout:
 // scale/16^p x8, -(2^23 + zero*16^p) x8 (p = 0 on the generic path).
+// group_kmask: the 32 groups' kept masks when already known (in shared memory), else NULL.
 __device__ __forceinline__ void dq_fill_constants(float4* s_const, const int32_t* __restrict__ keep_idx,
-                                                  const float* __restrict__ scale,
+                                                  const uint32_t* group_kmask, const float* __restrict__ scale,
                                                   const uint8_t* __restrict__ zero, int P, int H, int k,
                                                   int s, bool generic, int nthreads) {
   for (int idx = threadIdx.x; idx < P * 32; idx += nthreads) {
@@ -140,7 +149,7 @@ __device__ __forceinline__ void dq_fill_constants(float4* s_const, const int32_t
     const int hg = 8 * (s * kDqSliceGroups + g);
     float sc[8], off[8];
     uint32_t km = 0;
-    if (hg < H) km = group_layout(keep_idx, k, H, hg).kmask;
+    if (hg < H) km = group_kmask ? group_kmask[g] : group_layout(keep_idx, k, H, hg).kmask;
     int pos[8], jpos[8];
     dq_positions(km, pos, jpos);
 #pragma unroll
@@ -265,19 +274,24 @@ __device__ __forceinline__ void dq_finish_block(const DqLane& D, float (&acc)[R]
 struct DqSlice {
   int hs, he, ja, jb, Ca, Cb, w_first, n_words;
 };
-__device__ __forceinline__ DqSlice dq_slice(const int32_t* __restrict__ keep_idx, int H, int k, int s, int S) {
+__device__ __forceinline__ DqSlice dq_slice_from(int ja, int jb, int H, int k, int s, int S) {
   DqSlice q;
   const int Hr = H - k, Wr = Hr / 8;
   q.hs = 8 * s * kDqSliceGroups;
   q.he = min(H, q.hs + 8 * kDqSliceGroups);
-  q.ja = lower_bound_i32(keep_idx, k, q.hs);
-  q.jb = lower_bound_i32(keep_idx, k, q.he);
+  q.ja = ja;
+  q.jb = jb;
   if (threadIdx.x == 0 && ((s == 0 && q.ja != 0) || (s == S - 1 && q.jb != k))) record_error(HQ_ERR_BAD_INDEX);
   q.Ca = min(max(q.hs - q.ja, 0), Hr);
   q.Cb = min(max(q.he - q.jb, 0), Hr);
   q.w_first = q.Ca >> 3;
   q.n_words = max(0, min(Wr, (q.Cb >> 3) + 2) - q.w_first);  // words the slice needs per row, <= 35
   return q;
+}
+
+__device__ __forceinline__ DqSlice dq_slice(const int32_t* __restrict__ keep_idx, int H, int k, int s, int S) {
+  const int hs = 8 * s * kDqSliceGroups, he = min(H, hs + 8 * kDqSliceGroups);
+  return dq_slice_from(lower_bound_i32(keep_idx, k, hs), lower_bound_i32(keep_idx, k, he), H, k, s, S);
 }
 
 // ======================================================================== TMA kernel (default)
@@ -302,6 +316,10 @@ struct DtSmem {
   alignas(128) uint32_t tile[kDtStages][kDtG][kDtTileRows][kDtWords];
   alignas(128) uint16_t side[kDtStages][kDtG][kDtTileRows][kDtSideCols];
   float kept[kDtWarps][kDtR * 32];
+  int klist[8 * kDqSliceGroups];  // the slice's kept features
+  int kcnt[2];
+  uint32_t gkmask[kDqSliceGroups];  // per group of the slice: kept mask and kept features before it
+  int gj0[kDqSliceGroups];
   TmaRing<kDtStages> ring;
   int abort;
   // followed by the constants: float4 [P][4][32]
@@ -344,17 +362,19 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
   const int n_groups = (P + kDtG - 1) / kDtG;  // ring slots per block
   const int n_slots_total = nblk * n_groups;     // slot i = (block i / n_groups, rank group i % n_groups)
 
-  const DqSlice q = dq_slice(keep_idx, H, k, s, S);
-  const int w_a = q.w_first & ~3;  // 16-byte aligned x coordinate of the box
-  const int nk = q.jb - q.ja;
-  const int j_a = q.ja & ~7;       // 16-byte aligned x coordinate of the side box
-  const bool stage_side = nk > 0 && nk <= kDtMaxStagedKept && q.jb <= j_a + kDtSideCols;
   if (threadIdx.x == 0) {
     sm.ring.init(kDtWarps);
     sm.abort = 0;
     fence_barrier_init();
   }
-  __syncthreads();
+  // the slice's kept features, counted by the whole CTA (no dependent searches before the loads)
+  const int hs0 = 8 * s * kDqSliceGroups, he0 = min(H, hs0 + 8 * kDqSliceGroups);
+  const SliceKept sk = cta_slice_kept(keep_idx, k, hs0, he0, sm.kcnt, sm.klist, 8 * kDqSliceGroups);
+  const DqSlice q = dq_slice_from(sk.ja, sk.jb, H, k, s, S);
+  const int w_a = q.w_first & ~3;  // 16-byte aligned x coordinate of the box
+  const int nk = q.jb - q.ja;
+  const int j_a = q.ja & ~7;       // 16-byte aligned x coordinate of the side box
+  const bool stage_side = nk > 0 && nk <= kDtMaxStagedKept && q.jb <= j_a + kDtSideCols;
   volatile int* abort = &sm.abort;
 
   if (warp == kDtWarps) {  // ------------------------------------------------ producer
@@ -386,9 +406,22 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
   // ---------------------------------------------------------------------- consumers
   // (the producer is already loading while the consumers set up the slice's constants)
   constexpr int kConsumers = 32 * kDtWarps;
+  if (nk > 8 * kDqSliceGroups && threadIdx.x == 0) record_error(HQ_ERR_BAD_INDEX);
+  if (warp == 0) {  // the 32 groups' layouts from the kept list
+    const int h0 = hs0 + 8 * lane;
+    const GroupLayout L = h0 < H ? group_layout_list(sm.klist, min(nk, 8 * kDqSliceGroups), q.ja, H, k, h0)
+                                 : GroupLayout{0, 0, 0u, 0};
+    sm.gkmask[lane] = L.kmask;
+    sm.gj0[lane] = L.j0;
+  }
   const bool generic = named_barrier_or(kConsumers, dq_has_tiny_scale(scale, P, H, s, kConsumers));
-  dq_fill_constants(s_const, keep_idx, scale, zero, P, H, k, s, generic, kConsumers);
-  const DqLane D = dq_lane(keep_idx, k, H, s, lane, w_a, generic);
+  dq_fill_constants(s_const, keep_idx, sm.gkmask, scale, zero, P, H, k, s, generic, kConsumers);
+  GroupLayout Lg;
+  Lg.kmask = sm.gkmask[lane];
+  Lg.j0 = sm.gj0[lane];
+  Lg.n = 8 - __popc(Lg.kmask);
+  Lg.c0 = min(max(hs0 + 8 * lane - Lg.j0, 0), H - k);
+  const DqLane D = dq_lane_layout(Lg, hs0 + 8 * lane, H, w_a, kDtWords - 2, generic);
   named_barrier_sync(kConsumers);
   float* kept = sm.kept[warp];
   // staged kept sums: pair p = lane + 32c (c < n_slots) is (row p % kDtR, kept feature p / kDtR);
@@ -487,8 +520,8 @@ __global__ void __launch_bounds__(kDqThreads) dequant_reduce_kernel(
 
   const DqSlice q = dq_slice(keep_idx, H, k, s, S);
   const bool generic = __syncthreads_or(dq_has_tiny_scale(scale, P, H, s, kDqThreads)) != 0;
-  const DqLane D = dq_lane(keep_idx, k, H, s, lane, q.w_first, generic);
-  dq_fill_constants(s_const, keep_idx, scale, zero, P, H, k, s, generic, kDqThreads);
+  const DqLane D = dq_lane(keep_idx, k, H, s, lane, q.w_first, kDqWin - 2, generic);
+  dq_fill_constants(s_const, keep_idx, nullptr, scale, zero, P, H, k, s, generic, kDqThreads);
   __syncthreads();
 
   // this warp's row blocks: rows t_first + (warp + kDqWarps*bi)*kDqR + m

@@ -62,6 +62,9 @@ __global__ void __launch_bounds__(kFuThreads, 2) compress_reduce_kernel(
     sm.ring.init(kFuWarps);
     sm.abort = 0;
     fence_barrier_init();
+    // an index outside [0, H) belongs to no slice's groups: the end slices look for one
+    if (k > 0 && ((s == 0 && keep_idx[0] < 0) || (s == S - 1 && keep_idx[k - 1] >= H)))
+      record_error(HQ_ERR_BAD_INDEX);
   }
   __syncthreads();
   volatile int* abort = &sm.abort;

@@ -186,17 +186,28 @@ def test_bounded_wait_times_out_and_context_survives():
     compare_all(cfg, _batches(cfg, cs), synth.fill_cpu(cfg, synth.EVAL, 0, cs=cs))
 
 
-def test_bad_index_is_recorded_not_dereferenced():
-    """keep_idx holding an index outside [0, H): the kernels clamp it and report HQ_ERR_BAD_INDEX."""
-    P, T, H, k = 2, 8, 256, 8
+@pytest.mark.parametrize("H,k", [(256, 8), (4096, 128)], ids=["fallback_dequant", "tma_dequant"])
+@pytest.mark.parametrize("where", ["last", "first"])
+def test_bad_index_is_recorded_not_dereferenced(H, k, where):
+    """keep_idx holding an index outside [0, H): every kernel that reads it clamps it and reports
+    HQ_ERR_BAD_INDEX, and reading the error word clears it."""
+    P, T = 2, 40
     prm = params_to_dev(oracle.get().select_topk(-np.ones((P, H), np.float32), np.ones((P, H), np.float32), k))
     bad = prm["keep_idx"].clone()
-    bad[-1] = H + 1000
+    if where == "last":
+        bad[-1] = H + 1000
+    else:
+        bad[0] = -5
     prm["keep_idx"] = bad
     x = torch.zeros((P, T, H), dtype=torch.int16, device=DEV)
-    gpu_quantize(x, prm)
-    assert hq.hq_read_device_error() == hq.HQ_ERR_BAD_INDEX
+    codes, side = gpu_quantize(x, prm)
+    assert hq.hq_read_device_error() == hq.HQ_ERR_BAD_INDEX, "quantize-pack"
     assert hq.hq_read_device_error() == hq.HQ_OK, "reading clears the word"
+    gpu_dequant(codes, side, prm, H)
+    assert hq.hq_read_device_error() == hq.HQ_ERR_BAD_INDEX, "dequant-reduce"
+    gpu_fused(x, prm)
+    assert hq.hq_read_device_error() == hq.HQ_ERR_BAD_INDEX, "compress-reduce"
+    assert hq.hq_read_device_error() == hq.HQ_OK
 
 
 # ---------------------------------------------------------------------------------------------
