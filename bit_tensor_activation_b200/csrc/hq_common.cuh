@@ -145,17 +145,22 @@ __device__ __forceinline__ GroupLayout group_layout(const int32_t* __restrict__ 
   return L;
 }
 
-// The kept features of a feature range [lo, hi), for a whole CTA at once: ja = #{keep_idx < lo}
-// and jb = #{keep_idx < hi} (the lower bounds when keep_idx is ascending) from one coalesced pass
-// over keep_idx by all blockDim.x threads, and keep_idx[ja .. ja + min(jb-ja, cap)) copied to
-// list.  Every thread of the CTA must call it (it holds __syncthreads); all get ja and jb.
+// The kept features of a feature range [lo, hi), for a group of threads at once: ja =
+// #{keep_idx < lo} and jb = #{keep_idx < hi} (the lower bounds when keep_idx is ascending) from
+// one coalesced pass over keep_idx, and keep_idx[ja .. ja + min(jb-ja, cap)) copied to list.
+// Called by threads 0..nthreads-1 (whole warps), which it synchronises: with __syncthreads when
+// they are the whole CTA, else with named barrier 1.
 struct SliceKept {
   int ja, jb;
 };
-__device__ __forceinline__ SliceKept cta_slice_kept(const int32_t* __restrict__ keep_idx, int k, int lo, int hi,
-                                                    int* s_cnt, int* list, int cap) {
+__device__ __forceinline__ void group_sync(int nthreads) {
+  if (nthreads == (int)blockDim.x) __syncthreads();
+  else asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+}
+__device__ __forceinline__ SliceKept slice_kept(const int32_t* __restrict__ keep_idx, int k, int lo, int hi,
+                                                int* s_cnt, int* list, int cap, int nthreads) {
   int a = 0, b = 0;
-  for (int i = threadIdx.x; i < k; i += blockDim.x) {
+  for (int i = threadIdx.x; i < k; i += nthreads) {
     const int v = __ldg(keep_idx + i);
     a += v < lo;
     b += v < hi;
@@ -166,16 +171,16 @@ __device__ __forceinline__ SliceKept cta_slice_kept(const int32_t* __restrict__ 
     b += __shfl_down_sync(0xFFFFFFFFu, b, off);
   }
   if (threadIdx.x == 0) s_cnt[0] = s_cnt[1] = 0;
-  __syncthreads();
+  group_sync(nthreads);
   if ((threadIdx.x & 31) == 0) {
     atomicAdd(&s_cnt[0], a);
     atomicAdd(&s_cnt[1], b);
   }
-  __syncthreads();
+  group_sync(nthreads);
   const SliceKept r{s_cnt[0], s_cnt[1]};
   const int n = min(r.jb - r.ja, cap);
-  for (int i = threadIdx.x; i < n; i += blockDim.x) list[i] = __ldg(keep_idx + r.ja + i);
-  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += nthreads) list[i] = __ldg(keep_idx + r.ja + i);
+  group_sync(nthreads);
   return r;
 }
 

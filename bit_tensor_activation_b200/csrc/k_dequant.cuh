@@ -369,7 +369,7 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
   }
   // the slice's kept features, counted by the whole CTA (no dependent searches before the loads)
   const int hs0 = 8 * s * kDqSliceGroups, he0 = min(H, hs0 + 8 * kDqSliceGroups);
-  const SliceKept sk = cta_slice_kept(keep_idx, k, hs0, he0, sm.kcnt, sm.klist, 8 * kDqSliceGroups);
+  const SliceKept sk = slice_kept(keep_idx, k, hs0, he0, sm.kcnt, sm.klist, 8 * kDqSliceGroups, kDtThreads);
   const DqSlice q = dq_slice_from(sk.ja, sk.jb, H, k, s, S);
   const int w_a = q.w_first & ~3;  // 16-byte aligned x coordinate of the box
   const int nk = q.jb - q.ja;

@@ -56,6 +56,10 @@ constexpr unsigned kQtTileBytes = kQtTileRows * kQtBoxCols * 2;
 struct QtSmem {
   alignas(128) uint16_t tile[kQtStages][kQtTileRows][kQtBoxCols];
   uint32_t buf[kQtWarps][kQtRowsPerWarp][kQtBufWords];
+  int klist[kQtSlice];  // the slice's kept features
+  int kcnt[2];
+  uint32_t gkmask[kQtSlice / 8];  // per group of the slice: kept mask, kept features before it
+  int gj0[kQtSlice / 8];
   TmaRing<kQtStages> ring;
   int abort;
 };
@@ -66,14 +70,15 @@ struct QtSlice {
   bool halo_staged;  // every halo feature lies in the staged columns [ha, ha + kQtBoxCols)
 };
 
-__device__ __forceinline__ QtSlice qt_slice(const int32_t* __restrict__ keep_idx,
-                                            const int32_t* __restrict__ rest_idx, int H, int k, int s) {
+// ja, jb = number of kept features before ha and before hb.
+__device__ __forceinline__ QtSlice qt_slice(int ja, int jb, const int32_t* __restrict__ rest_idx, int H, int k,
+                                            int s) {
   QtSlice q;
   const int Hr = H - k;
   q.ha = s * kQtSlice;
   q.hb = min(H, q.ha + kQtSlice);
-  q.ja = lower_bound_i32(keep_idx, k, q.ha);
-  q.jb = lower_bound_i32(keep_idx, k, q.hb);
+  q.ja = ja;
+  q.jb = jb;
   q.Ca = min(max(q.ha - q.ja, 0), Hr);
   q.Cb = min(max(q.hb - q.jb, 0), Hr);
   q.Wb = (q.Ca + 7) >> 3;
@@ -135,8 +140,22 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
   const int Hr = H - k, Wr = Hr / 8, NG = H / 8;
   int r = u0 / NB, b = u0 - (u0 / NB) * NB;
   bool fresh = true;  // rank changed: reload this lane's parameters
-  const QtSlice q = qt_slice(keep_idx, rest_idx, H, k, s);
-  if (threadIdx.x == 0 && ((s == 0 && q.ja != 0) || (s == S - 1 && q.jb != k))) record_error(HQ_ERR_BAD_INDEX);
+  // the slice's kept features, counted by the consumer warps (the producer is already loading)
+  constexpr int kConsumers = 32 * kQtWarps;
+  const int ha0 = s * kQtSlice, hb0 = min(H, ha0 + kQtSlice);
+  const SliceKept sk = slice_kept(keep_idx, k, ha0, hb0, sm.kcnt, sm.klist, kQtSlice, kConsumers);
+  const QtSlice q = qt_slice(sk.ja, sk.jb, rest_idx, H, k, s);
+  if (threadIdx.x == 0 && ((s == 0 && q.ja != 0) || (s == S - 1 && q.jb != k) || q.jb - q.ja > kQtSlice))
+    record_error(HQ_ERR_BAD_INDEX);
+  // the groups' layouts, the same for every rank
+  if (warp == 0) {
+    const int g = s * (kQtSlice / 8) + lane;
+    const GroupLayout Lg = g < NG ? group_layout_list(sm.klist, min(q.jb - q.ja, kQtSlice), q.ja, H, k, 8 * g)
+                                  : GroupLayout{0, 0, 0u, 0};
+    sm.gkmask[lane] = Lg.kmask;
+    sm.gj0[lane] = Lg.j0;
+  }
+  group_sync(kConsumers);
   GroupLayout L{0, 0, 0u, 0};
   bool active = false;
   float inv[8];
@@ -187,7 +206,12 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
       const int g = s * (kQtSlice / 8) + lane;
       active = g < NG;
       L = GroupLayout{0, 0, 0u, 0};
-      if (active) L = group_layout(keep_idx, k, H, 8 * g);
+      if (active) {
+        L.kmask = sm.gkmask[lane];
+        L.j0 = sm.gj0[lane];
+        L.n = 8 - __popc(L.kmask);
+        L.c0 = min(max(8 * g - L.j0, 0), Hr);
+      }
       zbase = 0;
       int j = 0;
 #pragma unroll
