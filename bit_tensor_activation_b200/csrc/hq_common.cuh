@@ -32,11 +32,14 @@ __device__ __forceinline__ float bf16_at(const uint4& v, int i) {
 }
 
 // Two fp32 -> two bf16 (round to nearest even), NaN -> 0x7FC0; a in the low half.
+// cvt.rn.bf16x2.f32 writes every NaN, whatever its sign or payload, as 0x7FFF.  Read as signed
+// 16-bit values, every other half it can produce is below 0x7FC0 (finite values and +inf up to
+// 0x7F80, negative values below zero), so one signed 16-bit minimum with 0x7FC0 turns exactly the
+// NaNs into the canonical 0x7FC0 and leaves everything else unchanged.
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
-  if (a != a) r = (r & 0xFFFF0000u) | 0x7FC0u;
-  if (b != b) r = (r & 0x0000FFFFu) | 0x7FC00000u;
+  asm("min.s16x2 %0, %0, %1;" : "+r"(r) : "r"(0x7FC07FC0u));
   return r;
 }
 
