@@ -19,8 +19,9 @@ if not torch.cuda.is_available():
 
 import bit_tensor_activation_b200 as hq  # noqa: E402
 import oracle  # noqa: E402
-from gpu_helpers import (DEV, assert_no_device_error, compare_all, f32bits, gpu_calibrate_batches,  # noqa: E402
-                         gpu_dequant, gpu_fused, gpu_quantize, gpu_select, params_to_dev, to_dev_u16, u16, u32)
+from gpu_helpers import (DEV, assert_no_device_error, assert_same, compare_all, f32bits,  # noqa: E402
+                         gpu_calibrate_batches, gpu_dequant, gpu_fused, gpu_quantize, gpu_select, params_to_dev,
+                         to_dev_u16, u16, u32)
 
 
 def _batches(cfg, cs, T=None):
@@ -279,3 +280,60 @@ def test_full_size_select_quantize_reduce_sampled(name):
         assert np.array_equal(codes_h[:, t:t + 1], c_r), f"codes row {t}"
         assert np.array_equal(side_h[:, t:t + 1], s_r), f"side row {t}"
         assert np.array_equal(out_h[t:t + 1], o_r), f"out row {t}"
+
+
+# ---------------------------------------------------------------------------------------------
+# The 90 sweep workloads at full size, in the launch shapes the sweep tool times
+# ---------------------------------------------------------------------------------------------
+SWEEP = synth.sweep_configs()
+
+
+@pytest.mark.parametrize("cfg", SWEEP, ids=[c.name for c in SWEEP])
+def test_sweep_point_sampled(cfg):
+    """Calibration on sampled columns, selection in full, and quantize-pack, dequant-reduce and the
+    fused call on sampled rows (every feature of each), against the oracle; fused == split over
+    the whole output."""
+    o = oracle.get()
+    P, T, H, k = cfg.P, cfg.T, cfg.H, cfg.k
+    cs, _ = synth.colscale(cfg)
+    cs_dev = torch.from_numpy(cs).to(DEV)
+    buf = torch.empty((P, cfg.calib_T, H), dtype=torch.int16, device=DEV)
+    emin = torch.empty((P, H), dtype=torch.float32, device=DEV)
+    emax = torch.empty_like(emin)
+    for b in range(cfg.calib_batches):
+        synth.fill_gpu(cfg, synth.CALIB, b, buf, cs_dev, T=cfg.calib_T)
+        hq.hq_calibrate(buf, emin, emax, cfg.beta, b == 0)
+    del buf
+    gmin, gmax = emin.cpu().numpy(), emax.cpu().numpy()
+    rng = np.random.default_rng(cfg.seed)
+    for h in rng.choice(H, 3, replace=False):
+        r = int(rng.integers(P))
+        cal = [synth.fill_cpu(cfg, synth.CALIB, b, ranks=(r, r + 1), cols=(int(h), int(h) + 1), T=cfg.calib_T, cs=cs)
+               for b in range(cfg.calib_batches)]
+        em, ex = o.calibrate_batches(cal, cfg.beta)
+        assert f32bits(gmin[r, h]) == f32bits(em[0, 0]) and f32bits(gmax[r, h]) == f32bits(ex[0, 0]), (r, h)
+    sel = o.select_topk(gmin, gmax, k)
+    B = gpu_select(emin, emax, k)
+    for name in ("keep_idx", "rest_idx", "zero"):
+        assert np.array_equal(B[name].cpu().numpy(), sel[name]), name
+    for name in ("scale", "inv_scale"):
+        assert np.array_equal(f32bits(B[name]), f32bits(sel[name])), name
+    x = torch.empty((P, T, H), dtype=torch.int16, device=DEV)
+    synth.fill_gpu(cfg, synth.EVAL, 0, x, cs_dev)
+    codes, side = gpu_quantize(x, B)
+    out = gpu_dequant(codes, side, B, H)
+    fused, _, _ = gpu_fused(x, B)
+    assert_no_device_error()
+    assert torch.equal(out, fused), "fused == split over the whole output"
+    rows = sorted({0, T - 1, int(rng.integers(T)), int(rng.integers(T))})
+    ridx = torch.tensor(rows, device=DEV)
+    codes_h = u32(codes.index_select(1, ridx))
+    side_h = u16(side.index_select(1, ridx))
+    out_h = u16(out.index_select(0, ridx))
+    for i, t in enumerate(rows):
+        xr = synth.fill_cpu(cfg, synth.EVAL, 0, rows=(t, t + 1), cs=cs)
+        c_r, s_r = o.quantize_pack(xr, sel["keep_idx"], sel["rest_idx"], sel["inv_scale"], sel["zero"])
+        o_r = o.dequant_reduce(c_r, s_r, H, sel["keep_idx"], sel["rest_idx"], sel["scale"], sel["zero"])
+        assert_same(codes_h[:, i:i + 1], c_r, f"codes row {t}")
+        assert_same(side_h[:, i:i + 1], s_r, f"side row {t}")
+        assert_same(out_h[i:i + 1], o_r, f"out row {t}")
