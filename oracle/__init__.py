@@ -11,7 +11,7 @@ Every function takes and returns numpy arrays:
   ema_*     float32 [P, H]
   keep_idx  int32 [k], rest_idx int32 [H-k] (both ascending)
   scale, inv_scale float32 [P, H]; zero uint8 [P, H]
-  codes     uint32 [P, T, (H-k)/8]; side uint16 [P, T, k]
+  codes     uint32 [P, T, (H-k)/8]; side uint16 [P, k, T] (feature-major)
   out       uint16 [T, H] (bf16 bits) or float32 [T, H]
 """
 from __future__ import annotations
@@ -126,7 +126,7 @@ class Oracle:
         keep, rest = _c(keep_idx, np.int32), _c(rest_idx, np.int32)
         inv, zero = _c(inv_scale, np.float32), _c(zero, np.uint8)
         codes = np.empty((P, T, (H - k) // 8), np.uint32)
-        side = np.empty((P, T, k), np.uint16)
+        side = np.empty((P, k, T), np.uint16)
         self.lib.hq_ref_quantize_pack(_p(x), P, T, H, k, _p(keep), _p(rest), _p(inv), _p(zero),
                                       _p(codes), _p(side))
         return codes, side

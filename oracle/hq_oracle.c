@@ -25,7 +25,9 @@
  *   R6  q = clamp(rint(x*inv_scale) + zero, 0, 15), round-half-even, the product in fp32;
  *       +-inf saturate; NaN -> q = zero (dequantizes to exactly 0).
  *   R7  wire layout: only the H-k non-kept columns, in rest_idx order, 8 codes per uint32,
- *       code c in bits 4*(c%8)..4*(c%8)+3 of word c/8; k % 8 == 0 and H % 8 == 0.
+ *       code c in bits 4*(c%8)..4*(c%8)+3 of word c/8; k % 8 == 0 and H % 8 == 0.  The kept
+ *       features' bf16 bits travel feature-major, side[r][j][t] (kept feature j in keep_idx
+ *       order, all rows of one feature contiguous).
  *   R9  dequant-reduce of a non-kept column: acc = +0; for r = 0..P-1:
  *       acc = fma(float(q_r - zero_r), scale_r, acc)  (one rounding per rank).
  *   R10 kept column: acc = +0; for r = 0..P-1: acc = acc + float(side_r).
@@ -220,7 +222,7 @@ static unsigned ref_quantize(float v, float inv_scale, unsigned zero) {
 }
 
 /*
- * Inference, sending side: the kept features' bf16 bits go to side[r][t][k] in keep_idx
+ * Inference, sending side: the kept features' bf16 bits go to side[r][j][t] in keep_idx
  * order; every other feature is quantized to 4 bits and packed in rest_idx order into
  * codes[r][t][(H-k)/8] (R6, R7).
  */
@@ -231,9 +233,8 @@ void hq_ref_quantize_pack(const uint16_t* x, int P, int T, int H, int k, const i
   for (int r = 0; r < P; ++r) {
     for (int t = 0; t < T; ++t) {
       const uint16_t* row = x + ((size_t)r * T + t) * H;
-      uint16_t* srow = side + ((size_t)r * T + t) * k;
       uint32_t* crow = codes + ((size_t)r * T + t) * W;
-      for (int j = 0; j < k; ++j) srow[j] = row[keep_idx[j]];
+      for (int j = 0; j < k; ++j) side[((size_t)r * k + j) * T + t] = row[keep_idx[j]];
       for (int w = 0; w < W; ++w) crow[w] = 0u;
       for (int c = 0; c < Hr; ++c) {
         int h = rest_idx[c];
@@ -256,7 +257,7 @@ void hq_ref_dequant_reduce(const uint32_t* codes, const uint16_t* side, int P, i
   for (int t = 0; t < T; ++t) {
     for (int j = 0; j < k; ++j) {
       float acc = 0.0f;
-      for (int r = 0; r < P; ++r) acc = acc + ref_bf16_value(side[((size_t)r * T + t) * k + j]);
+      for (int r = 0; r < P; ++r) acc = acc + ref_bf16_value(side[((size_t)r * k + j) * T + t]);
       size_t o = (size_t)t * H + keep_idx[j];
       if (out_f32) ((float*)out)[o] = ref_canonical(acc);
       else ((uint16_t*)out)[o] = ref_bf16_round(acc);

@@ -266,7 +266,7 @@ def pin_pack_unpack(o):
             for c, h in enumerate(sel["rest_idx"]):
                 want = o.quantize_one(float(f[r, t, h]), float(sel["inv_scale"][r, h]), int(sel["zero"][r, h]))
                 assert q[r, t, c] == want, f"code ({r},{t},col {h})"
-    assert np.array_equal(side, x[:, :, sel["keep_idx"]]), "side"
+    assert np.array_equal(side, x[:, :, sel["keep_idx"]].transpose(0, 2, 1)), "side [P][k][T]"
 
 
 # ---------------------------------------------------------------------------------------------
@@ -333,9 +333,10 @@ def pin_reduce_dequant_sum(o):
     want = terms.sum(axis=0)
     bound = P * 2.0 ** -23 * np.abs(terms).sum(axis=0) + 1e-30
     assert np.all(np.abs(out[:, rest] - want) <= bound), "dequantized sum"
-    kept = bf16_to_f32(side).astype(np.float64).sum(axis=0)
-    assert np.all(np.abs(out[:, keep] - kept) <= P * 2.0 ** -23 * np.abs(bf16_to_f32(side)).sum(axis=0)), "kept sum"
-    assert np.array_equal(out[:, keep], _numpy_rank_sum(bf16_to_f32(side))), "kept: exact rank-ordered sum"
+    sf = bf16_to_f32(side).transpose(0, 2, 1)  # [P][T][k]
+    kept = sf.astype(np.float64).sum(axis=0)
+    assert np.all(np.abs(out[:, keep] - kept) <= P * 2.0 ** -23 * np.abs(sf).sum(axis=0)), "kept sum"
+    assert np.array_equal(out[:, keep], _numpy_rank_sum(sf)), "kept: exact rank-ordered sum"
 
 
 def pin_reduce_error_bound(o):

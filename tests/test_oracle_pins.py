@@ -36,7 +36,8 @@ MUTANTS = [
     ("rint_after_zero", "float n = rintf(a);", "float n = rintf(a + (float)zero) - (float)zero;"),
     ("nan_to_code_0", "if (isnan(a)) return zero;", "if (isnan(a)) return 0u;"),
     ("nibbles_reversed", "crow[c / 8] |= (uint32_t)q << (4 * (c % 8));", "crow[c / 8] |= (uint32_t)q << (4 * (7 - c % 8));"),
-    ("side_from_rest", "srow[j] = row[keep_idx[j]];", "srow[j] = row[rest_idx[j]];"),
+    ("side_from_rest", "* T + t] = row[keep_idx[j]];", "* T + t] = row[rest_idx[j]];"),
+    ("side_row_major", "side[((size_t)r * k + j) * T + t] = row", "side[((size_t)r * T + t) * k + j] = row"),
     ("reduce_drops_last_rank", "for (int r = 0; r < P; ++r) {\n        uint32_t word",
      "for (int r = 0; r < P - 1; ++r) {\n        uint32_t word"),
     ("dequant_sign_flipped", "(float)(q - (int)zero[p])", "(float)((int)zero[p] - q)"),
