@@ -10,7 +10,7 @@ built ``libhq.so`` raises.
 Shapes (P ranks, T rows, H features, k kept features, H' = H - k):
   x [P, T, H] bf16; ema_min/ema_max [P, H] f32; keep_idx [k] i32; rest_idx [H'] i32;
   scale/inv_scale [P, H] f32; zero [P, H] u8; codes [P, T, H'/8] i32 (bit pattern of uint32);
-  side [P, T, k] bf16; out [T, H] bf16 or f32.
+  side [P, k, T] bf16 (feature-major); out [T, H] bf16 or f32.
 """
 from __future__ import annotations
 
@@ -129,7 +129,7 @@ def hq_quantize_pack(x, keep_idx, rest_idx, inv_scale, zero, codes, side, stream
     args = (_ptr(x, _BF16, (P, T, H), "x"), P, T, H, k, _ptr(keep_idx, _I32, (k,), "keep_idx"),
             _ptr(rest_idx, _I32, (H - k,), "rest_idx"), _ptr(inv_scale, _F32, (P, H), "inv_scale"),
             _ptr(zero, _U8, (P, H), "zero"), _ptr(codes, _CODES, (P, T, (H - k) // 8), "codes"),
-            _ptr(side, _BF16, (P, T, k), "side"), _stream(stream, x.device))
+            _ptr(side, _BF16, (P, k, T), "side"), _stream(stream, x.device))
     _check(_lib.hq_quantize_pack(*args), "hq_quantize_pack")
 
 
@@ -140,7 +140,7 @@ def hq_dequant_reduce(codes, side, keep_idx, rest_idx, scale, zero, out, stream=
     if W != (H - k) // 8:
         raise ValueError("codes width does not match H and k")
     odt = HQ_OUT_F32 if out.dtype == torch.float32 else HQ_OUT_BF16
-    args = (_ptr(codes, _CODES, (P, T, W), "codes"), _ptr(side, _BF16, (P, T, k), "side"), P, T, H, k,
+    args = (_ptr(codes, _CODES, (P, T, W), "codes"), _ptr(side, _BF16, (P, k, T), "side"), P, T, H, k,
             _ptr(keep_idx, _I32, (k,), "keep_idx"), _ptr(rest_idx, _I32, (H - k,), "rest_idx"),
             _ptr(scale, _F32, (P, H), "scale"), _ptr(zero, _U8, (P, H), "zero"),
             _ptr(out, _BF16 + _F32, (T, H), "out"), odt, _stream(stream, codes.device))
@@ -156,7 +156,7 @@ def hq_compress_reduce(x, keep_idx, rest_idx, scale, inv_scale, zero, out, codes
             _ptr(rest_idx, _I32, (H - k,), "rest_idx"), _ptr(scale, _F32, (P, H), "scale"),
             _ptr(inv_scale, _F32, (P, H), "inv_scale"), _ptr(zero, _U8, (P, H), "zero"),
             _ptr(out, _BF16 + _F32, (T, H), "out"), odt,
-            _ptr(codes, _CODES, (P, T, (H - k) // 8), "codes"), _ptr(side, _BF16, (P, T, k), "side"),
+            _ptr(codes, _CODES, (P, T, (H - k) // 8), "codes"), _ptr(side, _BF16, (P, k, T), "side"),
             _stream(stream, x.device))
     _check(_lib.hq_compress_reduce(*args), "hq_compress_reduce")
 
@@ -186,5 +186,5 @@ class Buffers:
         self.inv_scale = torch.empty((P, H), dtype=torch.float32, device=dev)
         self.zero = torch.empty((P, H), dtype=torch.uint8, device=dev)
         self.codes = torch.empty((P, T, (H - k) // 8), dtype=torch.int32, device=dev)
-        self.side = torch.empty((P, T, k), dtype=torch.bfloat16, device=dev)
+        self.side = torch.empty((P, k, T), dtype=torch.bfloat16, device=dev)
         self.out = torch.empty((T, H), dtype=out_dtype, device=dev)

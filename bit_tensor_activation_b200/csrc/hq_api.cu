@@ -116,11 +116,13 @@ hq_status launch_dequant(const uint32_t* codes, const uint16_t* side, int P, int
   CUtensorMap map, map_side;
   const bool tma = Wr >= 4 && Wr % 4 == 0 && aligned(codes, 16) &&
                    encode_2d(&map, codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)Wr, (uint64_t)P * T,
-                             hq::kDtWords, hq::kDtTileRows) &&
-                   (k == 0 || encode_2d(&map_side, side, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)k,
-                                        (uint64_t)P * T, hq::kDtSideCols, hq::kDtTileRows,
-                                        CU_TENSOR_MAP_L2_PROMOTION_NONE));
-  if (k == 0) map_side = map;  // never read: no slice stages side values when k == 0
+                             hq::kDtWords, hq::kDtTileRows);
+  // side[r][j][t] as [P*k][T]: boxes of 32 rows (inner) x 32 kept features; needs rows of a
+  // multiple of 16 bytes (T % 8 == 0), else the kept sums read the side buffer directly
+  const bool side_tma = tma && k > 0 && T % 8 == 0 &&
+                        encode_2d(&map_side, side, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)T, (uint64_t)P * k,
+                                  hq::kDtTileRows, hq::kDtSideCols, CU_TENSOR_MAP_L2_PROMOTION_NONE);
+  if (!side_tma) map_side = map;  // never read
   if (tma) {
     const size_t smem = hq::dt_smem_bytes(P);
     auto kern = hq::dequant_reduce_tma_kernel<OutT>;
@@ -132,7 +134,8 @@ hq_status launch_dequant(const uint32_t* codes, const uint16_t* side, int P, int
     if (per_sm < 1) per_sm = 1;
     int chunks, rpc;
     slice_chunks(T, S, (long long)d.sms * per_sm, hq::kDtTileRows, &chunks, &rpc);
-    kern<<<(unsigned)(S * chunks), hq::kDtThreads, smem, st>>>(map, map_side, side, P, T, H, k, keep_idx, scale, zero,
+    kern<<<(unsigned)(S * chunks), hq::kDtThreads, smem, st>>>(map, map_side, side_tma ? 1 : 0, side, P, T, H, k,
+                                                                keep_idx, scale, zero,
                                                                 static_cast<OutT*>(out), S, chunks, rpc,
                                                                 hq::kWaitLimitCycles);
     return launched();

@@ -255,8 +255,8 @@ __device__ __forceinline__ void dq_finish_block(const DqLane& D, float (&acc)[R]
       const int t = t0 + m;
       float a = 0.0f;
       if (t < t_last) {
-        const uint16_t* sp = side + (size_t)t * k + ja + kc + jj;
-        const size_t rank_stride = (size_t)T * k;
+        const uint16_t* sp = side + (size_t)(ja + kc + jj) * T + t;  // side[r][j][t], feature-major
+        const size_t rank_stride = (size_t)k * T;
 #pragma unroll 8
         for (int r = 0; r < P; ++r)
           a = __fadd_rn(a, __uint_as_float((uint32_t)__ldg(sp + r * rank_stride) << 16));
@@ -307,14 +307,14 @@ constexpr int kDtWords = 40;                     // staged words per row (box in
 constexpr int kDtG = 4;                          // ranks per ring slot
 constexpr int kDtStages = 3;
 constexpr unsigned kDtTileBytes = kDtTileRows * kDtWords * 4;
-constexpr int kDtSideCols = 32;                  // side box width (bf16): kept features staged per slice
+constexpr int kDtSideCols = 32;                  // side box height: kept features staged per slice
 constexpr int kDtKeptSlots = 3;                  // (row, kept feature) pairs per lane
 constexpr int kDtMaxStagedKept = 32 * kDtKeptSlots / kDtR;  // slices with more read them from HBM
 constexpr unsigned kDtSideBytes = kDtTileRows * kDtSideCols * 2;
 
 struct DtSmem {
   alignas(128) uint32_t tile[kDtStages][kDtG][kDtTileRows][kDtWords];
-  alignas(128) uint16_t side[kDtStages][kDtG][kDtTileRows][kDtSideCols];
+  alignas(128) uint16_t side[kDtStages][kDtG][kDtSideCols][kDtTileRows];  // [kept feature][row]
   float kept[kDtWarps][kDtR * 32];
   int klist[8 * kDqSliceGroups];  // the slice's kept features
   int kcnt[2];
@@ -347,7 +347,7 @@ __device__ __forceinline__ void dt_slot(const DqLane& D, const DtSmem& sm, int s
 
 template <typename OutT>
 __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_kernel(
-    const __grid_constant__ CUtensorMap tmap_codes, const __grid_constant__ CUtensorMap tmap_side,
+    const __grid_constant__ CUtensorMap tmap_codes, const __grid_constant__ CUtensorMap tmap_side, int side_tma,
     const uint16_t* __restrict__ side, int P, int T, int H,
     int k, const int32_t* __restrict__ keep_idx, const float* __restrict__ scale,
     const uint8_t* __restrict__ zero, OutT* __restrict__ out, int S, int chunks, int rows_per_chunk,
@@ -373,8 +373,8 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
   const DqSlice q = dq_slice_from(sk.ja, sk.jb, H, k, s, S);
   const int w_a = q.w_first & ~3;  // 16-byte aligned x coordinate of the box
   const int nk = q.jb - q.ja;
-  const int j_a = q.ja & ~7;       // 16-byte aligned x coordinate of the side box
-  const bool stage_side = nk > 0 && nk <= kDtMaxStagedKept && q.jb <= j_a + kDtSideCols;
+  // the side box: rows t of the block (inner, 64 bytes) x the slice's kept features from ja on
+  const bool stage_side = side_tma != 0 && nk > 0 && nk <= kDtMaxStagedKept;
   volatile int* abort = &sm.abort;
 
   if (warp == kDtWarps) {  // ------------------------------------------------ producer
@@ -390,7 +390,9 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
         for (int j = 0; j < nr; ++j) {
           const int row = (r0 + j) * T + t_first + bi * kDtTileRows;
           tma_load_2d(&sm.tile[st][j][0][0], &tmap_codes, w_a, row, &sm.ring.full[st]);
-          if (stage_side) tma_load_2d(&sm.side[st][j][0][0], &tmap_side, j_a, row, &sm.ring.full[st]);
+          if (stage_side)
+            tma_load_2d(&sm.side[st][j][0][0], &tmap_side, t_first + bi * kDtTileRows, (r0 + j) * k + q.ja,
+                        &sm.ring.full[st]);
         }
         ++issued;
         if (++g == n_groups) {
@@ -425,7 +427,7 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
   named_barrier_sync(kConsumers);
   float* kept = sm.kept[warp];
   // staged kept sums: pair p = lane + 32c (c < n_slots) is (row p % kDtR, kept feature p / kDtR);
-  // koff[c] = its element offset inside a rank's side tile.  n_slots is the same in every lane;
+  // koff[c] = its element offset inside a rank's side tile ([kept feature][row]).  n_slots is the same in every lane;
   // a lane without a pair in a slot reads element 0 of the tile into a sum it never uses, so
   // the slot loop has no per-lane branch.
   const int n_pairs = stage_side ? kDtR * nk : 0;
@@ -434,7 +436,7 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
 #pragma unroll
   for (int c = 0; c < kDtKeptSlots; ++c) {
     const int p = lane + 32 * c;
-    koff[c] = (p < n_pairs) ? (warp * kDtR + p % kDtR) * kDtSideCols + (q.ja - j_a + p / kDtR) : 0;
+    koff[c] = (p < n_pairs) ? (p / kDtR) * kDtTileRows + warp * kDtR + p % kDtR : 0;
   }
   int st_i = 0;
   unsigned phase = 0;

@@ -167,13 +167,15 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
   uint32_t h_pack[kQtHaloSlots];
   float h_inv[kQtHaloSlots];
   // kept copies: pair p = lane + 32c (c < kQtKeptSlots) is (row lane % 8, kept feature
-  // lane / 8 + 4c), present while lane / 8 + 4c < nk; byte c of k_cols = its column - ha, its
-  // side element (within the unit) is k_side0 + 4c
+  // lane / 8 + 4c), present while lane / 8 + 4c < nk; byte c of k_cols = its column - ha.  The
+  // side buffer is feature-major, side[r][j][t]: the pair's element, counted from the unit's
+  // rank and the warp's first row, is k_side0 + 4c*T, and the 8 rows of one kept feature are
+  // contiguous (the CTA's warps fill 128 contiguous bytes per kept feature and tile).
   const int nk = q.jb - q.ja;
   const bool k_generic = nk > kQtMaxFastKept;
   const int k_m = lane % kQtRowsPerWarp, k_j = lane / kQtRowsPerWarp;
   const int k_row_off = (warp * kQtRowsPerWarp + k_m) * kQtBoxCols;
-  const int k_side0 = k_m * k + q.ja + k_j;
+  const size_t k_side0 = (size_t)(q.ja + k_j) * T + k_m;
   uint32_t k_cols = 0;
 #pragma unroll
   for (int c = 0; c < kQtKeptSlots; ++c) {
@@ -290,17 +292,18 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
       }
     }
     // kept values straight from the staged tile
-    uint16_t* srow = side + ((size_t)r * T + t_base) * k;
+    uint16_t* srow = side + (size_t)r * k * T + t_base;
     if (!k_generic) {
 #pragma unroll
       for (int c = 0; c < kQtKeptSlots; ++c)
-        if (k_j + 4 * c < nk && k_m < nrows) srow[k_side0 + 4 * c] = tile[k_row_off + ((k_cols >> (8 * c)) & 255u)];
+        if (k_j + 4 * c < nk && k_m < nrows)
+          srow[k_side0 + (size_t)(4 * c) * T] = tile[k_row_off + ((k_cols >> (8 * c)) & 255u)];
     } else {
       for (int p = lane; p < nk * kQtRowsPerWarp; p += 32) {
         const int jj = p / kQtRowsPerWarp, m = p % kQtRowsPerWarp;
         if (m < nrows) {
           const int col = checked_col(keep_idx, q.ja + jj, H);
-          srow[(size_t)m * k + q.ja + jj] =
+          srow[(size_t)(q.ja + jj) * T + m] =
               tile[(warp * kQtRowsPerWarp + m) * kQtBoxCols + min(max(col - q.ha, 0), kQtSlice - 1)];
         }
       }

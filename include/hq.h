@@ -95,14 +95,15 @@ hq_status hq_select_topk(const float* ema_min, const float* ema_max, int P, int 
 
 /*
  * Quantize-pack, the sending side of bullet "Inference" (R6, R7).  For every rank r and row t:
- *   side[r][t][j]  = x[r][t][keep_idx[j]]                     (bf16 bits, unchanged)
+ *   side[r][j][t]  = x[r][t][keep_idx[j]]                     (bf16 bits, unchanged)
  *   code of compact column c (feature h = rest_idx[c]):
  *     q = clamp(rint(x * inv_scale[r][h]) + zero[r][h], 0, 15), the product in fp32,
  *     round half to even; +-inf saturate to 15 / 0; NaN gives q = zero[r][h].
  *   codes[r][t][c/8] holds code c in bits 4*(c%8) .. 4*(c%8)+3.
  *   x     bf16 [P][T][H]      (T >= 0; T == 0 enqueues nothing)
  *   codes uint32 [P][T][H'/8] -- the wire buffer of the 4-bit part
- *   side  bf16 [P][T][k]      -- the wire buffer of the BF16 part
+ *   side  bf16 [P][k][T]      -- the wire buffer of the BF16 part, feature-major: the T rows of
+ *                                kept feature j are contiguous
  */
 hq_status hq_quantize_pack(const uint16_t* x, int P, int T, int H, int k, const int32_t* keep_idx,
                            const int32_t* rest_idx, const float* inv_scale, const uint8_t* zero,
@@ -113,7 +114,7 @@ hq_status hq_quantize_pack(const uint16_t* x, int P, int T, int H, int k, const 
  * and the ranks are summed in rank order (R9, R10, R11).  For row t:
  *   non-kept feature h = rest_idx[c]:  acc = +0;  for r = 0..P-1:
  *       acc = fma(float(q_r - zero[r][h]), scale[r][h], acc)      (one rounding per rank)
- *   kept feature h = keep_idx[j]:      acc = +0;  for r = 0..P-1:  acc = acc + side[r][t][j]
+ *   kept feature h = keep_idx[j]:      acc = +0;  for r = 0..P-1:  acc = acc + side[r][j][t]
  *   out[t][h] = acc as fp32 (HQ_OUT_F32), or rounded to bf16 nearest-even (HQ_OUT_BF16); a
  *   NaN sum is written as the canonical quiet NaN (0x7FC00000 / 0x7FC0).
  *   codes, side as written by hq_quantize_pack; out [T][H] of the chosen type.

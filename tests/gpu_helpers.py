@@ -62,7 +62,7 @@ def gpu_quantize(x, prm):
     P, T, H = x.shape
     k = prm["keep_idx"].shape[0]
     codes = torch.empty((P, T, (H - k) // 8), dtype=torch.int32, device=DEV)
-    side = torch.empty((P, T, k), dtype=torch.int16, device=DEV)
+    side = torch.empty((P, k, T), dtype=torch.int16, device=DEV)
     hq.hq_quantize_pack(x, prm["keep_idx"], prm["rest_idx"], prm["inv_scale"], prm["zero"], codes, side)
     return codes, side
 
@@ -81,7 +81,7 @@ def gpu_fused(x, prm, out_f32=False, wire=False):
     codes = side = None
     if wire:
         codes = torch.empty((P, T, (H - k) // 8), dtype=torch.int32, device=DEV)
-        side = torch.empty((P, T, k), dtype=torch.int16, device=DEV)
+        side = torch.empty((P, k, T), dtype=torch.int16, device=DEV)
     hq.hq_compress_reduce(x, prm["keep_idx"], prm["rest_idx"], prm["scale"], prm["inv_scale"], prm["zero"],
                           out, codes, side)
     return out, codes, side

@@ -67,7 +67,7 @@ def test_outputs_stay_in_bounds(cfg):
     hq.hq_select_topk(emin, emax, k, keep, rest, scale, inv, zero)
     x = to_dev_u16(x_np)
     codes = g("codes", (P, T, (H - k) // 8), torch.int32)
-    side = g("side", (P, T, k), torch.int16)
+    side = g("side", (P, k, T), torch.int16)
     hq.hq_quantize_pack(x, keep, rest, inv, zero, codes, side)
     out_b = g("out_bf16", (T, H), torch.int16)
     out_f = g("out_f32", (T, H), torch.float32)
@@ -75,7 +75,7 @@ def test_outputs_stay_in_bounds(cfg):
     hq.hq_dequant_reduce(codes, side, keep, rest, scale, zero, out_f)
     fused = g("fused", (T, H), torch.int16)
     wcodes = g("wire_codes", (P, T, (H - k) // 8), torch.int32)
-    wside = g("wire_side", (P, T, k), torch.int16)
+    wside = g("wire_side", (P, k, T), torch.int16)
     hq.hq_compress_reduce(x, keep, rest, scale, inv, zero, fused, wcodes, wside)
     torch.cuda.synchronize()
     assert_no_device_error()

@@ -278,7 +278,7 @@ def test_full_size_select_quantize_reduce_sampled(name):
         c_r, s_r = o.quantize_pack(xr, sel["keep_idx"], sel["rest_idx"], sel["inv_scale"], sel["zero"])
         o_r = o.dequant_reduce(c_r, s_r, cfg.H, sel["keep_idx"], sel["rest_idx"], sel["scale"], sel["zero"])
         assert np.array_equal(codes_h[:, t:t + 1], c_r), f"codes row {t}"
-        assert np.array_equal(side_h[:, t:t + 1], s_r), f"side row {t}"
+        assert np.array_equal(side_h[:, :, t:t + 1], s_r), f"side row {t}"
         assert np.array_equal(out_h[t:t + 1], o_r), f"out row {t}"
 
 
@@ -328,12 +328,12 @@ def test_sweep_point_sampled(cfg):
     rows = sorted({0, T - 1, int(rng.integers(T)), int(rng.integers(T))})
     ridx = torch.tensor(rows, device=DEV)
     codes_h = u32(codes.index_select(1, ridx))
-    side_h = u16(side.index_select(1, ridx))
+    side_h = u16(side.index_select(2, ridx))
     out_h = u16(out.index_select(0, ridx))
     for i, t in enumerate(rows):
         xr = synth.fill_cpu(cfg, synth.EVAL, 0, rows=(t, t + 1), cs=cs)
         c_r, s_r = o.quantize_pack(xr, sel["keep_idx"], sel["rest_idx"], sel["inv_scale"], sel["zero"])
         o_r = o.dequant_reduce(c_r, s_r, H, sel["keep_idx"], sel["rest_idx"], sel["scale"], sel["zero"])
         assert_same(codes_h[:, i:i + 1], c_r, f"codes row {t}")
-        assert_same(side_h[:, i:i + 1], s_r, f"side row {t}")
+        assert_same(side_h[:, :, i:i + 1], s_r, f"side row {t}")
         assert_same(out_h[i:i + 1], o_r, f"out row {t}")
