@@ -10,8 +10,10 @@
 // ranks in order.  The CTA's warps share the slice's per-(rank, feature) constants in shared
 // memory.  Two ways of staging the code words:
 //   - dequant_reduce_tma_kernel (default): a producer warp loads, per (32-row block, rank), one
-//     32 x 40-word TMA tile into an 8-stage mbarrier ring; eight consumer warps take 4 rows each.
-//     Needs code rows whose byte length is a multiple of 16 ((H-k) % 32 == 0).
+//     32 x 40-word TMA tile (and a 32-row x 32-feature tile of the side buffer) into a 3-stage
+//     mbarrier ring whose slots hold 4 ranks; eight consumer warps take 4 rows each and a
+//     kept-sum warp sums the staged side values.  Needs code rows whose byte length is a
+//     multiple of 16 ((H-k) % 32 == 0).
 //   - dequant_reduce_kernel (any shape): each warp stages its own rows with 4-byte cp.async
 //     copies, 8 tiles ahead.
 //
@@ -24,8 +26,9 @@
 // v2 = v >> 4b.  Scales below 2^-109 could lose bits when divided by 16^4: a slice that has one
 // decodes with explicit shifts and undivided constants instead ("generic" path).  Adds and FMAs
 // go two at a time through add/fma.rn.f32x2 (per-lane IEEE, so bit-identical).  A kept feature
-// gets scale 0 (its decoded value is then multiplied by 0); its sum over the side values is
-// formed by "kept lanes" and written into the owner's registers through a small warp buffer.
+// gets scale 0 (its decoded value is then multiplied by 0); its sum over the side values, in
+// rank order, is formed elsewhere (the kept-sum warp, or lanes of the owning warp reading the
+// side buffer) and copied over the owner's sum through shared memory.
 //
 // Roofline: HBM-bound; per output element P*(0.5*H'/H + 2*k/H) bytes read + 2 (or 4) written.
 // No memory beyond the inputs and outputs is used.
@@ -299,7 +302,8 @@ __device__ __forceinline__ DqSlice dq_slice(const int32_t* __restrict__ keep_idx
 // rows, so a consumer warp waits and releases once per kDtG ranks, and the rank loop inside a
 // slot has no synchronisation in it.
 constexpr int kDtWarps = 8;                      // consumer warps
-constexpr int kDtThreads = 32 * (kDtWarps + 1);  // + one producer warp
+constexpr int kDtKeptWarp = kDtWarps + 1;        // the kept-sum warp (warp kDtWarps loads)
+constexpr int kDtThreads = 32 * (kDtWarps + 2);  // + the producer warp + the kept-sum warp
 constexpr int kDtR = 4;                          // rows per consumer warp per block
 constexpr int kDtMinBlocks = 2;                  // CTAs per SM the register budget is set for
 constexpr int kDtTileRows = kDtWarps * kDtR;     // 32
@@ -308,14 +312,20 @@ constexpr int kDtG = 4;                          // ranks per ring slot
 constexpr int kDtStages = 3;
 constexpr unsigned kDtTileBytes = kDtTileRows * kDtWords * 4;
 constexpr int kDtSideCols = 32;                  // side box height: kept features staged per slice
-constexpr int kDtKeptSlots = 3;                  // (row, kept feature) pairs per lane
-constexpr int kDtMaxStagedKept = 32 * kDtKeptSlots / kDtR;  // slices with more read them from HBM
+constexpr int kDtMaxStagedKept = kDtSideCols;    // slices with more read the side buffer from HBM
 constexpr unsigned kDtSideBytes = kDtTileRows * kDtSideCols * 2;
+static_assert(kDtR == 4, "a consumer lane reads its rows' kept sums as one float4");
+static_assert(kDtTileRows == 32, "the kept-sum warp gives one lane to each row of a block");
 
 struct DtSmem {
   alignas(128) uint32_t tile[kDtStages][kDtG][kDtTileRows][kDtWords];
   alignas(128) uint16_t side[kDtStages][kDtG][kDtSideCols][kDtTileRows];  // [kept feature][row]
-  float kept[kDtWarps][kDtR * 32];
+  union {
+    float kept[kDtWarps][kDtR * 32];           // side read from HBM: per-warp kept sums
+    float ksum[2][kDtSideCols][kDtTileRows];   // side staged: a block's kept sums, [kept feature][row]
+  } k;
+  uint64_t ksum_full[2];   // the kept-sum warp has written ksum[b]
+  uint64_t ksum_empty[2];  // every consumer warp has read ksum[b]
   int klist[8 * kDqSliceGroups];  // the slice's kept features
   int kcnt[2];
   uint32_t gkmask[kDqSliceGroups];  // per group of the slice: kept mask and kept features before it
@@ -328,19 +338,92 @@ struct DtSmem {
 inline size_t dt_smem_bytes(int P) { return sizeof(DtSmem) + 128 + (size_t)P * 4 * 32 * 16; }
 
 // The nr ranks of one ring slot, in rank order: 4-bit features of the warp's rows into acc
-// (cst = this lane's constants of the slot's first rank), the first NS kept-pair slots into
-// kacc.
-template <bool kFast, int NS>
+// (cst = this lane's constants of the slot's first rank).
+template <bool kFast>
 __device__ __forceinline__ void dt_slot(const DqLane& D, const DtSmem& sm, int st_i, int warp, int nr,
-                                        const float4* __restrict__ cst, const int (&koff)[kDtKeptSlots],
-                                        float (&acc)[kDtR][8], float (&kacc)[kDtKeptSlots]) {
+                                        const float4* __restrict__ cst, float (&acc)[kDtR][8]) {
 #pragma unroll
-  for (int j = 0; j < kDtG; ++j) {
-    if (j < nr) {
-      if (D.decode) dq_decode_rows<kFast, kDtR>(D, &sm.tile[st_i][j][warp * kDtR][0], kDtWords, cst + j * 4 * 32, acc);
-      const uint16_t* sside = &sm.side[st_i][j][0][0];
+  for (int j = 0; j < kDtG; ++j)
+    if (j < nr && D.decode)
+      dq_decode_rows<kFast, kDtR>(D, &sm.tile[st_i][j][warp * kDtR][0], kDtWords, cst + j * 4 * 32, acc);
+}
+
+// The kept-sum warp, for slices whose side values are staged: lane l sums rows 4(l % 8) ..
+// 4(l % 8) + 3 of kept features l / 8, l / 8 + 4, ... (< nk <= NK) over the ranks in order, four
+// rows per 8-byte load of a side tile; the sums of block bi go to ksum[bi & 1].  It releases ring
+// slots like a consumer warp.
+template <int NK>
+__device__ __forceinline__ void dt_kept_sums(DtSmem& sm, int nk, int P, int nblk, int n_groups,
+                                             volatile int* abort, long long wait_limit) {
+  constexpr int NF = NK / 4;  // kept features per lane
+  const int lane = threadIdx.x & 31;
+  const int m0 = 4 * (lane & 7), f0 = lane >> 3;
+  int st_i = 0;
+  unsigned phase = 0;
+  for (int bi = 0; bi < nblk && !*abort; ++bi) {
+    float a[NF][4];
 #pragma unroll
-      for (int c = 0; c < NS; ++c) kacc[c] = __fadd_rn(kacc[c], __uint_as_float((uint32_t)sside[koff[c]] << 16));
+    for (int i = 0; i < NF; ++i)
+#pragma unroll
+      for (int m = 0; m < 4; ++m) a[i][m] = 0.0f;
+    bool ok = true;
+    for (int g = 0; g < n_groups; ++g) {
+      if (!mbar_wait(&sm.ring.full[st_i], phase, abort, wait_limit)) {
+        ok = false;
+        break;
+      }
+      const int nr = min(kDtG, P - g * kDtG);
+#pragma unroll
+      for (int j = 0; j < kDtG; ++j) {
+        if (j < nr) {
+#pragma unroll
+          for (int i = 0; i < NF; ++i) {
+            if (f0 + 4 * i < nk) {
+              const uint2 w = *reinterpret_cast<const uint2*>(&sm.side[st_i][j][f0 + 4 * i][m0]);
+              fadd2(a[i][0], a[i][1], a[i][0], a[i][1], __uint_as_float(w.x << 16),
+                    __uint_as_float(w.x & 0xFFFF0000u));
+              fadd2(a[i][2], a[i][3], a[i][2], a[i][3], __uint_as_float(w.y << 16),
+                    __uint_as_float(w.y & 0xFFFF0000u));
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.ring.empty[st_i]);
+      if (++st_i == kDtStages) {
+        st_i = 0;
+        phase ^= 1u;
+      }
+    }
+    if (!ok) break;
+    const int buf = bi & 1;
+    if (bi >= 2 && !mbar_wait(&sm.ksum_empty[buf], ((bi >> 1) - 1) & 1, abort, wait_limit)) break;
+#pragma unroll
+    for (int i = 0; i < NF; ++i)
+      if (f0 + 4 * i < nk)
+        *reinterpret_cast<float4*>(&sm.k.ksum[buf][f0 + 4 * i][m0]) = make_float4(a[i][0], a[i][1], a[i][2], a[i][3]);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.ksum_full[buf]);
+  }
+}
+
+// Owners of the slice's kept features take the sums of the warp's kDtR rows from one ksum buffer.
+__device__ __forceinline__ void dt_patch_kept(const DqLane& D, float (&acc)[kDtR][8], const float* ksum, int ja,
+                                              int nk, int warp) {
+  if (D.L.kmask) {
+    int jj = D.L.j0 - ja;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if ((D.L.kmask >> i) & 1u) {
+        if (jj >= 0 && jj < nk) {
+          const float4 v = reinterpret_cast<const float4*>(ksum + jj * kDtTileRows)[warp];
+          acc[0][i] = v.x;
+          acc[1][i] = v.y;
+          acc[2][i] = v.z;
+          acc[3][i] = v.w;
+        }
+        ++jj;
+      }
     }
   }
 }
@@ -363,7 +446,11 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
   const int n_slots_total = nblk * n_groups;     // slot i = (block i / n_groups, rank group i % n_groups)
 
   if (threadIdx.x == 0) {
-    sm.ring.init(kDtWarps);
+    sm.ring.init(kDtWarps + 1);  // the consumer warps and the kept-sum warp release each slot
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.ksum_full[b], 1);
+      mbar_init(&sm.ksum_empty[b], kDtWarps);
+    }
     sm.abort = 0;
     fence_barrier_init();
   }
@@ -405,6 +492,26 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
     return;
   }
 
+  if (warp == kDtKeptWarp) {  // ------------------------------------------ kept sums
+    if (stage_side) {
+      if (nk <= 8) dt_kept_sums<8>(sm, nk, P, nblk, n_groups, abort, wait_limit);
+      else if (nk <= 16) dt_kept_sums<16>(sm, nk, P, nblk, n_groups, abort, wait_limit);
+      else dt_kept_sums<kDtSideCols>(sm, nk, P, nblk, n_groups, abort, wait_limit);
+    } else if (lane == 0) {  // only releases the ring slots
+      int st_i = 0;
+      unsigned phase = 0;
+      for (int i = 0; i < n_slots_total; ++i) {
+        if (!mbar_wait(&sm.ring.full[st_i], phase, abort, wait_limit)) break;
+        mbar_arrive(&sm.ring.empty[st_i]);
+        if (++st_i == kDtStages) {
+          st_i = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    return;
+  }
+
   // ---------------------------------------------------------------------- consumers
   // (the producer is already loading while the consumers set up the slice's constants)
   constexpr int kConsumers = 32 * kDtWarps;
@@ -425,19 +532,6 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
   Lg.c0 = min(max(hs0 + 8 * lane - Lg.j0, 0), H - k);
   const DqLane D = dq_lane_layout(Lg, hs0 + 8 * lane, H, w_a, kDtWords - 2, generic);
   named_barrier_sync(kConsumers);
-  float* kept = sm.kept[warp];
-  // staged kept sums: pair p = lane + 32c (c < n_slots) is (row p % kDtR, kept feature p / kDtR);
-  // koff[c] = its element offset inside a rank's side tile ([kept feature][row]).  n_slots is the same in every lane;
-  // a lane without a pair in a slot reads element 0 of the tile into a sum it never uses, so
-  // the slot loop has no per-lane branch.
-  const int n_pairs = stage_side ? kDtR * nk : 0;
-  const int n_slots = (n_pairs + 31) >> 5;
-  int koff[kDtKeptSlots];
-#pragma unroll
-  for (int c = 0; c < kDtKeptSlots; ++c) {
-    const int p = lane + 32 * c;
-    koff[c] = (p < n_pairs) ? (p / kDtR) * kDtTileRows + warp * kDtR + p % kDtR : 0;
-  }
   int st_i = 0;
   unsigned phase = 0;
   for (int bi = 0; bi < nblk && !*abort; ++bi) {
@@ -447,9 +541,6 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
     for (int m = 0; m < kDtR; ++m)
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[m][e] = 0.0f;
-    float kacc[kDtKeptSlots];
-#pragma unroll
-    for (int c = 0; c < kDtKeptSlots; ++c) kacc[c] = 0.0f;
     bool ok = true;
     for (int g = 0; g < n_groups; ++g) {
       if (!mbar_wait(&sm.ring.full[st_i], phase, abort, wait_limit)) {
@@ -458,16 +549,8 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
       }
       const int nr = min(kDtG, P - g * kDtG);
       const float4* cst = s_const + (size_t)g * kDtG * 4 * 32 + lane;
-      if (generic) {
-        dt_slot<false, kDtKeptSlots>(D, sm, st_i, warp, nr, cst, koff, acc, kacc);
-      } else {
-        switch (n_slots) {  // the same in every lane of the CTA
-          case 0: dt_slot<true, 0>(D, sm, st_i, warp, nr, cst, koff, acc, kacc); break;
-          case 1: dt_slot<true, 1>(D, sm, st_i, warp, nr, cst, koff, acc, kacc); break;
-          case 2: dt_slot<true, 2>(D, sm, st_i, warp, nr, cst, koff, acc, kacc); break;
-          default: dt_slot<true, kDtKeptSlots>(D, sm, st_i, warp, nr, cst, koff, acc, kacc); break;
-        }
-      }
+      if (generic) dt_slot<false>(D, sm, st_i, warp, nr, cst, acc);
+      else dt_slot<true>(D, sm, st_i, warp, nr, cst, acc);
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.ring.empty[st_i]);
       if (++st_i == kDtStages) {
@@ -477,17 +560,14 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
     }
     if (!ok) break;
     if (stage_side) {
-#pragma unroll
-      for (int c = 0; c < kDtKeptSlots; ++c) {
-        const int p = lane + 32 * c;
-        if (p < n_pairs) kept[(p % kDtR) * 32 + p / kDtR] = kacc[c];
-      }
+      const int buf = bi & 1;
+      if (!mbar_wait(&sm.ksum_full[buf], (bi >> 1) & 1, abort, wait_limit)) break;
+      dt_patch_kept(D, acc, &sm.k.ksum[buf][0][0], q.ja, nk, warp);
       __syncwarp();
-      dq_patch_kept<kDtR>(D, acc, kept, q.ja, 0, nk);
-      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.ksum_empty[buf]);
       dq_store_rows<OutT, kDtR>(D, acc, H, t0, t_last, out);
     } else {
-      dq_finish_block<OutT, kDtR>(D, acc, side, kept, P, T, H, k, q.ja, q.jb, t0, t_last, out);
+      dq_finish_block<OutT, kDtR>(D, acc, side, sm.k.kept[warp], P, T, H, k, q.ja, q.jb, t0, t_last, out);
     }
   }
 }

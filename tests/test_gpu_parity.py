@@ -95,6 +95,41 @@ def test_clustered_kept_features_bit_exact(P, T, H, k, big):
     assert np.array_equal(u16(out), out_r) and np.array_equal(u16(fused), out_r)
 
 
+# Kept features per 256-feature slice of H = 4096, planted: every count the kept-sum paths of the
+# TMA dequant-reduce distinguish (none, up to 8, 16 and 32 staged kept features, more than fit the
+# staged side tile), with row counts that give a CTA one row block or several.
+SLICE_KEPT = [0, 1, 3, 4, 5, 7, 8, 9, 15, 16, 17, 24, 31, 32, 33, 19]
+
+
+@pytest.mark.parametrize("P,T", [(5, 72), (8, 72), (2, 2048), (4, 4096)])
+def test_kept_counts_per_slice_bit_exact(P, T):
+    o = oracle.get()
+    H = 4096
+    rng = np.random.default_rng(11)
+    big = np.sort(np.concatenate([256 * s + rng.choice(256, n, replace=False) for s, n in enumerate(SLICE_KEPT)]))
+    k = len(big)
+    assert (H - k) % 32 == 0 and T % 8 == 0  # code rows and side rows both staged by TMA
+    x = synth.fill_cpu(synth.CONFIGS["decode"].with_(P=P, T=T, H=H, n_out=4), synth.EVAL, 0, cs=np.ones(H))
+    emin = -np.ones((P, H), np.float32) - rng.uniform(0, 0.01, (P, H)).astype(np.float32)
+    emax = np.ones((P, H), np.float32)
+    emax[:, big] = 40.0
+    sel = o.select_topk(emin, emax, k)
+    assert np.array_equal(sel["keep_idx"], big)
+    prm = params_to_dev(sel)
+    codes_r, side_r = o.quantize_pack(x, sel["keep_idx"], sel["rest_idx"], sel["inv_scale"], sel["zero"])
+    out_r = o.dequant_reduce(codes_r, side_r, H, sel["keep_idx"], sel["rest_idx"], sel["scale"], sel["zero"])
+    out_rf = o.dequant_reduce(codes_r, side_r, H, sel["keep_idx"], sel["rest_idx"], sel["scale"], sel["zero"],
+                              out_f32=True)
+    codes, side = gpu_quantize(to_dev_u16(x), prm)
+    out = gpu_dequant(codes, side, prm, H)
+    out_f = gpu_dequant(codes, side, prm, H, out_f32=True)
+    assert_no_device_error()
+    assert_same(u32(codes), codes_r, "codes")
+    assert_same(u16(side), side_r, "side")
+    assert_same(u16(out), out_r, "out bf16")
+    assert_same(f32bits(out_f), f32bits(out_rf), "out f32")
+
+
 def test_select_ties_and_special_values():
     o = oracle.get()
     P, H = 3, 4096
