@@ -24,11 +24,11 @@
 // gives (q - zero)*16^p_i exactly, and the FMA uses scale/16^p_i, so the product is exactly
 // (q - zero)*scale.  p_i <= 4 is arranged by reading features 5..7 from a second view
 // v2 = v >> 4b.  Scales below 2^-109 could lose bits when divided by 16^4: a slice that has one
-// decodes with explicit shifts and undivided constants instead ("generic" path).  Adds and FMAs
-// go two at a time through add/fma.rn.f32x2 (per-lane IEEE, so bit-identical).  A kept feature
-// gets scale 0 (its decoded value is then multiplied by 0); its sum over the side values, in
-// rank order, is formed elsewhere (the kept-sum warp, or lanes of the owning warp reading the
-// side buffer) and copied over the owner's sum through shared memory.
+// decodes with explicit shifts and undivided constants instead ("generic" path).  The adds are
+// scalar and the FMAs go two at a time through fma.rn.f32x2 (per-lane IEEE, so bit-identical).
+// A kept feature gets scale 0 (its decoded value is then multiplied by 0); its sum over the side
+// values, in rank order, is formed elsewhere (the kept-sum warp, or lanes of the owning warp
+// reading the side buffer) and copied over the owner's sum through shared memory.
 //
 // Roofline: HBM-bound; per output element P*(0.5*H'/H + 2*k/H) bytes read + 2 (or 4) written.
 // No memory beyond the inputs and outputs is used.
@@ -199,10 +199,11 @@ __device__ __forceinline__ void dq_decode_rows(const DqLane& D, const uint32_t* 
 #pragma unroll
       for (int i = 0; i < 8; ++i) q[i] = __uint_as_float(((v >> D.key[i]) & 0xFu) | 0x4B000000u);
     }
+    // Scalar adds (exact: (q - zero) * 16^p) write their results straight into the register pair
+    // the packed FMA reads; a packed add would need its two LOP3 inputs moved into a pair first.
 #pragma unroll
     for (int i = 0; i < 8; i += 2) {
-      float d0, d1;
-      fadd2(d0, d1, q[i], q[i + 1], off[i], off[i + 1]);  // (q - zero) * 16^p, exact
+      const float d0 = __fadd_rn(q[i], off[i]), d1 = __fadd_rn(q[i + 1], off[i + 1]);
       ffma2_acc(acc[m][i], acc[m][i + 1], d0, d1, sc[i], sc[i + 1]);
     }
   }

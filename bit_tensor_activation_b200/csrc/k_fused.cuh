@@ -159,9 +159,10 @@ __global__ void __launch_bounds__(kFuThreads, 2) compress_reduce_kernel(
             int c0 = __float2int_rn(a0), c1 = __float2int_rn(a1);  // saturating; NaN -> 0
             c0 = min(max(c0, lo[e]), lo[e] + 15);
             c1 = min(max(c1, lo[e + 1]), lo[e + 1] + 15);
-            float d0, d1;
-            fadd2(d0, d1, __int_as_float(c0 + 0x4B400000), __int_as_float(c1 + 0x4B400000), -12582912.0f,
-                  -12582912.0f);
+            // float(c) by the 1.5 * 2^23 magic, as scalar adds: their results go straight into the
+            // register pair the packed FMA reads
+            const float d0 = __fadd_rn(__int_as_float(c0 + 0x4B400000), -12582912.0f);
+            const float d1 = __fadd_rn(__int_as_float(c1 + 0x4B400000), -12582912.0f);
             const float v0 = ((kmask >> e) & 1u) ? f0 : d0;
             const float v1 = ((kmask >> (e + 1)) & 1u) ? f1 : d1;
             ffma2_acc(acc[m][e], acc[m][e + 1], v0, v1, sc[e], sc[e + 1]);
