@@ -58,6 +58,8 @@ class Oracle:
         lib.hq_ref_quantize_pack.restype = None
         lib.hq_ref_dequant_reduce.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, i32]
         lib.hq_ref_dequant_reduce.restype = None
+        lib.hq_ref_dequant_reduce_bf16_shards.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, i32]
+        lib.hq_ref_dequant_reduce_bf16_shards.restype = None
         lib.hq_ref_compress_reduce.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, i32, vp, vp]
         lib.hq_ref_compress_reduce.restype = i32
         lib.hq_ref_bf16_round.argtypes = [f32]
@@ -131,15 +133,17 @@ class Oracle:
                                       _p(codes), _p(side))
         return codes, side
 
-    def dequant_reduce(self, codes, side, H, keep_idx, rest_idx, scale, zero, out_f32=False):
+    def dequant_reduce(self, codes, side, H, keep_idx, rest_idx, scale, zero, out_f32=False, bf16_shards=False):
+        """R9/R10/R11; bf16_shards=True: the literal variant R19 (each rank's dequantized value
+        rounded to bf16 before the rank-ordered sum)."""
         codes, side = _c(codes, np.uint32), _c(side, np.uint16)
         P, T = codes.shape[0], codes.shape[1]
         k = len(keep_idx)
         keep, rest = _c(keep_idx, np.int32), _c(rest_idx, np.int32)
         scale, zero = _c(scale, np.float32), _c(zero, np.uint8)
         out = np.empty((T, H), np.float32 if out_f32 else np.uint16)
-        self.lib.hq_ref_dequant_reduce(_p(codes), _p(side), P, T, H, k, _p(keep), _p(rest), _p(scale),
-                                       _p(zero), _p(out), int(bool(out_f32)))
+        fn = self.lib.hq_ref_dequant_reduce_bf16_shards if bf16_shards else self.lib.hq_ref_dequant_reduce
+        fn(_p(codes), _p(side), P, T, H, k, _p(keep), _p(rest), _p(scale), _p(zero), _p(out), int(bool(out_f32)))
         return out
 
     def compress_reduce(self, x, keep_idx, rest_idx, scale, inv_scale, zero, out_f32=False):

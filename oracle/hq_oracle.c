@@ -35,6 +35,12 @@
  *       canonical quiet NaN in both types (0x7FC00000 / 0x7FC0).
  *   R12 the fused compress-reduce equals quantize-pack followed by dequant-reduce.
  *   R14 parameters are computed for every column, kept ones included (unused there).
+ *   R19 the literal variant of the receiving side (every received tensor made BF16 before the
+ *       devices' tensors are combined): each
+ *       rank's dequantized value v_r = float(q_r - zero_r) * scale_r (one fp32 product) is
+ *       rounded to bf16 (nearest, ties to even) before the rank-ordered fp32 sum:
+ *       acc = +0; for r = 0..P-1: acc = acc + bf16(v_r).  Kept columns and the output
+ *       rounding are as in R10 and R11.
  * Calibration detail: batch min/max ignore NaN (no comparison with NaN is true); a batch
  * minimum or maximum of -0 is stored as +0 (adding +0.0f), so that results do not depend
  * on which zero a comparison happened to keep.
@@ -247,12 +253,15 @@ void hq_ref_quantize_pack(const uint16_t* x, int P, int T, int H, int k, const i
 }
 
 /*
- * Inference, receiving side: every rank's shard is converted back and the ranks are summed
- * in rank order (R9, R10); out is [T][H], fp32 (out_f32 != 0) or bf16 bits (R11).
+ * Inference, receiving side (section "The Hybrid Quantization Algorithm", bullet "Inference"):
+ * every rank's shard is converted back and the ranks are summed in rank order; out is [T][H],
+ * fp32 (out_f32 != 0) or bf16 bits (R11).  shard_bf16 == 0: a non-kept value enters the sum
+ * through one fused multiply-add per rank (R9).  shard_bf16 != 0: the literal reading, each
+ * rank's dequantized value is first rounded to bf16 (R19).  Kept columns: R10 in both.
  */
-void hq_ref_dequant_reduce(const uint32_t* codes, const uint16_t* side, int P, int T, int H, int k,
-                           const int32_t* keep_idx, const int32_t* rest_idx, const float* scale,
-                           const uint8_t* zero, void* out, int out_f32) {
+static void ref_dequant_reduce(const uint32_t* codes, const uint16_t* side, int P, int T, int H, int k,
+                               const int32_t* keep_idx, const int32_t* rest_idx, const float* scale,
+                               const uint8_t* zero, void* out, int out_f32, int shard_bf16) {
   const int Hr = H - k, W = Hr / 8;
   for (int t = 0; t < T; ++t) {
     for (int j = 0; j < k; ++j) {
@@ -269,13 +278,30 @@ void hq_ref_dequant_reduce(const uint32_t* codes, const uint16_t* side, int P, i
         uint32_t word = codes[((size_t)r * T + t) * W + c / 8];
         int q = (int)((word >> (4 * (c % 8))) & 0xFu);
         size_t p = (size_t)r * H + h;
-        acc = fmaf((float)(q - (int)zero[p]), scale[p], acc);
+        if (shard_bf16) {
+          float v = (float)(q - (int)zero[p]) * scale[p];
+          acc = acc + ref_bf16_value(ref_bf16_round(v));
+        } else {
+          acc = fmaf((float)(q - (int)zero[p]), scale[p], acc);
+        }
       }
       size_t o = (size_t)t * H + h;
       if (out_f32) ((float*)out)[o] = ref_canonical(acc);
       else ((uint16_t*)out)[o] = ref_bf16_round(acc);
     }
   }
+}
+
+void hq_ref_dequant_reduce(const uint32_t* codes, const uint16_t* side, int P, int T, int H, int k,
+                           const int32_t* keep_idx, const int32_t* rest_idx, const float* scale,
+                           const uint8_t* zero, void* out, int out_f32) {
+  ref_dequant_reduce(codes, side, P, T, H, k, keep_idx, rest_idx, scale, zero, out, out_f32, 0);
+}
+
+void hq_ref_dequant_reduce_bf16_shards(const uint32_t* codes, const uint16_t* side, int P, int T, int H,
+                                       int k, const int32_t* keep_idx, const int32_t* rest_idx,
+                                       const float* scale, const uint8_t* zero, void* out, int out_f32) {
+  ref_dequant_reduce(codes, side, P, T, H, k, keep_idx, rest_idx, scale, zero, out, out_f32, 1);
 }
 
 /* The fused call: quantize-pack then dequant-reduce, literally (R12).  codes/side may be

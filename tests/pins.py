@@ -449,10 +449,90 @@ def pin_selection_benefit(o):
     assert rand > 0.7 * none, f"random-k MSE {rand} vs pure Int4 {none}"
 
 
+# ---------------------------------------------------------------------------------------------
+# Dequant-reduce, literal variant: each rank's dequantized value rounded to bf16 (reading R19)
+# ---------------------------------------------------------------------------------------------
+def _one_group(qz_rows, scale_rows):
+    """Codes, zero points and scales for one 8-feature group of P ranks and one row, with
+    q - zero = qz_rows[r][i] in -15..15 (zero = max(0, -(q - zero)), so both stay in 0..15)."""
+    qz = np.asarray(qz_rows, np.int64)
+    P, n = qz.shape
+    zero = np.zeros((P, 8), np.uint8)
+    q = np.zeros((P, 8), np.int64)
+    zero[:, :n] = np.maximum(0, -qz)
+    q[:, :n] = qz + zero[:, :n]
+    words = np.zeros((P, 1, 1), np.uint32)
+    for r in range(P):
+        words[r, 0, 0] = sum(int(q[r, i]) << (4 * i) for i in range(8))
+    scale = np.ones((P, 8), np.float32)
+    scale[:, :n] = np.asarray(scale_rows, np.float32)
+    return words, zero, scale
+
+
+def pin_bf16_shards_golden(o):
+    """Values worked by hand (tests/golden/bf16_shards_cases.json): ties go to the even bf16
+    neighbour, each shard is rounded before the fp32 rank sum, the sum itself is not."""
+    g = _golden("bf16_shards_cases.json")
+    cases = g["cases"]
+    assert len(cases) == 8
+    words, zero, scale = _one_group([[c["qz"][r] for c in cases] for r in range(g["P"])],
+                                    [[c["scale"][r] for c in cases] for r in range(g["P"])])
+    keep, rest = np.zeros(0, np.int32), np.arange(8, dtype=np.int32)
+    side = np.zeros((g["P"], 0, 1), np.uint16)
+    lit = o.dequant_reduce(words, side, 8, keep, rest, scale, zero, out_f32=True, bf16_shards=True)
+    std = o.dequant_reduce(words, side, 8, keep, rest, scale, zero, out_f32=True)
+    for i, c in enumerate(cases):
+        assert f32_bits(lit[0, i]) == f32_bits(c["f32"]), f"case {i} ({c['why']}): {lit[0, i]} != {c['f32']}"
+        assert f32_bits(std[0, i]) == f32_bits(c["std"]), f"case {i} standard reading: {std[0, i]} != {c['std']}"
+
+
+def _random_wire(rng, P, T, H, k, scale):
+    zero = rng.integers(0, 16, (P, H)).astype(np.uint8)
+    codes = rng.integers(0, 2**32, (P, T, (H - k) // 8), dtype=np.uint64).astype(np.uint32)
+    side = _bf16_values(rng, P * k * T, 3.0).reshape(P, k, T)
+    keep = np.sort(rng.choice(H, k, replace=False)).astype(np.int32)
+    rest = np.setdiff1d(np.arange(H), keep).astype(np.int32)
+    return codes, side, keep, rest, scale.astype(np.float32), zero
+
+
+def pin_bf16_shards_exact_products(o):
+    """Power-of-two scales make every product (q - zero) * scale a bf16 value (at most 4
+    significant bits), so the literal reading must equal the standard one bit for bit, in both
+    output types, kept features included."""
+    rng = _rng(41)
+    P, T, H, k = 4, 6, 64, 16
+    scale = np.ldexp(1.0, rng.integers(-12, 6, (P, H)))
+    codes, side, keep, rest, scale, zero = _random_wire(rng, P, T, H, k, scale)
+    for f32 in (True, False):
+        lit = o.dequant_reduce(codes, side, H, keep, rest, scale, zero, out_f32=f32, bf16_shards=True)
+        std = o.dequant_reduce(codes, side, H, keep, rest, scale, zero, out_f32=f32)
+        assert np.array_equal(lit.view(np.uint32 if f32 else np.uint16), std.view(np.uint32 if f32 else np.uint16))
+
+
+def pin_bf16_shards_rounding_bound(o):
+    """One rank: the output is the shard's value rounded to bf16, so it is a bf16 number within
+    half a bf16 spacing of the fp32 product (bf16 has 8 significant bits: at most 2^-8 of the
+    value), and differs from the product wherever the product is not a bf16 number."""
+    rng = _rng(43)
+    P, T, H, k = 1, 40, 64, 8
+    scale = rng.uniform(0.01, 3.0, (P, H))
+    codes, side, keep, rest, scale, zero = _random_wire(rng, P, T, H, k, scale)
+    lit = o.dequant_reduce(codes, side, H, keep, rest, scale, zero, out_f32=True, bf16_shards=True)
+    nib = ((codes[..., None] >> (np.arange(8, dtype=np.uint32) * 4)) & 0xF).reshape(P, T, H - k)
+    v = ((nib.astype(np.float64) - zero[:, rest].astype(np.float64)[:, None, :])
+         * scale[:, rest].astype(np.float64)[:, None, :]).astype(np.float32)[0]   # fp32 products, [T][H-k]
+    got = lit[:, rest]
+    assert (got.view(np.uint32) & 0xFFFF == 0).all(), "a shard value that is not a bf16 number"
+    err = np.abs(got.astype(np.float64) - v.astype(np.float64))
+    assert (err <= np.ldexp(np.abs(v.astype(np.float64)), -8)).all(), "rounding error above half a bf16 spacing"
+    off_grid = (v.view(np.uint32) & 0xFFFF) != 0
+    assert off_grid.sum() > 100 and (err[off_grid] > 0).all(), "shards were not rounded"
+
+
 ALL_PINS = [
     pin_bf16_round, pin_quantize_golden, pin_quantize_nearest_grid, pin_params_golden,
     pin_params_closed_form, pin_calibrate_single_batch, pin_calibrate_ema, pin_select_golden,
     pin_select_brute_force, pin_pack_golden, pin_pack_unpack, pin_reduce_all_kept,
     pin_nan_outputs, pin_reduce_dequant_sum, pin_reduce_error_bound, pin_irwin_hall, pin_outliers_selected,
-    pin_selection_benefit,
+    pin_selection_benefit, pin_bf16_shards_golden, pin_bf16_shards_exact_products, pin_bf16_shards_rounding_bound,
 ]

@@ -40,11 +40,18 @@ MUTANTS = [
     ("side_row_major", "side[((size_t)r * k + j) * T + t] = row", "side[((size_t)r * T + t) * k + j] = row"),
     ("reduce_drops_last_rank", "for (int r = 0; r < P; ++r) {\n        uint32_t word",
      "for (int r = 0; r < P - 1; ++r) {\n        uint32_t word"),
-    ("dequant_sign_flipped", "(float)(q - (int)zero[p])", "(float)((int)zero[p] - q)"),
+    ("dequant_sign_flipped", "acc = fmaf((float)(q - (int)zero[p])", "acc = fmaf((float)((int)zero[p] - q)"),
     ("kept_sum_rank0_only", "for (int r = 0; r < P; ++r) acc = acc + ref_bf16_value(side",
      "for (int r = 0; r < 1; ++r) acc = acc + ref_bf16_value(side"),
     ("fp32_nan_payload_kept", "if (!isnan(f)) return f;", "return f;"),
     ("bf16_truncates", "if (dropped > 0x8000u || (dropped == 0x8000u && (keep & 1u))) keep += 1u;", ""),
+    ("bf16_shards_not_rounded", "acc = acc + ref_bf16_value(ref_bf16_round(v));", "acc = acc + v;"),
+    ("bf16_shards_truncated", "acc = acc + ref_bf16_value(ref_bf16_round(v));",
+     "uint32_t u; memcpy(&u, &v, sizeof u); acc = acc + ref_bf16_value((uint16_t)(u >> 16));"),
+    ("bf16_shards_rounds_the_sum", "acc = acc + ref_bf16_value(ref_bf16_round(v));",
+     "acc = ref_bf16_value(ref_bf16_round(acc + v));"),
+    ("bf16_shards_sign_flipped", "float v = (float)(q - (int)zero[p]) * scale[p];",
+     "float v = (float)((int)zero[p] - q) * scale[p];"),
     ("dequant_mul_then_add", "acc = fmaf((float)(q - (int)zero[p]), scale[p], acc);",
      "acc = acc + (float)(q - (int)zero[p]) * scale[p] * 1.0009765625f;"),
 ]
