@@ -32,10 +32,11 @@ _lib.hq_calibrate.argtypes = [_vp, _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp]
 _lib.hq_select_topk.argtypes = [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.hq_quantize_pack.argtypes = [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.hq_dequant_reduce.argtypes = [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _i32, _vp]
+_lib.hq_dequant_reduce_bf16_shards.argtypes = _lib.hq_dequant_reduce.argtypes
 _lib.hq_compress_reduce.argtypes = [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32,
                                     _vp, _vp, _vp]
 for _f in ("hq_calibrate", "hq_select_topk", "hq_quantize_pack", "hq_dequant_reduce",
-           "hq_compress_reduce", "hq_read_device_error"):
+           "hq_dequant_reduce_bf16_shards", "hq_compress_reduce", "hq_read_device_error"):
     getattr(_lib, _f).restype = _i32
 _lib.hq_read_device_error.argtypes = [_vp]
 _lib.hq_status_string.argtypes = [_i32]
@@ -49,7 +50,7 @@ HQ_OK, HQ_ERR_INVALID_ARG, HQ_ERR_MISALIGNED, HQ_ERR_CUDA, HQ_ERR_TIMEOUT, HQ_ER
 HQ_OUT_BF16, HQ_OUT_F32 = 0, 1
 
 EXPORTS = ["hq_calibrate", "hq_select_topk", "hq_quantize_pack", "hq_dequant_reduce",
-           "hq_compress_reduce", "hq_status_string", "hq_read_device_error", "hq_wire_bytes_per_row",
+           "hq_dequant_reduce_bf16_shards", "hq_compress_reduce", "hq_status_string", "hq_read_device_error", "hq_wire_bytes_per_row",
            "hq_selftest_bounded_wait"]
 
 
@@ -133,7 +134,7 @@ def hq_quantize_pack(x, keep_idx, rest_idx, inv_scale, zero, codes, side, stream
     _check(_lib.hq_quantize_pack(*args), "hq_quantize_pack")
 
 
-def hq_dequant_reduce(codes, side, keep_idx, rest_idx, scale, zero, out, stream=None) -> None:
+def _dequant_args(codes, side, keep_idx, rest_idx, scale, zero, out, stream):
     P, T, W = codes.shape
     k = keep_idx.shape[0]
     H = out.shape[1]
@@ -144,7 +145,18 @@ def hq_dequant_reduce(codes, side, keep_idx, rest_idx, scale, zero, out, stream=
             _ptr(keep_idx, _I32, (k,), "keep_idx"), _ptr(rest_idx, _I32, (H - k,), "rest_idx"),
             _ptr(scale, _F32, (P, H), "scale"), _ptr(zero, _U8, (P, H), "zero"),
             _ptr(out, _BF16 + _F32, (T, H), "out"), odt, _stream(stream, codes.device))
-    _check(_lib.hq_dequant_reduce(*args), "hq_dequant_reduce")
+    return args
+
+
+def hq_dequant_reduce(codes, side, keep_idx, rest_idx, scale, zero, out, stream=None) -> None:
+    _check(_lib.hq_dequant_reduce(*_dequant_args(codes, side, keep_idx, rest_idx, scale, zero, out, stream)),
+           "hq_dequant_reduce")
+
+
+def hq_dequant_reduce_bf16_shards(codes, side, keep_idx, rest_idx, scale, zero, out, stream=None) -> None:
+    """The literal variant: each rank's dequantized value is rounded to bf16 before it is added."""
+    _check(_lib.hq_dequant_reduce_bf16_shards(*_dequant_args(codes, side, keep_idx, rest_idx, scale, zero, out,
+                                                             stream)), "hq_dequant_reduce_bf16_shards")
 
 
 def hq_compress_reduce(x, keep_idx, rest_idx, scale, inv_scale, zero, out, codes=None, side=None,

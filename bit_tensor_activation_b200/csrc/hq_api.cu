@@ -107,7 +107,7 @@ void slice_chunks(int T, int S, long long resident, int rows_per_block, int* chu
   *chunks = (int)ceil_div(T, rpc);
 }
 
-template <typename OutT>
+template <typename OutT, bool kShard>
 hq_status launch_dequant(const uint32_t* codes, const uint16_t* side, int P, int T, int H, int k,
                          const int32_t* keep_idx, const float* scale, const uint8_t* zero, void* out,
                          cudaStream_t st, const DeviceInfo& d) {
@@ -125,7 +125,7 @@ hq_status launch_dequant(const uint32_t* codes, const uint16_t* side, int P, int
   if (!side_tma) map_side = map;  // never read
   if (tma) {
     const size_t smem = hq::dt_smem_bytes(P);
-    auto kern = hq::dequant_reduce_tma_kernel<OutT>;
+    auto kern = hq::dequant_reduce_tma_kernel<OutT, kShard>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
       return HQ_ERR_CUDA;
     int per_sm = 0;
@@ -141,7 +141,7 @@ hq_status launch_dequant(const uint32_t* codes, const uint16_t* side, int P, int
     return launched();
   }
   const size_t smem = hq::dq_smem_bytes(P);
-  auto kern = hq::dequant_reduce_kernel<OutT>;
+  auto kern = hq::dequant_reduce_kernel<OutT, kShard>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return HQ_ERR_CUDA;
   int per_sm = 0;
@@ -188,6 +188,29 @@ __global__ void selftest_wait_kernel(long long limit) {
   abort = 0;
   hq::fence_barrier_init();
   hq::mbar_wait(&bar, 0, &abort, limit);
+}
+
+// Argument checks and launch shared by the two reductions (kShard: each rank's value rounded to
+// bf16 before it is added).
+template <bool kShard>
+hq_status dequant_entry(const uint32_t* codes, const uint16_t* side, int P, int T, int H, int k,
+                        const int32_t* keep_idx, const int32_t* rest_idx, const float* scale,
+                        const uint8_t* zero, void* out, hq_out_dtype out_dtype, void* stream) {
+  if (check_shape(P, H, k) != HQ_OK || T < 0) return HQ_ERR_INVALID_ARG;
+  if (out_dtype != HQ_OUT_BF16 && out_dtype != HQ_OUT_F32) return HQ_ERR_INVALID_ARG;
+  if (!scale || !zero) return HQ_ERR_INVALID_ARG;
+  if ((k > 0 && !keep_idx) || (k < H && !rest_idx)) return HQ_ERR_INVALID_ARG;
+  if (T > 0 && (!out || (k > 0 && !side) || (k < H && !codes))) return HQ_ERR_INVALID_ARG;
+  if (!aligned(out, 16) || !aligned(side, 16) || !aligned(codes, 4) || !aligned(scale, 16) ||
+      !aligned(zero, 16) || !aligned(keep_idx, 4) || !aligned(rest_idx, 4))
+    return HQ_ERR_MISALIGNED;
+  if (T == 0) return HQ_OK;
+  DeviceInfo* d = nullptr;
+  if (device_info(&d) != HQ_OK) return HQ_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (out_dtype == HQ_OUT_BF16)
+    return launch_dequant<uint16_t, kShard>(codes, side, P, T, H, k, keep_idx, scale, zero, out, st, *d);
+  return launch_dequant<float, kShard>(codes, side, P, T, H, k, keep_idx, scale, zero, out, st, *d);
 }
 
 }  // namespace
@@ -270,21 +293,13 @@ hq_status hq_quantize_pack(const uint16_t* x, int P, int T, int H, int k, const 
 hq_status hq_dequant_reduce(const uint32_t* codes, const uint16_t* side, int P, int T, int H, int k,
                             const int32_t* keep_idx, const int32_t* rest_idx, const float* scale,
                             const uint8_t* zero, void* out, hq_out_dtype out_dtype, void* stream) {
-  if (check_shape(P, H, k) != HQ_OK || T < 0) return HQ_ERR_INVALID_ARG;
-  if (out_dtype != HQ_OUT_BF16 && out_dtype != HQ_OUT_F32) return HQ_ERR_INVALID_ARG;
-  if (!scale || !zero) return HQ_ERR_INVALID_ARG;
-  if ((k > 0 && !keep_idx) || (k < H && !rest_idx)) return HQ_ERR_INVALID_ARG;
-  if (T > 0 && (!out || (k > 0 && !side) || (k < H && !codes))) return HQ_ERR_INVALID_ARG;
-  if (!aligned(out, 16) || !aligned(side, 16) || !aligned(codes, 4) || !aligned(scale, 16) ||
-      !aligned(zero, 16) || !aligned(keep_idx, 4) || !aligned(rest_idx, 4))
-    return HQ_ERR_MISALIGNED;
-  if (T == 0) return HQ_OK;
-  DeviceInfo* d = nullptr;
-  if (device_info(&d) != HQ_OK) return HQ_ERR_CUDA;
-  cudaStream_t st = (cudaStream_t)stream;
-  if (out_dtype == HQ_OUT_BF16)
-    return launch_dequant<uint16_t>(codes, side, P, T, H, k, keep_idx, scale, zero, out, st, *d);
-  return launch_dequant<float>(codes, side, P, T, H, k, keep_idx, scale, zero, out, st, *d);
+  return dequant_entry<false>(codes, side, P, T, H, k, keep_idx, rest_idx, scale, zero, out, out_dtype, stream);
+}
+
+hq_status hq_dequant_reduce_bf16_shards(const uint32_t* codes, const uint16_t* side, int P, int T, int H, int k,
+                                        const int32_t* keep_idx, const int32_t* rest_idx, const float* scale,
+                                        const uint8_t* zero, void* out, hq_out_dtype out_dtype, void* stream) {
+  return dequant_entry<true>(codes, side, P, T, H, k, keep_idx, rest_idx, scale, zero, out, out_dtype, stream);
 }
 
 hq_status hq_compress_reduce(const uint16_t* x, int P, int T, int H, int k, const int32_t* keep_idx,

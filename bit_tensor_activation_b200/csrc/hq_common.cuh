@@ -43,6 +43,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return r;
 }
 
+// Two floats rounded to bf16 (nearest, ties to even) in one register: a in the low half, b in
+// the high half.  A NaN stays a NaN (its payload is not canonicalised).
+__device__ __forceinline__ uint32_t round_bf16x2(float a, float b) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+  return r;
+}
+
 // Streaming 16-byte load: read once, do not keep in L1.
 __device__ __forceinline__ uint4 ld_stream16(const void* p) {
   uint4 v;

@@ -174,8 +174,10 @@ __device__ __forceinline__ void dq_fill_constants(float4* s_const, const int32_t
   }
 }
 
-// Adds one rank's contribution for R staged rows (row m at st + m * stride words).
-template <bool kFast, int R>
+// Adds one rank's contribution for R staged rows (row m at st + m * stride words).  kShard: the
+// literal reading of the reduction, in which the rank's dequantized value (q - zero) * scale is
+// first rounded to bf16 and then added (the default adds the exact product with one FMA).
+template <bool kFast, int R, bool kShard>
 __device__ __forceinline__ void dq_decode_rows(const DqLane& D, const uint32_t* __restrict__ st, int stride,
                                                const float4* __restrict__ cst, float (&acc)[R][8]) {
   const float4 s0 = cst[0], s1 = cst[32], o0 = cst[64], o1 = cst[96];
@@ -204,7 +206,17 @@ __device__ __forceinline__ void dq_decode_rows(const DqLane& D, const uint32_t* 
 #pragma unroll
     for (int i = 0; i < 8; i += 2) {
       const float d0 = __fadd_rn(q[i], off[i]), d1 = __fadd_rn(q[i + 1], off[i + 1]);
-      ffma2_acc(acc[m][i], acc[m][i + 1], d0, d1, sc[i], sc[i + 1]);
+      if (kShard) {
+        // (q - zero)*16^p times scale/16^p: the exact (q - zero)*scale, rounded once to fp32,
+        // then to bf16
+        float v0, v1;
+        fmul2(v0, v1, d0, d1, sc[i], sc[i + 1]);
+        const uint32_t b = round_bf16x2(v0, v1);
+        acc[m][i] = __fadd_rn(acc[m][i], __uint_as_float(b << 16));
+        acc[m][i + 1] = __fadd_rn(acc[m][i + 1], __uint_as_float(b & 0xFFFF0000u));
+      } else {
+        ffma2_acc(acc[m][i], acc[m][i + 1], d0, d1, sc[i], sc[i + 1]);
+      }
     }
   }
 }
@@ -241,31 +253,55 @@ __device__ __forceinline__ void dq_store_rows(const DqLane& D, const float (&acc
   }
 }
 
-// Kept features of the warp's slice for rows t0..t0+R-1, read from global memory:
-// (row, kept feature) pairs over the lanes sum the P side values in rank order; owners copy them
-// into their sums; then the rows are stored.  Warp-level only (uses `kept`, R x 32 floats of
-// shared memory per warp).
-template <typename OutT, int R>
+// Kept features of the warp's slice for rows t0..t0+R-1, read from global memory: each kept
+// feature's R side values summed over the P ranks in rank order; owners copy them into their
+// sums; then the rows are stored.  When the R rows are whole and 8-byte aligned (R == 4,
+// T % 4 == 0) lane l takes kept feature kc + l and reads its 4 rows with one 8-byte load per
+// rank (kVec; the TMA kernel, whose register budget is tighter and which stages the side values of
+// all but crowded slices, leaves it out); otherwise the lanes take (row, kept feature) pairs,
+// 4 rows of 8 features per warp load.  Warp-level only (uses `kept`, R x 32 floats of shared
+// memory per warp).
+template <typename OutT, int R, bool kVec>
 __device__ __forceinline__ void dq_finish_block(const DqLane& D, float (&acc)[R][8],
                                                 const uint16_t* __restrict__ side, float* kept, int P,
                                                 int T, int H, int k, int ja, int jb, int t0, int t_last,
                                                 OutT* __restrict__ out) {
   const int lane = threadIdx.x & 31;
   const int nk = jb - ja;
+  const size_t rank_stride = (size_t)k * T;
+  const bool vec = kVec && R == 4 && (T & 3) == 0 && t0 + R <= t_last;
   for (int kc = 0; kc < nk; kc += 32) {
     const int kw = min(32, nk - kc);
-    for (int p = lane; p < R * kw; p += 32) {
-      const int m = p / kw, jj = p - m * kw;
-      const int t = t0 + m;
-      float a = 0.0f;
-      if (t < t_last) {
-        const uint16_t* sp = side + (size_t)(ja + kc + jj) * T + t;  // side[r][j][t], feature-major
-        const size_t rank_stride = (size_t)k * T;
-#pragma unroll 8
-        for (int r = 0; r < P; ++r)
-          a = __fadd_rn(a, __uint_as_float((uint32_t)__ldg(sp + r * rank_stride) << 16));
+    if (vec) {
+      if (lane < kw) {
+        const uint16_t* sp = side + (size_t)(ja + kc + lane) * T + t0;  // side[r][j][t], feature-major
+        float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
+#pragma unroll 4
+        for (int r = 0; r < P; ++r) {
+          const uint2 w = __ldg(reinterpret_cast<const uint2*>(sp + r * rank_stride));
+          a0 = __fadd_rn(a0, __uint_as_float(w.x << 16));
+          a1 = __fadd_rn(a1, __uint_as_float(w.x & 0xFFFF0000u));
+          a2 = __fadd_rn(a2, __uint_as_float(w.y << 16));
+          a3 = __fadd_rn(a3, __uint_as_float(w.y & 0xFFFF0000u));
+        }
+        kept[0 * 32 + lane] = a0;
+        kept[1 * 32 + lane] = a1;
+        kept[2 * 32 + lane] = a2;
+        kept[3 * 32 + lane] = a3;
       }
-      kept[m * 32 + jj] = a;
+    } else {
+      for (int p = lane; p < R * kw; p += 32) {
+        const int jj = p / R, m = p - jj * R;
+        const int t = t0 + m;
+        float a = 0.0f;
+        if (t < t_last) {
+          const uint16_t* sp = side + (size_t)(ja + kc + jj) * T + t;
+#pragma unroll 8
+          for (int r = 0; r < P; ++r)
+            a = __fadd_rn(a, __uint_as_float((uint32_t)__ldg(sp + r * rank_stride) << 16));
+        }
+        kept[m * 32 + jj] = a;
+      }
     }
     __syncwarp();
     dq_patch_kept<R>(D, acc, kept, ja, kc, kw);
@@ -340,13 +376,13 @@ inline size_t dt_smem_bytes(int P) { return sizeof(DtSmem) + 128 + (size_t)P * 4
 
 // The nr ranks of one ring slot, in rank order: 4-bit features of the warp's rows into acc
 // (cst = this lane's constants of the slot's first rank).
-template <bool kFast>
+template <bool kFast, bool kShard>
 __device__ __forceinline__ void dt_slot(const DqLane& D, const DtSmem& sm, int st_i, int warp, int nr,
                                         const float4* __restrict__ cst, float (&acc)[kDtR][8]) {
 #pragma unroll
   for (int j = 0; j < kDtG; ++j)
     if (j < nr && D.decode)
-      dq_decode_rows<kFast, kDtR>(D, &sm.tile[st_i][j][warp * kDtR][0], kDtWords, cst + j * 4 * 32, acc);
+      dq_decode_rows<kFast, kDtR, kShard>(D, &sm.tile[st_i][j][warp * kDtR][0], kDtWords, cst + j * 4 * 32, acc);
 }
 
 // The kept-sum warp, for slices whose side values are staged: lane l sums rows 4(l % 8) ..
@@ -429,7 +465,7 @@ __device__ __forceinline__ void dt_patch_kept(const DqLane& D, float (&acc)[kDtR
   }
 }
 
-template <typename OutT>
+template <typename OutT, bool kShard>
 __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_kernel(
     const __grid_constant__ CUtensorMap tmap_codes, const __grid_constant__ CUtensorMap tmap_side, int side_tma,
     const uint16_t* __restrict__ side, int P, int T, int H,
@@ -550,8 +586,8 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
       }
       const int nr = min(kDtG, P - g * kDtG);
       const float4* cst = s_const + (size_t)g * kDtG * 4 * 32 + lane;
-      if (generic) dt_slot<false>(D, sm, st_i, warp, nr, cst, acc);
-      else dt_slot<true>(D, sm, st_i, warp, nr, cst, acc);
+      if (generic) dt_slot<false, kShard>(D, sm, st_i, warp, nr, cst, acc);
+      else dt_slot<true, kShard>(D, sm, st_i, warp, nr, cst, acc);
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.ring.empty[st_i]);
       if (++st_i == kDtStages) {
@@ -568,7 +604,7 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
       if (lane == 0) mbar_arrive(&sm.ksum_empty[buf]);
       dq_store_rows<OutT, kDtR>(D, acc, H, t0, t_last, out);
     } else {
-      dq_finish_block<OutT, kDtR>(D, acc, side, sm.k.kept[warp], P, T, H, k, q.ja, q.jb, t0, t_last, out);
+      dq_finish_block<OutT, kDtR, false>(D, acc, side, sm.k.kept[warp], P, T, H, k, q.ja, q.jb, t0, t_last, out);
     }
   }
 }
@@ -586,7 +622,7 @@ inline size_t dq_smem_bytes(int P) {
          + (size_t)kDqWarps * kDqR * 32 * 4;                // kept sums
 }
 
-template <typename OutT>
+template <typename OutT, bool kShard>
 __global__ void __launch_bounds__(kDqThreads) dequant_reduce_kernel(
     const uint32_t* __restrict__ codes, const uint16_t* __restrict__ side, int P, int T, int H,
     int k, const int32_t* __restrict__ keep_idx, const float* __restrict__ scale,
@@ -655,12 +691,12 @@ __global__ void __launch_bounds__(kDqThreads) dequant_reduce_kernel(
       const uint32_t* st = my_tiles + (size_t)(tile % kDqD) * kDqR * kDqWin;
       const float4* cst = s_const + (size_t)r * 4 * 32 + lane;
       if (D.decode) {
-        if (generic) dq_decode_rows<false, kDqR>(D, st, kDqWin, cst, acc);
-        else dq_decode_rows<true, kDqR>(D, st, kDqWin, cst, acc);
+        if (generic) dq_decode_rows<false, kDqR, kShard>(D, st, kDqWin, cst, acc);
+        else dq_decode_rows<true, kDqR, kShard>(D, st, kDqWin, cst, acc);
       }
       __syncwarp();  // the stage is free for the copy issued next iteration
     }
-    dq_finish_block<OutT, kDqR>(D, acc, side, my_kept, P, T, H, k, q.ja, q.jb, t0, t_last, out);
+    dq_finish_block<OutT, kDqR, true>(D, acc, side, my_kept, P, T, H, k, q.ja, q.jb, t0, t_last, out);
   }
   cp_async_wait<0>();
 }

@@ -124,6 +124,22 @@ hq_status hq_dequant_reduce(const uint32_t* codes, const uint16_t* side, int P, 
                             const uint8_t* zero, void* out, hq_out_dtype out_dtype, void* stream);
 
 /*
+ * Dequant-reduce, literal reading of bullet "Inference" (R19): after communication each rank's
+ * tensor is first made BF16 and the ranks' BF16 tensors are then combined.  Same arguments,
+ * layouts, ownership and errors as hq_dequant_reduce; only non-kept features differ:
+ *   non-kept feature h = rest_idx[c]:  acc = +0;  for r = 0..P-1:
+ *       v = float(q_r - zero[r][h]) * scale[r][h]            (one fp32 product)
+ *       acc = acc + bf16(v)          (v rounded to bf16, nearest-even, then added in fp32)
+ * Kept features and the output are as in hq_dequant_reduce.  Used to measure what the extra
+ * per-rank rounding costs in accuracy (the selection ablation); the default reading keeps each
+ * rank's exact product.
+ */
+hq_status hq_dequant_reduce_bf16_shards(const uint32_t* codes, const uint16_t* side, int P, int T, int H,
+                                        int k, const int32_t* keep_idx, const int32_t* rest_idx,
+                                        const float* scale, const uint8_t* zero, void* out,
+                                        hq_out_dtype out_dtype, void* stream);
+
+/*
  * Fused compress-reduce (section "Combating Quantization Errors with Tensor Parallelism": the
  * partial sums are quantized and then summed): out equals hq_quantize_pack followed by
  * hq_dequant_reduce, bit for bit (R12), computed from x in one pass without a wire buffer.

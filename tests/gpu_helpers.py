@@ -67,10 +67,11 @@ def gpu_quantize(x, prm):
     return codes, side
 
 
-def gpu_dequant(codes, side, prm, H, out_f32=False):
+def gpu_dequant(codes, side, prm, H, out_f32=False, bf16_shards=False):
     T = codes.shape[1]
     out = torch.empty((T, H), dtype=torch.float32 if out_f32 else torch.int16, device=DEV)
-    hq.hq_dequant_reduce(codes, side, prm["keep_idx"], prm["rest_idx"], prm["scale"], prm["zero"], out)
+    fn = hq.hq_dequant_reduce_bf16_shards if bf16_shards else hq.hq_dequant_reduce
+    fn(codes, side, prm["keep_idx"], prm["rest_idx"], prm["scale"], prm["zero"], out)
     return out
 
 
@@ -112,7 +113,12 @@ def oracle_pipeline(cfg: synth.Config, cal, x):
     out_b = o.dequant_reduce(codes, side, cfg.H, sel["keep_idx"], sel["rest_idx"], sel["scale"], sel["zero"])
     out_f = o.dequant_reduce(codes, side, cfg.H, sel["keep_idx"], sel["rest_idx"], sel["scale"], sel["zero"],
                              out_f32=True)
-    return dict(emin=emin, emax=emax, sel=sel, codes=codes, side=side, out_b=out_b, out_f=out_f)
+    lit_b = o.dequant_reduce(codes, side, cfg.H, sel["keep_idx"], sel["rest_idx"], sel["scale"], sel["zero"],
+                             bf16_shards=True)
+    lit_f = o.dequant_reduce(codes, side, cfg.H, sel["keep_idx"], sel["rest_idx"], sel["scale"], sel["zero"],
+                             out_f32=True, bf16_shards=True)
+    return dict(emin=emin, emax=emax, sel=sel, codes=codes, side=side, out_b=out_b, out_f=out_f,
+                lit_b=lit_b, lit_f=lit_f)
 
 
 def compare_all(cfg, cal, x_np):
@@ -124,6 +130,8 @@ def compare_all(cfg, cal, x_np):
     codes, side = gpu_quantize(x, B)
     out_b = gpu_dequant(codes, side, B, cfg.H)
     out_f = gpu_dequant(codes, side, B, cfg.H, out_f32=True)
+    lit_b = gpu_dequant(codes, side, B, cfg.H, bf16_shards=True)
+    lit_f = gpu_dequant(codes, side, B, cfg.H, out_f32=True, bf16_shards=True)
     fb, _, _ = gpu_fused(x, B)
     ff, wc, ws = gpu_fused(x, B, out_f32=True, wire=True)
     assert_no_device_error()
@@ -138,6 +146,8 @@ def compare_all(cfg, cal, x_np):
     assert_same(u16(side), ref["side"], "side")
     assert_same(u16(out_b), ref["out_b"], "out bf16")
     assert_same(f32bits(out_f), f32bits(ref["out_f"]), "out f32")
+    assert_same(u16(lit_b), ref["lit_b"], "bf16-shard reduction, bf16 out")
+    assert_same(f32bits(lit_f), f32bits(ref["lit_f"]), "bf16-shard reduction, f32 out")
     assert_same(u16(fb), ref["out_b"], "fused bf16")
     assert_same(f32bits(ff), f32bits(ref["out_f"]), "fused f32")
     assert_same(u32(wc), ref["codes"], "fused wire codes")

@@ -61,6 +61,8 @@ def _calls(lib):
             c(x), P, T, H, k, c(keep), c(rest), c(A), c(A), c(codes), c(side), None),
         "dequant": lambda P=2, T=4, H=64, k=8, out=A, odt=0, side=A: lib.hq_dequant_reduce(
             c(A), c(side), P, T, H, k, c(A), c(A), c(A), c(A), c(out), odt, None),
+        "dequant_bf16_shards": lambda P=2, T=4, H=64, k=8, out=A, odt=0, side=A: lib.hq_dequant_reduce_bf16_shards(
+            c(A), c(side), P, T, H, k, c(A), c(A), c(A), c(A), c(out), odt, None),
         "fused": lambda P=2, T=4, H=64, k=8, out=A, codes=None, side=None: lib.hq_compress_reduce(
             c(A), P, T, H, k, c(A), c(A), c(A), c(A), c(A), c(out), 0, c(codes) if codes else None,
             c(side) if side else None, None),
@@ -81,6 +83,9 @@ def _calls(lib):
     ("quantize", dict(codes=A + 2), 2),
     ("dequant", dict(odt=2), 1), ("dequant", dict(out=0), 1), ("dequant", dict(out=MIS), 2),
     ("dequant", dict(side=0), 1),
+    ("dequant_bf16_shards", dict(odt=2), 1), ("dequant_bf16_shards", dict(out=0), 1),
+    ("dequant_bf16_shards", dict(out=MIS), 2), ("dequant_bf16_shards", dict(side=0), 1),
+    ("dequant_bf16_shards", dict(k=12), 1),
     ("fused", dict(codes=A), 1), ("fused", dict(side=A), 1), ("fused", dict(out=MIS), 2),
     ("fused", dict(P=70), 1),
 ])
@@ -96,6 +101,7 @@ def test_empty_arrays_may_be_null(hq):
     assert lib.hq_quantize_pack(c(A), 2, 0, 64, 0, None, c(A), c(A), c(A), c(A), None, None) == 0
     assert lib.hq_quantize_pack(c(A), 2, 0, 64, 64, c(A), None, c(A), c(A), None, c(A), None) == 0
     assert lib.hq_dequant_reduce(None, c(A), 2, 0, 64, 64, c(A), None, c(A), c(A), c(A), 0, None) == 0
+    assert lib.hq_dequant_reduce_bf16_shards(None, c(A), 2, 0, 64, 64, c(A), None, c(A), c(A), c(A), 0, None) == 0
     assert lib.hq_compress_reduce(c(A), 2, 0, 64, 0, None, c(A), c(A), c(A), c(A), c(A), 1, None, None, None) == 0
 
 

@@ -73,6 +73,8 @@ def test_outputs_stay_in_bounds(cfg):
     out_f = g("out_f32", (T, H), torch.float32)
     hq.hq_dequant_reduce(codes, side, keep, rest, scale, zero, out_b)
     hq.hq_dequant_reduce(codes, side, keep, rest, scale, zero, out_f)
+    lit_b = g("bf16_shards_bf16", (T, H), torch.int16)
+    hq.hq_dequant_reduce_bf16_shards(codes, side, keep, rest, scale, zero, lit_b)
     fused = g("fused", (T, H), torch.int16)
     wcodes = g("wire_codes", (P, T, (H - k) // 8), torch.int32)
     wside = g("wire_side", (P, k, T), torch.int16)
@@ -87,6 +89,7 @@ def test_outputs_stay_in_bounds(cfg):
     assert_same(u16(side), ref["side"], "side")
     assert_same(u16(out_b), ref["out_b"], "out bf16")
     assert_same(f32bits(out_f), f32bits(ref["out_f"]), "out f32")
+    assert_same(u16(lit_b), ref["lit_b"], "bf16-shard reduction")
     assert_same(u16(fused), ref["out_b"], "fused")
     assert_same(u32(wcodes), ref["codes"], "wire codes")
     assert_same(u16(wside), ref["side"], "wire side")

@@ -120,14 +120,18 @@ def test_kept_counts_per_slice_bit_exact(P, T):
     out_r = o.dequant_reduce(codes_r, side_r, H, sel["keep_idx"], sel["rest_idx"], sel["scale"], sel["zero"])
     out_rf = o.dequant_reduce(codes_r, side_r, H, sel["keep_idx"], sel["rest_idx"], sel["scale"], sel["zero"],
                               out_f32=True)
+    lit_r = o.dequant_reduce(codes_r, side_r, H, sel["keep_idx"], sel["rest_idx"], sel["scale"], sel["zero"],
+                             bf16_shards=True)
     codes, side = gpu_quantize(to_dev_u16(x), prm)
     out = gpu_dequant(codes, side, prm, H)
     out_f = gpu_dequant(codes, side, prm, H, out_f32=True)
+    lit = gpu_dequant(codes, side, prm, H, bf16_shards=True)
     assert_no_device_error()
     assert_same(u32(codes), codes_r, "codes")
     assert_same(u16(side), side_r, "side")
     assert_same(u16(out), out_r, "out bf16")
     assert_same(f32bits(out_f), f32bits(out_rf), "out f32")
+    assert_same(u16(lit), lit_r, "bf16-shard reduction")
 
 
 def test_select_ties_and_special_values():
@@ -302,19 +306,23 @@ def test_full_size_select_quantize_reduce_sampled(name):
     x = _gpu_batch(cfg, synth.EVAL, 0, torch.from_numpy(cs).to(DEV))
     codes, side = gpu_quantize(x, prm)
     out = gpu_dequant(codes, side, prm, cfg.H)
+    lit = gpu_dequant(codes, side, prm, cfg.H, bf16_shards=True)
     fused, _, _ = gpu_fused(x, prm)
     assert_no_device_error()
     assert torch.equal(out, fused), "fused == split over the whole output"
     rng = np.random.default_rng(23)
     rows = np.unique(np.concatenate([[0, cfg.T - 1], rng.integers(0, cfg.T, 10)]))
-    codes_h, side_h, out_h = u32(codes), u16(side), u16(out)
+    codes_h, side_h, out_h, lit_h = u32(codes), u16(side), u16(out), u16(lit)
     for t in rows:
         xr = synth.fill_cpu(cfg, synth.EVAL, 0, rows=(int(t), int(t) + 1), cs=cs)
         c_r, s_r = o.quantize_pack(xr, sel["keep_idx"], sel["rest_idx"], sel["inv_scale"], sel["zero"])
         o_r = o.dequant_reduce(c_r, s_r, cfg.H, sel["keep_idx"], sel["rest_idx"], sel["scale"], sel["zero"])
+        l_r = o.dequant_reduce(c_r, s_r, cfg.H, sel["keep_idx"], sel["rest_idx"], sel["scale"], sel["zero"],
+                               bf16_shards=True)
         assert np.array_equal(codes_h[:, t:t + 1], c_r), f"codes row {t}"
         assert np.array_equal(side_h[:, :, t:t + 1], s_r), f"side row {t}"
         assert np.array_equal(out_h[t:t + 1], o_r), f"out row {t}"
+        assert np.array_equal(lit_h[t:t + 1], l_r), f"bf16-shard reduction row {t}"
 
 
 # ---------------------------------------------------------------------------------------------
