@@ -22,6 +22,7 @@
 namespace {
 
 constexpr int kMaxRanks = 64;
+static_assert(kMaxRanks <= hq::kSelMaxRanks, "the parameter kernel stages one range per rank");
 constexpr int kMaxDevices = 64;
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -252,7 +253,7 @@ hq_status hq_select_topk(const float* ema_min, const float* ema_max, int P, int 
     }
   }
   // parameters and keys over the whole GPU, then the selection in one CTA (same stream)
-  const unsigned pgrid = (unsigned)ceil_div(H, hq::kSelParamThreads);
+  const unsigned pgrid = (unsigned)ceil_div(H, hq::kSelParamFeatures);
   hq::select_params_kernel<<<pgrid, hq::kSelParamThreads, 0, (cudaStream_t)stream>>>(
       ema_min, ema_max, P, H, k, keep_idx, rest_idx, scale, inv_scale, zero);
   if (cudaGetLastError() != cudaSuccess) return HQ_ERR_CUDA;

@@ -3,12 +3,13 @@
 // "Selection of High Precision Features"), with the 4-bit grid of bullet "Calibration".
 //
 // Two kernels, no memory beyond the inputs and outputs:
-//   1. select_params_kernel, one thread per feature over the whole GPU: for each rank in order,
-//      lo = min(ema_min,0), hi = max(ema_max,0), scale = (hi-lo)/15, inv_scale = 1/scale,
-//      zero = clamp(rint(-lo*inv_scale),0,15) (degenerate scale -> 1, 0), and the feature's score
-//      = sum over ranks of (hi-lo) in rank order.  The score's fp32 bits (non-negative, so their
-//      unsigned order is the numeric order; NaN ranks as +inf) are parked in the index outputs:
-//      slot h of the H slots rest_idx[0..H-k) followed by keep_idx[0..k).
+//   1. select_params_kernel, one thread per (feature, rank) over the whole GPU (a CTA takes 32
+//      features): lo = min(ema_min,0), hi = max(ema_max,0), scale = (hi-lo)/15,
+//      inv_scale = 1/scale, zero = clamp(rint(-lo*inv_scale),0,15) (degenerate scale -> 1, 0);
+//      the ranges go to shared memory, and one thread per feature sums them in rank order into
+//      the feature's score.  The score's fp32 bits (non-negative, so their unsigned order is the
+//      numeric order; NaN ranks as +inf) are parked in the index outputs: slot h of the H slots
+//      rest_idx[0..H-k) followed by keep_idx[0..k).
 //   2. select_topk_kernel, one CTA of 1024 threads: reads the H keys into shared memory, then a
 //      radix select, 8 bits per pass from the top, finds the k-th largest key tau and how many
 //      features equal to tau are still to be taken, and a block-wide ordered scan takes every
@@ -55,19 +56,25 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int& tot
 }
 
 constexpr int kSelParamThreads = 256;
+constexpr int kSelParamFeatures = 32;                                    // features per CTA
+constexpr int kSelParamRankSlots = kSelParamThreads / kSelParamFeatures;  // ranks handled at once
+constexpr int kSelMaxRanks = 64;
 
 __global__ void __launch_bounds__(kSelParamThreads) select_params_kernel(
     const float* __restrict__ ema_min, const float* __restrict__ ema_max, int P, int H, int k,
     int32_t* __restrict__ keep_idx, int32_t* __restrict__ rest_idx, float* __restrict__ scale,
     float* __restrict__ inv_scale, uint8_t* __restrict__ zero) {
-  for (int h = blockIdx.x * blockDim.x + threadIdx.x; h < H; h += gridDim.x * blockDim.x) {
-    float score = 0.0f;
-    for (int r = 0; r < P; ++r) {
+  __shared__ float s_range[kSelMaxRanks][kSelParamFeatures];
+  const int f = threadIdx.x % kSelParamFeatures;
+  const int h = blockIdx.x * kSelParamFeatures + f;
+  for (int r = threadIdx.x / kSelParamFeatures; r < P; r += kSelParamRankSlots) {
+    float range = 0.0f;
+    if (h < H) {
       const size_t i = (size_t)r * H + h;
       const float emin = ema_min[i], emax = ema_max[i];
       const float lo = (emin < 0.0f) ? emin : 0.0f;
       const float hi = (emax > 0.0f) ? emax : 0.0f;
-      const float range = __fsub_rn(hi, lo);
+      range = __fsub_rn(hi, lo);
       float s = __fdiv_rn(range, 15.0f);
       float inv = 1.0f;
       float zf = 0.0f;
@@ -81,8 +88,13 @@ __global__ void __launch_bounds__(kSelParamThreads) select_params_kernel(
       scale[i] = s;
       inv_scale[i] = inv;
       zero[i] = (uint8_t)(int)zf;
-      score = __fadd_rn(score, range);
     }
+    s_range[r][f] = range;
+  }
+  __syncthreads();
+  if (threadIdx.x < kSelParamFeatures && h < H) {
+    float score = 0.0f;
+    for (int r = 0; r < P; ++r) score = __fadd_rn(score, s_range[r][f]);
     const uint32_t key = (score != score) ? 0x7F800000u : __float_as_uint(score);
     if (h < H - k) rest_idx[h] = (int32_t)key;
     else keep_idx[h - (H - k)] = (int32_t)key;
