@@ -380,3 +380,33 @@ def test_sweep_point_sampled(cfg):
         assert_same(codes_h[:, i:i + 1], c_r, f"codes row {t}")
         assert_same(side_h[:, :, i:i + 1], s_r, f"side row {t}")
         assert_same(out_h[i:i + 1], o_r, f"out row {t}")
+
+
+def test_per_rank_calls_equal_the_batched_call():
+    """A real rank calls quantize-pack with P = 1 on its own partial sum and its own parameter
+    row; stacking those wire buffers gives the batched (P > 1) call's buffers bit for bit, and
+    reducing them gives the batched output."""
+    cfg = synth.CONFIGS["prefill7b"].with_(name="per_rank", P=5, T=72, H=2048, k=64, n_out=16, calib_batches=2,
+                                           calib_T=40)
+    cs, _ = synth.colscale(cfg)
+    cal = _batches(cfg, cs)
+    x_np = synth.fill_cpu(cfg, synth.EVAL, 0, cs=cs)
+    emin, emax = gpu_calibrate_batches(cal, cfg.beta, cfg.P, cfg.H)
+    B = gpu_select(emin, emax, cfg.k)
+    x = to_dev_u16(x_np)
+    codes, side = gpu_quantize(x, B)
+    out = gpu_dequant(codes, side, B, cfg.H)
+    per_codes, per_side = [], []
+    for r in range(cfg.P):
+        row = {n: (B[n][r:r + 1].contiguous() if n in ("scale", "inv_scale", "zero") else B[n]) for n in B}
+        # calibration of one rank alone gives that rank's row of the batched statistics
+        e1, e2 = gpu_calibrate_batches([c[r:r + 1] for c in cal], cfg.beta, 1, cfg.H)
+        assert torch.equal(e1, emin[r:r + 1]) and torch.equal(e2, emax[r:r + 1])
+        c_r, s_r = gpu_quantize(x[r:r + 1].contiguous(), row)
+        per_codes.append(c_r)
+        per_side.append(s_r)
+    assert_no_device_error()
+    assert torch.equal(torch.cat(per_codes), codes)
+    assert torch.equal(torch.cat(per_side), side)
+    out2 = gpu_dequant(torch.cat(per_codes), torch.cat(per_side), B, cfg.H)
+    assert torch.equal(out2, out)
