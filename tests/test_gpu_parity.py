@@ -101,7 +101,7 @@ def test_clustered_kept_features_bit_exact(P, T, H, k, big):
 SLICE_KEPT = [0, 1, 3, 4, 5, 7, 8, 9, 15, 16, 17, 24, 31, 32, 33, 19]
 
 
-@pytest.mark.parametrize("P,T", [(5, 72), (8, 72), (2, 2048), (4, 4096)])
+@pytest.mark.parametrize("P,T", [(5, 72), (8, 72), (2, 2048), (4, 4096), (16, 64), (64, 8)])
 def test_kept_counts_per_slice_bit_exact(P, T):
     o = oracle.get()
     H = 4096
