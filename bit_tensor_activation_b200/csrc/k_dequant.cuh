@@ -375,13 +375,15 @@ struct DtSmem {
 inline size_t dt_smem_bytes(int P) { return sizeof(DtSmem) + 128 + (size_t)P * 4 * 32 * 16; }
 
 // The nr ranks of one ring slot, in rank order: 4-bit features of the warp's rows into acc
-// (cst = this lane's constants of the slot's first rank).
-template <bool kFast, bool kShard>
+// (cst = this lane's constants of the slot's first rank).  kFull: the slot holds kDtG ranks, so
+// the rank loop carries no per-rank test (worth 5% of the kernel's time).
+template <bool kFast, bool kShard, bool kFull>
 __device__ __forceinline__ void dt_slot(const DqLane& D, const DtSmem& sm, int st_i, int warp, int nr,
                                         const float4* __restrict__ cst, float (&acc)[kDtR][8]) {
+  if (!D.decode) return;
 #pragma unroll
   for (int j = 0; j < kDtG; ++j)
-    if (j < nr && D.decode)
+    if (kFull || j < nr)
       dq_decode_rows<kFast, kDtR, kShard>(D, &sm.tile[st_i][j][warp * kDtR][0], kDtWords, cst + j * 4 * 32, acc);
 }
 
@@ -586,8 +588,9 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
       }
       const int nr = min(kDtG, P - g * kDtG);
       const float4* cst = s_const + (size_t)g * kDtG * 4 * 32 + lane;
-      if (generic) dt_slot<false, kShard>(D, sm, st_i, warp, nr, cst, acc);
-      else dt_slot<true, kShard>(D, sm, st_i, warp, nr, cst, acc);
+      if (generic) dt_slot<false, kShard, false>(D, sm, st_i, warp, nr, cst, acc);
+      else if (nr == kDtG) dt_slot<true, kShard, true>(D, sm, st_i, warp, nr, cst, acc);
+      else dt_slot<true, kShard, false>(D, sm, st_i, warp, nr, cst, acc);
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.ring.empty[st_i]);
       if (++st_i == kDtStages) {

@@ -124,7 +124,8 @@ __global__ void __launch_bounds__(kFuThreads, 2) compress_reduce_kernel(
   const int h0 = hs + 8 * lane;
   const bool active = h0 < H;
   const uint32_t kmask = __float_as_uint(s_const[128 + lane].z);
-  int i = 0;
+  int st_i = 0;  // ring stage of the next tile and the parity of its fill
+  unsigned phase = 0;
   for (int bi = 0; bi < nblk && !*abort; ++bi) {
     const int t0 = t_first + bi * kFuTileRows + warp * kFuR;
     float acc[kFuR][8];
@@ -133,8 +134,8 @@ __global__ void __launch_bounds__(kFuThreads, 2) compress_reduce_kernel(
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[m][e] = 0.0f;
     bool ok = true;
-    for (int r = 0; r < P; ++r, ++i) {
-      if (!sm.ring.wait_full(i, abort, wait_limit)) {
+    for (int r = 0; r < P; ++r) {
+      if (!mbar_wait(&sm.ring.full[st_i], phase, abort, wait_limit)) {
         ok = false;
         break;
       }
@@ -144,12 +145,15 @@ __global__ void __launch_bounds__(kFuThreads, 2) compress_reduce_kernel(
         const float inv[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
         const float sc[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
         const uint32_t zlo = __float_as_uint(zz.x), zhi = __float_as_uint(zz.y);
-        int lo[8];
+        int lo[8], hi[8];  // clamp bounds of c: -zero and 15 - zero
 #pragma unroll
-        for (int e = 0; e < 8; ++e) lo[e] = -(int)(((e < 4 ? zlo : zhi) >> (8 * (e & 3))) & 0xFFu);
+        for (int e = 0; e < 8; ++e) {
+          lo[e] = -(int)(((e < 4 ? zlo : zhi) >> (8 * (e & 3))) & 0xFFu);
+          hi[e] = lo[e] + 15;
+        }
 #pragma unroll
         for (int m = 0; m < kFuR; ++m) {
-          const uint4 xv = reinterpret_cast<const uint4*>(&sm.tile[i % kFuStages][warp * kFuR + m][0])[lane];
+          const uint4 xv = reinterpret_cast<const uint4*>(&sm.tile[st_i][warp * kFuR + m][0])[lane];
           const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
           for (int e = 0; e < 8; e += 2) {
@@ -157,8 +161,8 @@ __global__ void __launch_bounds__(kFuThreads, 2) compress_reduce_kernel(
             float a0, a1;
             fmul2(a0, a1, f0, f1, inv[e], inv[e + 1]);
             int c0 = __float2int_rn(a0), c1 = __float2int_rn(a1);  // saturating; NaN -> 0
-            c0 = min(max(c0, lo[e]), lo[e] + 15);
-            c1 = min(max(c1, lo[e + 1]), lo[e + 1] + 15);
+            c0 = min(max(c0, lo[e]), hi[e]);
+            c1 = min(max(c1, lo[e + 1]), hi[e + 1]);
             // float(c) by the 1.5 * 2^23 magic, as scalar adds: their results go straight into the
             // register pair the packed FMA reads
             const float d0 = __fadd_rn(__int_as_float(c0 + 0x4B400000), -12582912.0f);
@@ -170,7 +174,11 @@ __global__ void __launch_bounds__(kFuThreads, 2) compress_reduce_kernel(
         }
       }
       __syncwarp();
-      if (lane == 0) sm.ring.release(i);
+      if (lane == 0) mbar_arrive(&sm.ring.empty[st_i]);
+      if (++st_i == kFuStages) {
+        st_i = 0;
+        phase ^= 1u;
+      }
     }
     if (!ok) break;
     if (active) {
