@@ -12,7 +12,7 @@
  *     features by quantization range, keep the top ones in BF16), Inference (the rest go to
  *     4 bits; after communication everything is converted back and summed across devices).
  * The page gives no formula, bit layout or interface; the exact arithmetic below is a stated
- * reading of it (the readings are numbered R1..R14 where they are used).
+ * reading of it (the readings are numbered R1..R19 where they are used).
  *
  * Notation: P ranks, T rows (tokens), H features (columns), k features kept in BF16, H' = H - k.
  * One GPU simulates the P ranks: a tensor [P][T][H] holds every rank's partial sum, and the
