@@ -410,3 +410,14 @@ def test_per_rank_calls_equal_the_batched_call():
     assert torch.equal(torch.cat(per_side), side)
     out2 = gpu_dequant(torch.cat(per_codes), torch.cat(per_side), B, cfg.H)
     assert torch.equal(out2, out)
+
+
+@pytest.mark.parametrize("P,T,H,k", [(2, 40, 32768, 1024), (64, 8, 32768, 512)], ids=["h_max", "p_and_h_max"])
+def test_maximum_sizes_bit_exact(P, T, H, k):
+    """The largest shapes the ABI accepts: H = 32768 (selection keys fill 128 KB of shared memory)
+    and P = 64 ranks (the TMA dequant-reduce kernel's constants then take 128 KB of its shared
+    memory), through the whole path, element by element against the oracle."""
+    cfg = synth.CONFIGS["decode"].with_(name=f"max_{P}_{H}", P=P, T=T, H=H, k=k, n_out=64, calib_batches=2,
+                                        calib_T=16)
+    cs, _ = synth.colscale(cfg)
+    compare_all(cfg, _batches(cfg, cs), synth.fill_cpu(cfg, synth.EVAL, 0, cs=cs))
