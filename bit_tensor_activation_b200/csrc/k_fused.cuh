@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(kFuThreads, 2) compress_reduce_kernel(
   }
 
   // ---------------------------------------------------------------------- consumers
-  // constants [P][5][32]: inv 0-3, inv 4-7, scale 0-3, scale 4-7 (1 for kept), (zero bytes, kmask),
+  // constants [P][5][32]: inv 0-3, inv 4-7, scale 0-3, scale 4-7 (1 for kept), (-zero as signed bytes, kmask),
   // filled while the producer is already loading
   for (int idx = threadIdx.x; idx < P * 32; idx += kConsumers) {
     const int r = idx >> 5, g = idx & 31;
@@ -105,9 +105,9 @@ __global__ void __launch_bounds__(kFuThreads, 2) compress_reduce_kernel(
         const size_t p = (size_t)r * H + hg + i;
         iv[i] = inv_scale[p];
         sc[i] = ((km >> i) & 1u) ? 1.0f : scale[p];
-        const uint32_t z = zero[p];
-        if (i < 4) zlo |= z << (8 * i);
-        else zhi |= z << (8 * (i - 4));
+        const uint32_t nz = (uint32_t)(-(int)zero[p]) & 0xFFu;  // -zero as a signed byte
+        if (i < 4) zlo |= nz << (8 * i);
+        else zhi |= nz << (8 * (i - 4));
       }
     } else {
 #pragma unroll
@@ -148,7 +148,7 @@ __global__ void __launch_bounds__(kFuThreads, 2) compress_reduce_kernel(
         int lo[8], hi[8];  // clamp bounds of c: -zero and 15 - zero
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          lo[e] = -(int)(((e < 4 ? zlo : zhi) >> (8 * (e & 3))) & 0xFFu);
+          lo[e] = (int)(int8_t)(uint8_t)((e < 4 ? zlo : zhi) >> (8 * (e & 3)));  // sign-extended byte
           hi[e] = lo[e] + 15;
         }
 #pragma unroll
