@@ -321,16 +321,19 @@ def run_hq(args, cfg, world, rank, local):
     names = (["calibrate", "select", "quantize_pack", "dequant_reduce"] if args.path == "split"
              else ["calibrate", "select", "compress_reduce"])
 
-    def step_calls(xin):
+    def step_calls(xin, res=None):
+        """The step's calls on input xin; the reduced result goes to res (default: the path's own
+        output buffer)."""
+        if res is None:
+            res = B.out if args.path == "split" else fused_out
         yield lambda: hq.hq_calibrate(xin, B.ema_min, B.ema_max, cfg.beta, False)
         yield lambda: hq.hq_select_topk(B.ema_min, B.ema_max, k, B.keep_idx, B.rest_idx, B.scale,
                                         B.inv_scale, B.zero)
         if args.path == "split":
             yield lambda: hq.hq_quantize_pack(xin, B.keep_idx, B.rest_idx, B.inv_scale, B.zero, B.codes, B.side)
-            yield lambda: hq.hq_dequant_reduce(B.codes, B.side, B.keep_idx, B.rest_idx, B.scale, B.zero, B.out)
+            yield lambda: hq.hq_dequant_reduce(B.codes, B.side, B.keep_idx, B.rest_idx, B.scale, B.zero, res)
         else:
-            yield lambda: hq.hq_compress_reduce(xin, B.keep_idx, B.rest_idx, B.scale, B.inv_scale, B.zero,
-                                                fused_out)
+            yield lambda: hq.hq_compress_reduce(xin, B.keep_idx, B.rest_idx, B.scale, B.inv_scale, B.zero, res)
 
     def run_steps(n, xin, events=None):
         for i in range(n):
@@ -412,31 +415,69 @@ def run_hq(args, cfg, world, rank, local):
     fused_equal = bool(torch.equal(B.out.view(torch.int16), fused_out.view(torch.int16)))
 
     # ---- e2e: public API with pinned host buffers, copies inside the timed region ----------------
+    # Every step copies its input from pinned host memory and its result back, inside the timed
+    # region. Steps are pipelined the way a serving loop would run them: the next step's input
+    # copy (its own stream) overlaps this step's compute and result copy (a third stream), with
+    # two device input and result buffers and events ordering every reuse.
     e2e = None
     if args.e2e_steps > 0:
         xh = x.cpu().pin_memory()
-        oh = torch.empty(B.out.shape, dtype=B.out.dtype).pin_memory()
-        xd = torch.empty_like(x)
-        for _ in range(2):
-            xd.copy_(xh, non_blocking=True)
-            for call in step_calls(xd):
-                call()
-            oh.copy_(B.out, non_blocking=True)
+        xd = [torch.empty_like(x) for _ in range(2)]
+        res = [torch.empty_like(B.out if args.path == "split" else fused_out) for _ in range(2)]
+        oh = [torch.empty(r.shape, dtype=r.dtype).pin_memory() for r in res]
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        in_ready = [torch.cuda.Event() for _ in range(2)]
+        computed = [torch.cuda.Event() for _ in range(2)]
+        copied_out = [torch.cuda.Event() for _ in range(2)]
+
+        def e2e_steps(n):
+            for i in range(n):
+                b = i & 1
+                with torch.cuda.stream(s_in):
+                    if i >= 2:
+                        s_in.wait_event(computed[b])  # step i-2 is done with xd[b]
+                    xd[b].copy_(xh, non_blocking=True)
+                    in_ready[b].record(s_in)
+                stream.wait_event(in_ready[b])
+                if i >= 2:
+                    stream.wait_event(copied_out[b])  # step i-2's result has left res[b]
+                for call in step_calls(xd[b], res[b]):
+                    call()
+                computed[b].record(stream)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(computed[b])
+                    oh[b].copy_(res[b], non_blocking=True)
+                    copied_out[b].record(s_out)
+
+        e2e_steps(2)
         torch.cuda.synchronize()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(args.e2e_steps):
-            xd.copy_(xh, non_blocking=True)
-            for call in step_calls(xd):
-                call()
-            oh.copy_(B.out, non_blocking=True)
+        s_in.wait_event(e0)
+        s_out.wait_event(e0)
+        e2e_steps(args.e2e_steps)
+        tail = torch.cuda.Event()
+        tail.record(s_out)
+        stream.wait_event(tail)
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world, dev)
         e2e = {"value": world * P * T * H * 2 / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                "h2d_bytes_per_step": xh.numel() * xh.element_size(),
-               "d2h_bytes_per_step": oh.numel() * oh.element_size(), "ms_per_step": e2e_ms}
+               "d2h_bytes_per_step": oh[0].numel() * oh[0].element_size(), "ms_per_step": e2e_ms,
+               "pipelined": "next step's input copy overlaps this step's compute and result copy"}
+        # the last step's copied-back result against the same reduction of x on the parameters that
+        # step selected (calibration moves them a little every step)
+        check = torch.empty_like(res[0])
+        if args.path == "split":
+            hq.hq_quantize_pack(x, B.keep_idx, B.rest_idx, B.inv_scale, B.zero, B.codes, B.side)
+            hq.hq_dequant_reduce(B.codes, B.side, B.keep_idx, B.rest_idx, B.scale, B.zero, check)
+        else:
+            hq.hq_compress_reduce(x, B.keep_idx, B.rest_idx, B.scale, B.inv_scale, B.zero, check)
+        torch.cuda.synchronize()
+        if not torch.equal(oh[(args.e2e_steps - 1) & 1].view(torch.int16).to(dev), check.view(torch.int16)):
+            raise RuntimeError("the end-to-end result differs from the device-resident reduction")
 
     st = hq.hq_read_device_error()
     if st != hq.HQ_OK:
