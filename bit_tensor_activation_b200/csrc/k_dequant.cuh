@@ -352,7 +352,7 @@ constexpr int kDtSideCols = 32;                  // side box height: kept featur
 constexpr int kDtMaxStagedKept = kDtSideCols;    // slices with more read the side buffer from HBM
 constexpr unsigned kDtSideBytes = kDtTileRows * kDtSideCols * 2;
 static_assert(kDtR == 4, "a consumer lane reads its rows' kept sums as one float4");
-static_assert(kDtTileRows == 32, "the kept-sum warp gives one lane to each row of a block");
+static_assert(kDtTileRows == 32, "the kept-sum warp covers a block's 32 rows with 8 lanes of 4 rows");
 
 struct DtSmem {
   alignas(128) uint32_t tile[kDtStages][kDtG][kDtTileRows][kDtWords];
