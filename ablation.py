@@ -22,6 +22,14 @@ Variants:
   because they are computed for every feature.
 - ``int4_only``: k = 0.
 - ``bf16_only``: k = H, the uncompressed bf16 wire; only the fp32 summation remains.
+- ``two_step``: a two-step compressed all-reduce (reduce-scatter, then all-gather), the scheme
+  the "Flash Communication" abstract among the source pages names without an algorithm. The design
+  used here: step 1 is the ``topk`` path with bf16 output, and reducer j owns row block j of
+  it. In step 2 each reducer quantizes its block again with the same hybrid scheme, and every
+  rank dequantizes all blocks (a reduction over P = 1). The step-2 grids and kept features come
+  from calibration and selection with P = 1 on the reduced calibration batches. On one GPU the
+  row blocks together are the whole output, so step 2 is one quantize-pack and one
+  dequant-reduce call with P = 1; the time reported is step 2's.
 
 For every variant the tool reports MSE, MSE relative to the mean square of the exact sum, the
 largest absolute error and the wire compression ratio.  It also times the variant's reduction:
@@ -48,7 +56,7 @@ if ROOT not in sys.path:
 import bit_tensor_activation_b200 as hq  # noqa: E402
 import synth  # noqa: E402
 
-VARIANTS = ("topk", "topk_bf16_shards", "random_k", "int4_only", "bf16_only")
+VARIANTS = ("topk", "topk_bf16_shards", "random_k", "int4_only", "bf16_only", "two_step")
 
 
 def peak_gbs() -> float:
@@ -119,6 +127,9 @@ def run_workload(cfg: synth.Config, reps: int, flush: torch.Tensor, seed: int) -
     out = torch.empty((T, H), dtype=torch.float32, device=dev)
     rows = []
     for name in VARIANTS:
+        if name == "two_step":
+            rows.append(two_step(cfg, x, exact, mean_sq, keep, rest, scale, inv, zero, cs_dev, reps, flush))
+            continue
         kk, rr = sets["topk" if name == "topk_bf16_shards" else name]
         kn = kk.shape[0]
         codes = torch.empty((P, T, (H - kn) // 8), dtype=torch.int32, device=dev)
@@ -143,6 +154,56 @@ def run_workload(cfg: synth.Config, reps: int, flush: torch.Tensor, seed: int) -
     if st != hq.HQ_OK:
         raise RuntimeError(f"{cfg.name}: device error {hq.hq_status_string(st)}")
     return rows
+
+
+def one_step_bf16(x, keep, rest, scale, inv, zero):
+    """Step 1: the hybrid quantize-pack of every rank and the rank-ordered reduction, bf16 out."""
+    P, T, H = x.shape
+    k = keep.shape[0]
+    codes = torch.empty((P, T, (H - k) // 8), dtype=torch.int32, device=x.device)
+    side = torch.empty((P, k, T), dtype=torch.int16, device=x.device)
+    hq.hq_quantize_pack(x, keep, rest, inv, zero, codes, side)
+    y = torch.empty((T, H), dtype=torch.int16, device=x.device)
+    hq.hq_dequant_reduce(codes, side, keep, rest, scale, zero, y)
+    return y
+
+
+def two_step(cfg, x, exact, mean_sq, keep, rest, scale, inv, zero, cs_dev, reps, flush) -> dict:
+    dev = x.device
+    P, T, H, k = cfg.P, cfg.T, cfg.H, cfg.k
+    # step-2 grids: calibration (P = 1) on the reduced calibration batches, then selection
+    e2min = torch.empty((1, H), dtype=torch.float32, device=dev)
+    e2max = torch.empty_like(e2min)
+    cal = torch.empty((P, cfg.calib_T, H), dtype=torch.int16, device=dev)
+    for b in range(cfg.calib_batches):
+        synth.fill_gpu(cfg, synth.CALIB, b, cal, cs_dev, T=cfg.calib_T)
+        y_cal = one_step_bf16(cal, keep, rest, scale, inv, zero)
+        hq.hq_calibrate(y_cal[None], e2min, e2max, cfg.beta, b == 0)
+    del cal
+    keep2 = torch.empty(k, dtype=torch.int32, device=dev)
+    rest2 = torch.empty(H - k, dtype=torch.int32, device=dev)
+    scale2 = torch.empty((1, H), dtype=torch.float32, device=dev)
+    inv2 = torch.empty_like(scale2)
+    zero2 = torch.empty((1, H), dtype=torch.uint8, device=dev)
+    hq.hq_select_topk(e2min, e2max, k, keep2, rest2, scale2, inv2, zero2)
+    # step 1 on the evaluation batch, then step 2: quantize the reduced rows again, dequantize
+    y = one_step_bf16(x, keep, rest, scale, inv, zero)[None].contiguous()
+    codes2 = torch.empty((1, T, (H - k) // 8), dtype=torch.int32, device=dev)
+    side2 = torch.empty((1, k, T), dtype=torch.int16, device=dev)
+    out = torch.empty((T, H), dtype=torch.float32, device=dev)
+
+    def step2():
+        hq.hq_quantize_pack(y, keep2, rest2, inv2, zero2, codes2, side2)
+        hq.hq_dequant_reduce(codes2, side2, keep2, rest2, scale2, zero2, out)
+
+    us = timed_us(step2, reps, flush)
+    step2()
+    err = out.double() - exact
+    mse = float((err * err).mean())
+    step2_bytes = (2 * T * H + T * (H - k) // 2 + 2 * T * k) + (T * (H - k) // 2 + 2 * T * k + 4 * T * H)
+    return {"workload": cfg.name, "variant": "two_step", "k": k, "mse": mse, "rel_mse": mse / mean_sq,
+            "max_abs_err": float(err.abs().max()), "ratio": 2 * H / ((H - k) / 2 + 2 * k),
+            "reduce_us": us, "reduce_gbs": step2_bytes / us / 1e3}
 
 
 def main() -> None:
