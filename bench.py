@@ -250,7 +250,8 @@ def run_reference(args, cfg, world, rank):
         "data": "synthetic",
         "config": {"workload": describe(cfg), "P": cfg.P, "T": cfg.T, "H": cfg.H, "k": cfg.k,
                    "path": "split", "parallelism": "replicas"},
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "host_cpus": os.cpu_count(), "kind": "oracle",
+                         "sample": sample},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "compression_ratio": compression_ratio(cfg),
     }
@@ -492,7 +493,8 @@ def run_hq(args, cfg, world, rank, local):
         t = step.run(S)
         reps = max(1, round(args.cpu_seconds / t))
         t += sum(step.run(S) for _ in range(reps - 1))
-        cpu = {"value": reps * P * S * H * 2 / t / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+        cpu = {"value": reps * P * S * H * 2 / t / 1e9, "unit": "GB/s", "cores": 1, "host_cpus": os.cpu_count(),
+               "kind": "oracle",
                "sample": f"rows 0..{S - 1} of the evaluation batch, all {P} ranks, {reps} passes of calibrate + "
                          f"select + quantize-pack + dequant-reduce, {t:.1f} s single-threaded"}
 
