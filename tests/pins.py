@@ -197,6 +197,24 @@ def pin_calibrate_ema(o):
         assert np.all(np.abs(emx - want) <= tol) and np.all(np.abs(emn - want) <= tol), f"beta^{n} * m0"
 
 
+def pin_calibrate_ema_golden(o):
+    """One moving-average update worked by hand (tests/golden/ema_cases.json): two products and
+    a sum, each rounded to fp32, with 1 - beta an fp32 subtraction.  Each case's value differs
+    from the one a single rounding (fused, double-precision or delta-form update) or the literal
+    0.1f would give."""
+    g = _golden("ema_cases.json")
+    for c in g["cases"]:
+        a = f32_to_bf16_torch(np.array([c["a"]], np.float32))[0]
+        b = f32_to_bf16_torch(np.array([c["b"]], np.float32))[0]
+        assert bf16_to_f32(np.array([a]))[0] == c["a"] and bf16_to_f32(np.array([b]))[0] == c["b"]
+        emn, emx = o.calibrate(np.full((1, 3, 8), a, np.uint16), g["beta"], True)
+        emn, emx = o.calibrate(np.full((1, 3, 8), b, np.uint16), g["beta"], False, emn, emx)
+        want = int(c["ema_hex"], 16)
+        for name, v in (("ema_min", emn), ("ema_max", emx)):
+            got = v.view(np.uint32)
+            assert np.all(got == want), f"{name} after (a={c['a']}, b={c['b']}): {got[0, 0]:08X}, want {want:08X}"
+
+
 # ---------------------------------------------------------------------------------------------
 # Selection (readings R4, R5)
 # ---------------------------------------------------------------------------------------------
@@ -206,6 +224,18 @@ def pin_select_golden(o):
     for c in g["cases"]:
         keep, rest, score = o.select(rng_, c["k"])
         assert score.tolist() == g["expect_score"], "score = sum over ranks"
+        assert keep.tolist() == c["keep"] and rest.tolist() == c["rest"], f"k={c['k']}: keep {keep}, rest {rest}"
+
+
+def pin_select_rank_order_golden(o):
+    """The score is summed in fp32 in rank order (tests/golden/order_cases.json, "score"): at
+    2^24 the spacing is 2, so ranges 2^24, 1, 1 sum to 2^24, not 2^24 + 2, and that decides
+    which feature is kept."""
+    g = _golden("order_cases.json")["score"]
+    rng_ = np.array(g["range"], np.float32)
+    for c in g["cases"]:
+        keep, rest, score = o.select(rng_, c["k"])
+        assert score.tolist() == g["expect_score"], f"score {score.tolist()}"
         assert keep.tolist() == c["keep"] and rest.tolist() == c["rest"], f"k={c['k']}: keep {keep}, rest {rest}"
 
 
@@ -337,6 +367,37 @@ def pin_reduce_dequant_sum(o):
     kept = sf.astype(np.float64).sum(axis=0)
     assert np.all(np.abs(out[:, keep] - kept) <= P * 2.0 ** -23 * np.abs(sf).sum(axis=0)), "kept sum"
     assert np.array_equal(out[:, keep], _numpy_rank_sum(sf)), "kept: exact rank-ordered sum"
+
+
+def pin_reduce_order_golden(o):
+    """Rounding and rank order of the reduction, worked by hand (tests/golden/order_cases.json):
+    a 4-bit feature takes one rounding per rank (a fused multiply-add), and both 4-bit and kept
+    features are summed in rank order 0..P-1 -- cases whose result changes under a separate
+    multiply and add, under reversed rank order, or with an exact accumulator."""
+    g = _golden("order_cases.json")
+    P = g["P"]
+    cases = g["dequant_4bit"]
+    words, zero, scale = _one_group([[c["qz"][r] for c in cases] for r in range(P)],
+                                    [[c["scale"][r] for c in cases] for r in range(P)])
+    side = np.zeros((P, 0, 1), np.uint16)
+    out = o.dequant_reduce(words, side, 8, np.zeros(0, np.int32), np.arange(8, dtype=np.int32), scale, zero,
+                           out_f32=True)
+    for i, c in enumerate(cases):
+        got = f32_bits(out[0, i])
+        assert got == int(c["out_hex"], 16), f"4-bit case {i}: {got:08X}, want {c['out_hex']}"
+    kept = g["kept"]
+    k = 8
+    side = np.zeros((P, k, 1), np.uint16)
+    for j, c in enumerate(kept):
+        for r in range(P):
+            side[r, j, 0] = int(c["side_hex"][r], 16)
+    keep = np.arange(k, dtype=np.int32)
+    words = np.zeros((P, 1, 0), np.uint32)
+    out = o.dequant_reduce(words, side, k, keep, np.zeros(0, np.int32), np.ones((P, k), np.float32),
+                           np.zeros((P, k), np.uint8), out_f32=True)
+    for j, c in enumerate(kept):
+        got = f32_bits(out[0, j])
+        assert got == int(c["out_hex"], 16), f"kept case {j}: {got:08X}, want {c['out_hex']}"
 
 
 def pin_reduce_error_bound(o):
@@ -531,8 +592,9 @@ def pin_bf16_shards_rounding_bound(o):
 
 ALL_PINS = [
     pin_bf16_round, pin_quantize_golden, pin_quantize_nearest_grid, pin_params_golden,
-    pin_params_closed_form, pin_calibrate_single_batch, pin_calibrate_ema, pin_select_golden,
-    pin_select_brute_force, pin_pack_golden, pin_pack_unpack, pin_reduce_all_kept,
-    pin_nan_outputs, pin_reduce_dequant_sum, pin_reduce_error_bound, pin_irwin_hall, pin_outliers_selected,
+    pin_params_closed_form, pin_calibrate_single_batch, pin_calibrate_ema, pin_calibrate_ema_golden,
+    pin_select_golden, pin_select_rank_order_golden, pin_select_brute_force, pin_pack_golden, pin_pack_unpack,
+    pin_reduce_all_kept, pin_nan_outputs, pin_reduce_dequant_sum, pin_reduce_order_golden, pin_reduce_error_bound,
+    pin_irwin_hall, pin_outliers_selected,
     pin_selection_benefit, pin_bf16_shards_golden, pin_bf16_shards_exact_products, pin_bf16_shards_rounding_bound,
 ]

@@ -52,8 +52,28 @@ MUTANTS = [
      "acc = ref_bf16_value(ref_bf16_round(acc + v));"),
     ("bf16_shards_sign_flipped", "float v = (float)(q - (int)zero[p]) * scale[p];",
      "float v = (float)((int)zero[p] - q) * scale[p];"),
+    # rounding and order choices of the readings R1, R3, R4, R9, R10
     ("dequant_mul_then_add", "acc = fmaf((float)(q - (int)zero[p]), scale[p], acc);",
-     "acc = acc + (float)(q - (int)zero[p]) * scale[p] * 1.0009765625f;"),
+     "acc = acc + (float)(q - (int)zero[p]) * scale[p];"),
+    ("dequant_exact_accumulator", "acc = fmaf((float)(q - (int)zero[p]), scale[p], acc);",
+     "static double dacc; if (r == 0) dacc = 0.0; dacc += (double)(q - (int)zero[p]) * scale[p]; acc = (float)dacc;"),
+    ("dequant_ranks_reversed", "for (int r = 0; r < P; ++r) {\n        uint32_t word",
+     "for (int r = P - 1; r >= 0; --r) {\n        uint32_t word"),
+    ("kept_ranks_reversed", "for (int r = 0; r < P; ++r) acc = acc + ref_bf16_value(side",
+     "for (int r = P - 1; r >= 0; --r) acc = acc + ref_bf16_value(side"),
+    ("score_ranks_reversed", "for (int r = 0; r < P; ++r) acc = acc + range[(size_t)r * H + h];",
+     "for (int r = P - 1; r >= 0; --r) acc = acc + range[(size_t)r * H + h];"),
+    ("score_in_double", "float acc = 0.0f;\n    for (int r = 0; r < P; ++r) acc = acc + range[(size_t)r * H + h];",
+     "double dacc = 0.0;\n    for (int r = 0; r < P; ++r) dacc = dacc + range[(size_t)r * H + h];\n    float acc = (float)dacc;"),
+    ("decay_complement_literal", "const float one_minus_beta = 1.0f - beta;", "const float one_minus_beta = 0.1f;"),
+    ("ema_fused_update", "a = beta * ema_max[i];\n        b = one_minus_beta * bmax;\n        ema_max[i] = a + b;",
+     "ema_max[i] = fmaf(beta, ema_max[i], one_minus_beta * bmax);"),
+    ("ema_delta_form", "a = beta * ema_max[i];\n        b = one_minus_beta * bmax;\n        ema_max[i] = a + b;",
+     "ema_max[i] = ema_max[i] + one_minus_beta * (bmax - ema_max[i]);"),
+    ("ema_in_double", "a = beta * ema_max[i];\n        b = one_minus_beta * bmax;\n        ema_max[i] = a + b;",
+     "ema_max[i] = (float)((double)beta * ema_max[i] + (double)one_minus_beta * bmax);"),
+    ("inv_scale_15_over_range", "float inv = 1.0f / s;", "float inv = 15.0f / rg;"),
+    ("scale_times_reciprocal", "float s = rg / 15.0f;", "float s = rg * (1.0f / 15.0f);"),
 ]
 
 
