@@ -43,6 +43,8 @@ _lib.hq_status_string.argtypes = [_i32]
 _lib.hq_status_string.restype = ctypes.c_char_p
 _lib.hq_selftest_bounded_wait.argtypes = [ctypes.c_longlong, _vp]
 _lib.hq_selftest_bounded_wait.restype = _i32
+_lib.hq_selftest_set_pipeline_stall.argtypes = [ctypes.c_longlong, ctypes.c_longlong]
+_lib.hq_selftest_set_pipeline_stall.restype = _i32
 _lib.hq_wire_bytes_per_row.argtypes = [_i32, _i32]
 _lib.hq_wire_bytes_per_row.restype = ctypes.c_int64
 
@@ -51,7 +53,7 @@ HQ_OUT_BF16, HQ_OUT_F32 = 0, 1
 
 EXPORTS = ["hq_calibrate", "hq_select_topk", "hq_quantize_pack", "hq_dequant_reduce",
            "hq_dequant_reduce_bf16_shards", "hq_compress_reduce", "hq_status_string", "hq_read_device_error", "hq_wire_bytes_per_row",
-           "hq_selftest_bounded_wait"]
+           "hq_selftest_bounded_wait", "hq_selftest_set_pipeline_stall"]
 
 
 class HQError(RuntimeError):
@@ -179,8 +181,16 @@ def hq_selftest_bounded_wait(limit_cycles: int, stream=None, device=None) -> Non
     _check(_lib.hq_selftest_bounded_wait(int(limit_cycles), _stream(stream, device)), "hq_selftest_bounded_wait")
 
 
+def hq_selftest_set_pipeline_stall(consumer_limit_cycles: int, producer_delay_cycles: int) -> None:
+    """Self-test of the pipelines' abort path: later pipeline launches delay their producers and
+    bound their consumers' waits by consumer_limit_cycles; (0, 0) restores the normal bounds."""
+    _check(_lib.hq_selftest_set_pipeline_stall(int(consumer_limit_cycles), int(producer_delay_cycles)),
+           "hq_selftest_set_pipeline_stall")
+
+
 def hq_read_device_error(stream=None, device=None) -> int:
-    """Synchronises the stream; returns and clears the device error word (0 = none)."""
+    """Takes and clears the device error word atomically, after the work ordered before it on the
+    stream (0 = none)."""
     return int(_lib.hq_read_device_error(_stream(stream, device)))
 
 

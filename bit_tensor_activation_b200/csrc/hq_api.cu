@@ -8,6 +8,8 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
+#include <type_traits>
 #include <mutex>
 
 #include "hq.h"
@@ -24,6 +26,7 @@ namespace {
 constexpr int kMaxRanks = 64;
 static_assert(kMaxRanks <= hq::kSelMaxRanks, "the parameter kernel stages one range per rank");
 constexpr int kMaxDevices = 64;
+constexpr long long kMaxStallDelayCycles = 1LL << 31;  // about a second
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
@@ -34,11 +37,22 @@ hq_status check_shape(int P, int H, int k) {
   return HQ_OK;
 }
 
+// Resident CTAs per SM of one kernel for each rank count P (its shared memory grows with P),
+// queried once per device; the kernel's dynamic shared-memory limit is raised to the largest size
+// requested so far.
+struct OccupancyCache {
+  int smem_set = 0;
+  int per_sm[kMaxRanks + 1] = {};
+};
+
 // Launch-shape facts cached per device: SM count and resident CTAs per SM of each kernel.
 struct DeviceInfo {
   int sms = 0;
   int qt_blocks = 0;
   bool select_smem_set = false;
+  OccupancyCache dequant_tma[2][2];  // [fp32 out][bf16 shards]
+  OccupancyCache dequant_cp[2][2];
+  OccupancyCache fused[2];           // [fp32 out]
 };
 
 // cuTensorMapEncodeTiled, fetched once through the runtime (no link-time libcuda dependency).
@@ -95,6 +109,37 @@ hq_status device_info(DeviceInfo** out) {
 
 hq_status launched() { return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA; }
 
+// CTAs of `kern` resident per SM with `smem` bytes of dynamic shared memory (at least 1), from the
+// device's cache; the first use for a P sets the shared-memory limit and runs the query.
+template <typename Kernel>
+hq_status occupancy(OccupancyCache& c, Kernel kern, int threads, size_t smem, int P, int* per_sm) {
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  if (c.per_sm[P] == 0) {
+    if ((int)smem > c.smem_set) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return HQ_ERR_CUDA;
+      c.smem_set = (int)smem;
+    }
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, smem) != cudaSuccess) return HQ_ERR_CUDA;
+    c.per_sm[P] = n < 1 ? 1 : n;
+  }
+  *per_sm = c.per_sm[P];
+  return HQ_OK;
+}
+
+// Wait bounds of the pipeline kernels.  Normal launches use the long default everywhere; the
+// abort self-test (hq_selftest_set_pipeline_stall) shortens the consumers' bound and delays the
+// producers' first loads.
+std::atomic<long long> g_stall_consumer_limit{0};
+std::atomic<long long> g_stall_producer_delay{0};
+
+hq::WaitLimits wait_limits() {
+  const long long c = g_stall_consumer_limit.load(), d = g_stall_producer_delay.load();
+  if (c == 0 && d == 0) return hq::WaitLimits{hq::kWaitLimitCycles, hq::kWaitLimitCycles, 0};
+  return hq::WaitLimits{c, hq::kWaitLimitCycles, d};
+}
+
 long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
 
 // Slices x row chunks for the dequant-reduce and fused kernels: one wave of CTAs at most.
@@ -111,7 +156,7 @@ void slice_chunks(int T, int S, long long resident, int rows_per_block, int* chu
 template <typename OutT, bool kShard>
 hq_status launch_dequant(const uint32_t* codes, const uint16_t* side, int P, int T, int H, int k,
                          const int32_t* keep_idx, const float* scale, const uint8_t* zero, void* out,
-                         cudaStream_t st, const DeviceInfo& d) {
+                         cudaStream_t st, DeviceInfo& d) {
   const int S = (H + 8 * hq::kDqSliceGroups - 1) / (8 * hq::kDqSliceGroups);
   const int Wr = (H - k) / 8;
   CUtensorMap map, map_side;
@@ -124,31 +169,24 @@ hq_status launch_dequant(const uint32_t* codes, const uint16_t* side, int P, int
                         encode_2d(&map_side, side, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)T, (uint64_t)P * k,
                                   hq::kDtTileRows, hq::kDtSideCols, CU_TENSOR_MAP_L2_PROMOTION_NONE);
   if (!side_tma) map_side = map;  // never read
+  constexpr int kF32 = std::is_same<OutT, float>::value ? 1 : 0;
   if (tma) {
     const size_t smem = hq::dt_smem_bytes(P);
     auto kern = hq::dequant_reduce_tma_kernel<OutT, kShard>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return HQ_ERR_CUDA;
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, hq::kDtThreads, smem) != cudaSuccess)
-      return HQ_ERR_CUDA;
-    if (per_sm < 1) per_sm = 1;
+    if (occupancy(d.dequant_tma[kF32][kShard], kern, hq::kDtThreads, smem, P, &per_sm) != HQ_OK) return HQ_ERR_CUDA;
     int chunks, rpc;
     slice_chunks(T, S, (long long)d.sms * per_sm, hq::kDtTileRows, &chunks, &rpc);
     kern<<<(unsigned)(S * chunks), hq::kDtThreads, smem, st>>>(map, map_side, side_tma ? 1 : 0, side, P, T, H, k,
                                                                 keep_idx, scale, zero,
                                                                 static_cast<OutT*>(out), S, chunks, rpc,
-                                                                hq::kWaitLimitCycles);
+                                                                wait_limits());
     return launched();
   }
   const size_t smem = hq::dq_smem_bytes(P);
   auto kern = hq::dequant_reduce_kernel<OutT, kShard>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return HQ_ERR_CUDA;
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, hq::kDqThreads, smem) != cudaSuccess)
-    return HQ_ERR_CUDA;
-  if (per_sm < 1) per_sm = 1;
+  if (occupancy(d.dequant_cp[kF32][kShard], kern, hq::kDqThreads, smem, P, &per_sm) != HQ_OK) return HQ_ERR_CUDA;
   int chunks, rpc;
   slice_chunks(T, S, (long long)d.sms * per_sm, hq::kDqR, &chunks, &rpc);
   kern<<<(unsigned)(S * chunks), hq::kDqThreads, smem, st>>>(codes, side, P, T, H, k, keep_idx, scale,
@@ -159,7 +197,7 @@ hq_status launch_dequant(const uint32_t* codes, const uint16_t* side, int P, int
 template <typename OutT>
 hq_status launch_fused(const uint16_t* x, int P, int T, int H, int k, const int32_t* keep_idx,
                        const float* scale, const float* inv_scale, const uint8_t* zero, void* out,
-                       cudaStream_t st, const DeviceInfo& d) {
+                       cudaStream_t st, DeviceInfo& d) {
   const int S = (H + hq::kFuSlice - 1) / hq::kFuSlice;
   CUtensorMap map;
   if (!encode_2d(&map, x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)H, (uint64_t)P * T, hq::kFuSlice,
@@ -167,19 +205,23 @@ hq_status launch_fused(const uint16_t* x, int P, int T, int H, int k, const int3
     return HQ_ERR_CUDA;
   const size_t smem = hq::fu_smem_bytes(P);
   auto kern = hq::compress_reduce_kernel<OutT>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return HQ_ERR_CUDA;
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, hq::kFuThreads, smem) != cudaSuccess)
+  if (occupancy(d.fused[std::is_same<OutT, float>::value ? 1 : 0], kern, hq::kFuThreads, smem, P, &per_sm) != HQ_OK)
     return HQ_ERR_CUDA;
-  if (per_sm < 1) per_sm = 1;
   int chunks, rpc;
   slice_chunks(T, S, (long long)d.sms * per_sm, hq::kFuTileRows, &chunks, &rpc);
   kern<<<(unsigned)(S * chunks), hq::kFuThreads, smem, st>>>(map, P, T, H, k, keep_idx, scale, inv_scale, zero,
                                                               static_cast<OutT*>(out), S, chunks, rpc,
-                                                              hq::kWaitLimitCycles);
+                                                              wait_limits());
   return launched();
 }
+
+// hq_read_device_error: the error word is taken and cleared in one atomic exchange, so an error a
+// kernel on another stream records at the same moment lands either in this read or in the word
+// for the next one; the value goes through a second device word to the host.
+__device__ unsigned int g_error_taken = 0;
+__global__ void take_error_kernel() { g_error_taken = atomicExch(&hq::g_error_word, 0u); }
+std::mutex g_error_mu;  // one read at a time per process (they share g_error_taken)
 
 // Bounded-wait self-test: one thread waits on an mbarrier that nothing arrives on.
 __global__ void selftest_wait_kernel(long long limit) {
@@ -287,7 +329,7 @@ hq_status hq_quantize_pack(const uint16_t* x, int P, int T, int H, int k, const 
   hq::quantize_pack_tma_kernel<<<(unsigned)(S * J), hq::kQtThreads, sizeof(hq::QtSmem) + 128,
                                  (cudaStream_t)stream>>>(map_x, x, P, T, H, k, keep_idx, rest_idx,
                                                          inv_scale, zero, codes, side, S, (int)J,
-                                                         hq::kWaitLimitCycles);
+                                                         wait_limits());
   return launched();
 }
 
@@ -346,12 +388,11 @@ const char* hq_status_string(hq_status s) {
 
 hq_status hq_read_device_error(void* stream) {
   cudaStream_t st = (cudaStream_t)stream;
+  std::lock_guard<std::mutex> lock(g_error_mu);
+  take_error_kernel<<<1, 1, 0, st>>>();
+  if (cudaGetLastError() != cudaSuccess) return HQ_ERR_CUDA;
   unsigned int v = 0;
-  if (cudaMemcpyFromSymbolAsync(&v, hq::g_error_word, sizeof v, 0, cudaMemcpyDeviceToHost, st) != cudaSuccess)
-    return HQ_ERR_CUDA;
-  if (cudaStreamSynchronize(st) != cudaSuccess) return HQ_ERR_CUDA;
-  const unsigned int zero = 0;
-  if (cudaMemcpyToSymbolAsync(hq::g_error_word, &zero, sizeof zero, 0, cudaMemcpyHostToDevice, st) != cudaSuccess)
+  if (cudaMemcpyFromSymbolAsync(&v, g_error_taken, sizeof v, 0, cudaMemcpyDeviceToHost, st) != cudaSuccess)
     return HQ_ERR_CUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess) return HQ_ERR_CUDA;
   return (hq_status)v;
@@ -361,6 +402,15 @@ hq_status hq_selftest_bounded_wait(long long limit_cycles, void* stream) {
   if (limit_cycles < 0) return HQ_ERR_INVALID_ARG;
   selftest_wait_kernel<<<1, 1, 0, (cudaStream_t)stream>>>(limit_cycles);
   return launched();
+}
+
+hq_status hq_selftest_set_pipeline_stall(long long consumer_limit_cycles, long long producer_delay_cycles) {
+  if (consumer_limit_cycles < 0 || producer_delay_cycles < 0 || producer_delay_cycles > kMaxStallDelayCycles)
+    return HQ_ERR_INVALID_ARG;
+  if ((consumer_limit_cycles == 0) != (producer_delay_cycles == 0)) return HQ_ERR_INVALID_ARG;
+  g_stall_consumer_limit.store(consumer_limit_cycles);
+  g_stall_producer_delay.store(producer_delay_cycles);
+  return HQ_OK;
 }
 
 int64_t hq_wire_bytes_per_row(int H, int k) {

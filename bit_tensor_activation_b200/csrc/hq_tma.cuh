@@ -20,6 +20,23 @@ namespace hq {
 // Default bound of one wait: about one second at B200 clocks.
 constexpr long long kWaitLimitCycles = 2000000000LL;
 
+// Bounds of a pipeline's waits, in clock cycles.  consumer: a consumer waiting for a stage to
+// fill (or for another warp's hand-off); producer: the producer waiting for a stage to be
+// released, and its drain after an abort.  start_delay: cycles the producer lane idles before its
+// first load -- 0 in every normal launch; the abort self-test sets it above a short consumer
+// bound, so that the consumers give up while the producer still has loads to issue and drain.
+struct WaitLimits {
+  long long consumer;
+  long long producer;
+  long long start_delay;
+};
+
+__device__ __forceinline__ void producer_start_delay(long long cycles) {
+  if (cycles <= 0) return;
+  const long long t0 = clock64();
+  while (clock64() - t0 < cycles) __nanosleep(1000);
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
 }

@@ -473,7 +473,7 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
     const uint16_t* __restrict__ side, int P, int T, int H,
     int k, const int32_t* __restrict__ keep_idx, const float* __restrict__ scale,
     const uint8_t* __restrict__ zero, OutT* __restrict__ out, int S, int chunks, int rows_per_chunk,
-    long long wait_limit) {
+    WaitLimits lim) {
   extern __shared__ __align__(128) unsigned char s_raw[];
   DtSmem& sm = *reinterpret_cast<DtSmem*>(s_raw);
   float4* s_const = reinterpret_cast<float4*>(s_raw + ((sizeof(DtSmem) + 127) & ~size_t(127)));
@@ -507,9 +507,10 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
     if (lane == 0) {
       prefetch_tensor_map(&tmap_codes);
       if (stage_side) prefetch_tensor_map(&tmap_side);
+      producer_start_delay(lim.start_delay);
       int issued = 0, bi = 0, g = 0;
       for (int i = 0; i < n_slots_total; ++i) {
-        if (!sm.ring.acquire(i, abort, wait_limit)) break;
+        if (!sm.ring.acquire(i, abort, lim.producer)) break;
         const int st = i % kDtStages;
         const int r0 = g * kDtG, nr = min(kDtG, P - r0);
         mbar_arrive_expect_tx(&sm.ring.full[st], (unsigned)nr * (kDtTileBytes + (stage_side ? kDtSideBytes : 0u)));
@@ -526,21 +527,21 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
           ++bi;
         }
       }
-      if (*abort) sm.ring.drain(issued, wait_limit);
+      if (*abort) sm.ring.drain(issued, lim.producer);
     }
     return;
   }
 
   if (warp == kDtKeptWarp) {  // ------------------------------------------ kept sums
     if (stage_side) {
-      if (nk <= 8) dt_kept_sums<8>(sm, nk, P, nblk, n_groups, abort, wait_limit);
-      else if (nk <= 16) dt_kept_sums<16>(sm, nk, P, nblk, n_groups, abort, wait_limit);
-      else dt_kept_sums<kDtSideCols>(sm, nk, P, nblk, n_groups, abort, wait_limit);
+      if (nk <= 8) dt_kept_sums<8>(sm, nk, P, nblk, n_groups, abort, lim.consumer);
+      else if (nk <= 16) dt_kept_sums<16>(sm, nk, P, nblk, n_groups, abort, lim.consumer);
+      else dt_kept_sums<kDtSideCols>(sm, nk, P, nblk, n_groups, abort, lim.consumer);
     } else if (lane == 0) {  // only releases the ring slots
       int st_i = 0;
       unsigned phase = 0;
       for (int i = 0; i < n_slots_total; ++i) {
-        if (!mbar_wait(&sm.ring.full[st_i], phase, abort, wait_limit)) break;
+        if (!mbar_wait(&sm.ring.full[st_i], phase, abort, lim.consumer)) break;
         mbar_arrive(&sm.ring.empty[st_i]);
         if (++st_i == kDtStages) {
           st_i = 0;
@@ -582,7 +583,7 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
       for (int e = 0; e < 8; ++e) acc[m][e] = 0.0f;
     bool ok = true;
     for (int g = 0; g < n_groups; ++g) {
-      if (!mbar_wait(&sm.ring.full[st_i], phase, abort, wait_limit)) {
+      if (!mbar_wait(&sm.ring.full[st_i], phase, abort, lim.consumer)) {
         ok = false;
         break;
       }
@@ -601,7 +602,7 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
     if (!ok) break;
     if (stage_side) {
       const int buf = bi & 1;
-      if (!mbar_wait(&sm.ksum_full[buf], (bi >> 1) & 1, abort, wait_limit)) break;
+      if (!mbar_wait(&sm.ksum_full[buf], (bi >> 1) & 1, abort, lim.consumer)) break;
       dt_patch_kept(D, acc, &sm.k.ksum[buf][0][0], q.ja, nk, warp);
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.ksum_empty[buf]);

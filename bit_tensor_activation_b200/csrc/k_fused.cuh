@@ -47,7 +47,7 @@ __global__ void __launch_bounds__(kFuThreads, 2) compress_reduce_kernel(
     const __grid_constant__ CUtensorMap tmap_x, int P, int T, int H, int k,
     const int32_t* __restrict__ keep_idx, const float* __restrict__ scale,
     const float* __restrict__ inv_scale, const uint8_t* __restrict__ zero, OutT* __restrict__ out, int S,
-    int chunks, int rows_per_chunk, long long wait_limit) {
+    int chunks, int rows_per_chunk, WaitLimits lim) {
   extern __shared__ __align__(128) unsigned char s_raw[];
   FuSmem& sm = *reinterpret_cast<FuSmem*>(s_raw);
   float4* s_const = reinterpret_cast<float4*>(s_raw + ((sizeof(FuSmem) + 127) & ~size_t(127)));
@@ -73,9 +73,10 @@ __global__ void __launch_bounds__(kFuThreads, 2) compress_reduce_kernel(
   if (warp == kFuWarps) {  // ------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tensor_map(&tmap_x);
+      producer_start_delay(lim.start_delay);
       int issued = 0, bi = 0, r = 0;
       for (int i = 0; i < n_tiles; ++i) {
-        if (!sm.ring.acquire(i, abort, wait_limit)) break;
+        if (!sm.ring.acquire(i, abort, lim.producer)) break;
         const int st = i % kFuStages;
         mbar_arrive_expect_tx(&sm.ring.full[st], kFuTileBytes);
         tma_load_2d(&sm.tile[st][0][0], &tmap_x, hs, r * T + t_first + bi * kFuTileRows, &sm.ring.full[st]);
@@ -85,7 +86,7 @@ __global__ void __launch_bounds__(kFuThreads, 2) compress_reduce_kernel(
           ++bi;
         }
       }
-      if (*abort) sm.ring.drain(issued, wait_limit);
+      if (*abort) sm.ring.drain(issued, lim.producer);
     }
     return;
   }
@@ -135,7 +136,7 @@ __global__ void __launch_bounds__(kFuThreads, 2) compress_reduce_kernel(
       for (int e = 0; e < 8; ++e) acc[m][e] = 0.0f;
     bool ok = true;
     for (int r = 0; r < P; ++r) {
-      if (!mbar_wait(&sm.ring.full[st_i], phase, abort, wait_limit)) {
+      if (!mbar_wait(&sm.ring.full[st_i], phase, abort, lim.consumer)) {
         ok = false;
         break;
       }

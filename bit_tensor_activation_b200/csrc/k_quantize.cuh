@@ -93,7 +93,7 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
     const __grid_constant__ CUtensorMap tmap_x, const uint16_t* __restrict__ x, int P, int T, int H,
     int k, const int32_t* __restrict__ keep_idx, const int32_t* __restrict__ rest_idx,
     const float* __restrict__ inv_scale, const uint8_t* __restrict__ zero, uint32_t* __restrict__ codes,
-    uint16_t* __restrict__ side, int S, int J, long long wait_limit) {
+    uint16_t* __restrict__ side, int S, int J, WaitLimits lim) {
   extern __shared__ __align__(128) unsigned char s_raw[];
   QtSmem& sm = *reinterpret_cast<QtSmem*>(s_raw);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -117,6 +117,7 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
   if (warp == kQtWarps) {
     if (lane == 0) {
       prefetch_tensor_map(&tmap_x);
+      producer_start_delay(lim.start_delay);
       int issued = 0;
       int r = u0 / NB, b = u0 - (u0 / NB) * NB;  // unit (rank r, row block b), advanced incrementally
       for (int i = 0; i < n_units; ++i) {
@@ -124,14 +125,14 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
           b = 0;
           ++r;
         }
-        if (!sm.ring.acquire(i, abort, wait_limit)) break;
+        if (!sm.ring.acquire(i, abort, lim.producer)) break;
         const int st = i % kQtStages;
         const int row = r * T + b * kQtTileRows;
         mbar_arrive_expect_tx(&sm.ring.full[st], kQtTileBytes);
         tma_load_2d(&sm.tile[st][0][0], &tmap_x, (s * kQtSlice) / 2, row, &sm.ring.full[st]);
         ++issued;
       }
-      if (*abort) sm.ring.drain(issued, wait_limit);
+      if (*abort) sm.ring.drain(issued, lim.producer);
     }
     return;
   }
@@ -248,7 +249,7 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
         }
       }
     }
-    if (!sm.ring.wait_full(i, abort, wait_limit)) break;
+    if (!sm.ring.wait_full(i, abort, lim.consumer)) break;
     const int st = i % kQtStages;
     const int t_base = b * kQtTileRows + warp * kQtRowsPerWarp;  // this warp's first row
     const int nrows = max(0, min(kQtRowsPerWarp, T - t_base));

@@ -21,7 +21,8 @@
  * Conventions for every call:
  *   - All arrays are dense, row-major, in device memory, owned by the caller.  The library
  *     allocates nothing and keeps no state between calls (apart from one device error word, see
- *     hq_read_device_error).  bf16 values are passed as their uint16_t bit patterns.
+ *     hq_read_device_error, cached launch facts per device, and the self-test setting of
+ *     hq_selftest_set_pipeline_stall).  bf16 values are passed as their uint16_t bit patterns.
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  Every call
  *     only enqueues work on it and returns; results are ready when the stream reaches them.
  *   - Arguments are checked on the host before anything is enqueued.  On a bad argument the
@@ -155,9 +156,14 @@ hq_status hq_compress_reduce(const uint16_t* x, int P, int T, int H, int k, cons
 const char* hq_status_string(hq_status s);
 
 /*
- * Synchronises `stream`, then returns and clears the device error word of the current device:
- * HQ_OK if no kernel recorded an error since the last call, else the first recorded status
- * (HQ_ERR_BAD_INDEX, HQ_ERR_TIMEOUT).  Returns HQ_ERR_CUDA if the synchronisation fails.
+ * Returns and clears the device error word of the current device: HQ_OK if no kernel recorded
+ * an error since the last call, else the first recorded status (HQ_ERR_BAD_INDEX,
+ * HQ_ERR_TIMEOUT).  The word is device-wide: kernels on every stream record into it.  The call
+ * enqueues one single-thread kernel on `stream` that exchanges the word with 0 atomically, copies
+ * the old value back and synchronises `stream`; so work ordered before it on `stream` has been
+ * counted, and an error recorded concurrently by a kernel on another stream is counted by this
+ * call or by the next one, never lost.  Calls from several host threads are serialised.  Returns
+ * HQ_ERR_CUDA if the launch, the copy or the synchronisation fails.
  */
 hq_status hq_read_device_error(void* stream);
 
@@ -169,6 +175,22 @@ hq_status hq_read_device_error(void* stream);
  * with hq_read_device_error) and returns; the context stays usable.
  */
 hq_status hq_selftest_bounded_wait(long long limit_cycles, void* stream);
+
+/*
+ * Self-test of the pipelines' abort path (no counterpart on the page; it exists so that failure
+ * detection in the real TMA pipelines -- quantize-pack, dequant-reduce and compress-reduce -- can
+ * be tested without faulting or hanging a GPU).  After hq_selftest_set_pipeline_stall(c, d) with
+ * c > 0 and d > 0, every pipeline kernel launched by this process lets its producer lane idle for
+ * d clock cycles before its first load, and bounds its consumers' waits by c cycles instead of
+ * about a second.  With c well below d the consumers give up: the kernel records HQ_ERR_TIMEOUT,
+ * raises its abort flag, the producer issues its first loads, sees the flag, waits (on the long
+ * bound) for those loads to land, and the kernel returns with its outputs unspecified.
+ * hq_selftest_set_pipeline_stall(0, 0) restores the normal bounds.  Process-wide; not for use
+ * while other threads launch work.
+ *   consumer_limit_cycles  >= 0;  producer_delay_cycles  0 .. 2^31 (about a second)
+ * Returns HQ_ERR_INVALID_ARG if either is out of range or exactly one of them is 0.
+ */
+hq_status hq_selftest_set_pipeline_stall(long long consumer_limit_cycles, long long producer_delay_cycles);
 
 /* Bytes of the two wire buffers per rank and row: 4-bit part (H-k)/2, BF16 part 2k. */
 int64_t hq_wire_bytes_per_row(int H, int k);
