@@ -1,10 +1,11 @@
 #!/usr/bin/env python
 """Throughput of the hybrid BF16/Int4 partial-sum compression path on B200.
 
-One step is one pass of the whole path over one batch of P ranks' bf16 partial sums, resident in
-HBM: hq_calibrate (one more moving-average update), hq_select_topk, hq_quantize_pack and
-hq_dequant_reduce (``--path split``, the default) or hq_compress_reduce (``--path fused``).
-``value`` is partial-sum bytes (P*T*H*2 per step, all ranks) per second over the timed steps.
+One step is one pass of the online path over one batch of P ranks' bf16 partial sums, resident in
+HBM: hq_quantize_pack then hq_dequant_reduce (``--path split``, the default) or
+hq_compress_reduce (``--path fused``).  ``value`` is partial-sum bytes (P*T*H*2 per step, all
+ranks) per second over the timed steps.  Calibration and selection run once per calibration, not
+per batch; they are timed on their own and reported under ``offline``.
 
 Prints one JSON line.  ``--impl reference`` times the CPU oracle instead (the reference arm of
 this benchmark: a plain single-threaded C restatement of the method).  Under torchrun each rank
@@ -31,17 +32,23 @@ import synth  # noqa: E402
 
 METRIC = "partial-sum GB/s compressed+reduced (1 B200), % of HBM peak; compression ratio"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal
+L2_BYTES = 126 * 2**20
+SECOND_WORKLOAD = {"prefill70b": "prefill7b", "prefill7b": "prefill70b"}
 
 
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["hq", "reference"], default="hq")
     ap.add_argument("--path", choices=["split", "fused"], default="split")
     ap.add_argument("--workload", default="prefill70b")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cold-reps", type=int, default=20, help="launches of each kernel timed alone, L2 flushed")
+    ap.add_argument("--second-steps", type=int, default=400,
+                    help="timed steps of the second large workload (0: skip it)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-clocks", action="store_true")
@@ -184,7 +191,8 @@ def barrier(world):
 # CPU oracle timing (cpu_baseline leg and the reference arm)
 # ---------------------------------------------------------------------------------------------
 class OracleStep:
-    """The whole path on the CPU oracle over rows [0, S) of the workload's evaluation batch."""
+    """The online path on the CPU oracle over rows [0, S) of the workload's evaluation batch:
+    quantize-pack and dequant-reduce, with parameters calibrated and selected once beforehand."""
 
     def __init__(self, cfg, x_rows: np.ndarray):
         import oracle
@@ -192,14 +200,13 @@ class OracleStep:
         self.o = oracle.get()
         self.cfg = cfg
         self.x = x_rows
-        self.emin, self.emax = self.o.calibrate(x_rows, cfg.beta, True)
+        emin, emax = self.o.calibrate(x_rows, cfg.beta, True)
+        self.sel = self.o.select_topk(emin, emax, cfg.k)
 
     def run(self, S: int) -> float:
-        cfg, o = self.cfg, self.o
+        cfg, o, sel = self.cfg, self.o, self.sel
         xs = np.ascontiguousarray(self.x[:, :S])
         t0 = time.perf_counter()
-        emin, emax = o.calibrate(xs, cfg.beta, False, self.emin, self.emax)
-        sel = o.select_topk(emin, emax, cfg.k)
         codes, side = o.quantize_pack(xs, sel["keep_idx"], sel["rest_idx"], sel["inv_scale"], sel["zero"])
         o.dequant_reduce(codes, side, cfg.H, sel["keep_idx"], sel["rest_idx"], sel["scale"], sel["zero"])
         return time.perf_counter() - t0
@@ -242,14 +249,14 @@ def run_reference(args, cfg, world, rank):
     part_bytes = cfg.P * S * cfg.H * 2
     value = part_bytes * args.steps / t / 1e9
     sample = (f"rows 0..{S - 1} of the evaluation batch, all {cfg.P} ranks, per step "
-              f"(calibrate + select + quantize-pack + dequant-reduce), single thread")
+              f"(quantize-pack + dequant-reduce), single thread")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": 0,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
         "config": {"workload": describe(cfg), "P": cfg.P, "T": cfg.T, "H": cfg.H, "k": cfg.k,
-                   "path": "split", "parallelism": "replicas"},
+                   "path": "split", "step": "quantize_pack+dequant_reduce", "parallelism": "replicas"},
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "host_cpus": os.cpu_count(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -295,6 +302,131 @@ def ncu_traffic(kernel: str, workload: str):
     return None
 
 
+def _kernel_entry(nbytes, t_ms, peak):
+    gbs = nbytes / (t_ms * 1e-3) / 1e9
+    return {"us": 1e3 * t_ms, "bytes": nbytes, "GB/s": gbs, "frac": gbs / peak, "frac_nominal": gbs / NOMINAL_HBM_GBS}
+
+
+class Workload:
+    """One workload resident on the GPU: calibration state and parameters (offline), the
+    evaluation batch x, and the wire and output buffers."""
+
+    def __init__(self, cfg, dev):
+        import torch
+
+        import bit_tensor_activation_b200 as hq
+
+        self.hq, self.cfg, self.dev = hq, cfg, dev
+        P, T, H, k = cfg.P, cfg.T, cfg.H, cfg.k
+        cs, _ = synth.colscale(cfg)
+        cs_dev = torch.from_numpy(cs).to(dev)
+        self.B = hq.Buffers(P, T, H, k, device=dev)
+        self.cal = torch.empty((P, cfg.calib_T, H), dtype=torch.int16, device=dev)
+        for b in range(cfg.calib_batches):
+            synth.fill_gpu(cfg, synth.CALIB, b, self.cal, cs_dev, T=cfg.calib_T)
+            hq.hq_calibrate(self.cal, self.B.ema_min, self.B.ema_max, cfg.beta, b == 0)
+        self.select()
+        self.x = torch.empty((P, T, H), dtype=torch.int16, device=dev)
+        synth.fill_gpu(cfg, synth.EVAL, 0, self.x, cs_dev)
+        self.fused_out = torch.empty_like(self.B.out)
+        torch.cuda.synchronize()
+
+    # offline calls (once per calibration)
+    def calibrate(self):
+        self.hq.hq_calibrate(self.cal, self.B.ema_min, self.B.ema_max, self.cfg.beta, False)
+
+    def select(self):
+        B = self.B
+        self.hq.hq_select_topk(B.ema_min, B.ema_max, self.cfg.k, B.keep_idx, B.rest_idx, B.scale, B.inv_scale,
+                               B.zero)
+
+    # online calls (every batch)
+    def quantize_pack(self, xin=None):
+        B = self.B
+        self.hq.hq_quantize_pack(self.x if xin is None else xin, B.keep_idx, B.rest_idx, B.inv_scale, B.zero,
+                                 B.codes, B.side)
+
+    def dequant_reduce(self, res=None):
+        B = self.B
+        self.hq.hq_dequant_reduce(B.codes, B.side, B.keep_idx, B.rest_idx, B.scale, B.zero,
+                                  B.out if res is None else res)
+
+    def compress_reduce(self, xin=None, res=None):
+        B = self.B
+        self.hq.hq_compress_reduce(self.x if xin is None else xin, B.keep_idx, B.rest_idx, B.scale, B.inv_scale,
+                                   B.zero, self.fused_out if res is None else res)
+
+    def step_calls(self, path, xin=None, res=None):
+        if path == "split":
+            return [("quantize_pack", lambda: self.quantize_pack(xin)), ("dequant_reduce", lambda: self.dequant_reduce(res))]
+        return [("compress_reduce", lambda: self.compress_reduce(xin, res))]
+
+
+def time_steps(W: Workload, path, K, warmup, stream):
+    """K steps back to back with an event before every call: (total ms, {kernel: mean ms})."""
+    import torch
+
+    calls = W.step_calls(path)
+    for _ in range(warmup):
+        for _, c in calls:
+            c()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in calls] for _ in range(K)]
+    ev.append([torch.cuda.Event(enable_timing=True)])
+    torch.cuda.synchronize()
+    for i in range(K):
+        for j, (_, c) in enumerate(calls):
+            ev[i][j].record(stream)
+            c()
+    ev[K][0].record(stream)
+    torch.cuda.synchronize()
+    per = {}
+    for j, (n, _) in enumerate(calls):
+        nxt = (lambda i: ev[i][j + 1]) if j + 1 < len(calls) else (lambda i: ev[i + 1][0])
+        per[n] = sum(ev[i][j].elapsed_time(nxt(i)) for i in range(K)) / K
+    return ev[0][0].elapsed_time(ev[K][0]), per
+
+
+def time_cold(fns, reps, stream, flush):
+    """Each call timed alone, the L2 flushed (a write larger than L2) before every launch: mean ms."""
+    import torch
+
+    out = {}
+    for n, f in fns:
+        f()  # warm the launch path
+        tot = 0.0
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            f()
+            b.record(stream)
+            b.synchronize()
+            tot += a.elapsed_time(b)
+        out[n] = tot / reps
+    return out
+
+
+def measure_workload(W: Workload, K, warmup, cold_reps, stream, flush, peak):
+    """Split and fused steps, per-kernel times in the step and cold, offline calls cold."""
+    cfg = W.cfg
+    ab = algo_bytes(cfg)
+    part = cfg.P * cfg.T * cfg.H * 2
+    ms_s, per_s = time_steps(W, "split", K, warmup, stream)
+    ms_f, per_f = time_steps(W, "fused", max(3, K // 2), warmup, stream)
+    cold = time_cold([("quantize_pack", W.quantize_pack), ("dequant_reduce", W.dequant_reduce),
+                      ("compress_reduce", W.compress_reduce)], cold_reps, stream, flush)
+    off = time_cold([("calibrate", W.calibrate), ("select", W.select)], max(3, cold_reps // 4), stream, flush)
+    return {
+        "split_ms": ms_s / K, "fused_ms": ms_f / max(3, K // 2),
+        "value": part / (ms_s / K * 1e-3) / 1e9,
+        "fused_value": part / (ms_f / max(3, K // 2) * 1e-3) / 1e9,
+        "kernels": {n: _kernel_entry(ab[n], t, peak) for n, t in per_s.items()},
+        "fused_kernel": {n: _kernel_entry(ab[n], t, peak) for n, t in per_f.items()},
+        "kernels_cold": {n: _kernel_entry(ab[n], t, peak) for n, t in cold.items()},
+        "offline": {n: _kernel_entry(ab[n], t, peak) for n, t in off.items()},
+    }
+
+
 def run_hq(args, cfg, world, rank, local):
     import torch
 
@@ -304,116 +436,62 @@ def run_hq(args, cfg, world, rank, local):
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
     P, T, H, k = cfg.P, cfg.T, cfg.H, cfg.k
+    peak, peak_src = measured_peak()
+    ab = algo_bytes(cfg)
+    part_bytes = P * T * H * 2
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
 
-    # ---- inputs resident in HBM: calibration state, then the evaluation batch ----------------
-    cs, _ = synth.colscale(cfg)
-    cs_dev = torch.from_numpy(cs).to(dev)
-    B = hq.Buffers(P, T, H, k, device=dev)
-    cal = torch.empty((P, cfg.calib_T, H), dtype=torch.int16, device=dev)
-    for b in range(cfg.calib_batches):
-        synth.fill_gpu(cfg, synth.CALIB, b, cal, cs_dev, T=cfg.calib_T)
-        hq.hq_calibrate(cal, B.ema_min, B.ema_max, cfg.beta, b == 0)
-    del cal
-    x = torch.empty((P, T, H), dtype=torch.int16, device=dev)
-    synth.fill_gpu(cfg, synth.EVAL, 0, x, cs_dev)
-    fused_out = torch.empty_like(B.out)
-    torch.cuda.synchronize()
-
-    names = (["calibrate", "select", "quantize_pack", "dequant_reduce"] if args.path == "split"
-             else ["calibrate", "select", "compress_reduce"])
-
-    def step_calls(xin, res=None):
-        """The step's calls on input xin; the reduced result goes to res (default: the path's own
-        output buffer)."""
-        if res is None:
-            res = B.out if args.path == "split" else fused_out
-        yield lambda: hq.hq_calibrate(xin, B.ema_min, B.ema_max, cfg.beta, False)
-        yield lambda: hq.hq_select_topk(B.ema_min, B.ema_max, k, B.keep_idx, B.rest_idx, B.scale,
-                                        B.inv_scale, B.zero)
-        if args.path == "split":
-            yield lambda: hq.hq_quantize_pack(xin, B.keep_idx, B.rest_idx, B.inv_scale, B.zero, B.codes, B.side)
-            yield lambda: hq.hq_dequant_reduce(B.codes, B.side, B.keep_idx, B.rest_idx, B.scale, B.zero, res)
-        else:
-            yield lambda: hq.hq_compress_reduce(xin, B.keep_idx, B.rest_idx, B.scale, B.inv_scale, B.zero, res)
-
-    def run_steps(n, xin, events=None):
-        for i in range(n):
-            for j, call in enumerate(step_calls(xin)):
-                if events is not None:
-                    events[i][j].record(stream)
-                call()
-        if events is not None:
-            events[n][0].record(stream)
-
-    run_steps(args.warmup, x)
+    W = Workload(cfg, dev)
+    names = [n for n, _ in W.step_calls(args.path)]
+    calls = W.step_calls(args.path)
+    for _ in range(args.warmup):
+        for _, c in calls:
+            c()
     torch.cuda.synchronize()
     st = hq.hq_read_device_error()
     if st != hq.HQ_OK:
         raise RuntimeError(f"device error after warm-up: {hq.hq_status_string(st)}")
 
+    # ---- the timed steps: inputs resident in HBM, larger than L2 ------------------------------------
     K = args.steps
-    nk = len(names)
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(nk)] for _ in range(K)]
-    events.append([torch.cuda.Event(enable_timing=True)])
-    t_begin = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in calls] for _ in range(K)]
+    ev.append([torch.cuda.Event(enable_timing=True)])
     barrier(world)
     torch.cuda.synchronize()
     clocks = ClockSampler(local, not args.no_clocks)
     time.sleep(0.3 if not args.no_clocks else 0.0)
     wall0 = time.perf_counter()
-    t_begin.record(stream)
-    run_steps(K, x, events)
-    t_end.record(stream)
+    for i in range(K):
+        for j, (_, c) in enumerate(calls):
+            ev[i][j].record(stream)
+            c()
+    ev[K][0].record(stream)
     torch.cuda.synchronize()
     wall = time.perf_counter() - wall0
     clk = clocks.stop()
     barrier(world)
-
-    ms_local = t_begin.elapsed_time(t_end)
+    ms_local = ev[0][0].elapsed_time(ev[K][0])
     ms = max_over_ranks(ms_local, world, dev)
     per_kernel = {}
     for j, n in enumerate(names):
-        tot = 0.0
-        for i in range(K):
-            nxt = events[i][j + 1] if j + 1 < nk else events[i + 1][0]
-            tot += events[i][j].elapsed_time(nxt)
-        per_kernel[n] = tot / K  # ms per launch (includes the launch gap on the stream)
+        nxt = (lambda i: ev[i][j + 1]) if j + 1 < len(names) else (lambda i: ev[i + 1][0])
+        per_kernel[n] = sum(ev[i][j].elapsed_time(nxt(i)) for i in range(K)) / K  # ms per launch
 
-    # ---- alternate path, measured the same way for the record ---------------------------------
-    alt = {}
+    # ---- each kernel alone with a cold L2, the alternate path, the offline calls --------------------
+    Ka = max(3, min(K, 400))
     alt_path = "fused" if args.path == "split" else "split"
-    saved = args.path
-    args.path = alt_path
-    alt_names = (["calibrate", "select", "quantize_pack", "dequant_reduce"] if alt_path == "split"
-                 else ["calibrate", "select", "compress_reduce"])
-    Ka = max(3, min(K, 200))
-    run_steps(3, x)
-    a0 = torch.cuda.Event(enable_timing=True)
-    a1 = torch.cuda.Event(enable_timing=True)
-    aev = [[torch.cuda.Event(enable_timing=True) for _ in alt_names] for _ in range(Ka)]
-    aev.append([torch.cuda.Event(enable_timing=True)])
-    torch.cuda.synchronize()
-    a0.record(stream)
-    run_steps(Ka, x, aev)
-    a1.record(stream)
-    torch.cuda.synchronize()
-    args.path = saved
-    alt_kernels = {}
-    for j, n in enumerate(alt_names):
-        tot = sum(aev[i][j].elapsed_time(aev[i][j + 1] if j + 1 < len(alt_names) else aev[i + 1][0])
-                  for i in range(Ka))
-        alt_kernels[n] = tot / Ka
-    alt_ms = a0.elapsed_time(a1) / Ka
-    alt[alt_path] = {"ms_per_step": alt_ms, "value": P * T * H * 2 / (alt_ms * 1e-3) / 1e9,
-                     "kernel_ms": alt_kernels}
+    ms_alt, per_alt = time_steps(W, alt_path, Ka, 3, stream)
+    cold = time_cold([("quantize_pack", W.quantize_pack), ("dequant_reduce", W.dequant_reduce),
+                      ("compress_reduce", W.compress_reduce)], args.cold_reps, stream, flush)
+    offline = time_cold([("calibrate", W.calibrate), ("select", W.select)], max(3, args.cold_reps // 4), stream,
+                        flush)
+    W.select()  # the parameters the checks below use
 
-    # ---- fused output equals split output on this workload ---------------------------------------
-    hq.hq_quantize_pack(x, B.keep_idx, B.rest_idx, B.inv_scale, B.zero, B.codes, B.side)
-    hq.hq_dequant_reduce(B.codes, B.side, B.keep_idx, B.rest_idx, B.scale, B.zero, B.out)
-    hq.hq_compress_reduce(x, B.keep_idx, B.rest_idx, B.scale, B.inv_scale, B.zero, fused_out)
-    fused_equal = bool(torch.equal(B.out.view(torch.int16), fused_out.view(torch.int16)))
+    # ---- fused output equals split output on this workload -------------------------------------------
+    W.quantize_pack()
+    W.dequant_reduce()
+    W.compress_reduce()
+    fused_equal = bool(torch.equal(W.B.out.view(torch.int16), W.fused_out.view(torch.int16)))
 
     # ---- e2e: public API with pinned host buffers, copies inside the timed region ----------------
     # Every step copies its input from pinned host memory and its result back, inside the timed
@@ -422,9 +500,10 @@ def run_hq(args, cfg, world, rank, local):
     # two device input and result buffers and events ordering every reuse.
     e2e = None
     if args.e2e_steps > 0:
+        x = W.x
         xh = x.cpu().pin_memory()
         xd = [torch.empty_like(x) for _ in range(2)]
-        res = [torch.empty_like(B.out if args.path == "split" else fused_out) for _ in range(2)]
+        res = [torch.empty_like(W.B.out) for _ in range(2)]
         oh = [torch.empty(r.shape, dtype=r.dtype).pin_memory() for r in res]
         s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         in_ready = [torch.cuda.Event() for _ in range(2)]
@@ -442,7 +521,7 @@ def run_hq(args, cfg, world, rank, local):
                 stream.wait_event(in_ready[b])
                 if i >= 2:
                     stream.wait_event(copied_out[b])  # step i-2's result has left res[b]
-                for call in step_calls(xd[b], res[b]):
+                for _, call in W.step_calls(args.path, xd[b], res[b]):
                     call()
                 computed[b].record(stream)
                 with torch.cuda.stream(s_out):
@@ -464,25 +543,37 @@ def run_hq(args, cfg, world, rank, local):
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world, dev)
-        e2e = {"value": world * P * T * H * 2 / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+        e2e = {"value": world * part_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                "h2d_bytes_per_step": xh.numel() * xh.element_size(),
                "d2h_bytes_per_step": oh[0].numel() * oh[0].element_size(), "ms_per_step": e2e_ms,
                "pipelined": "next step's input copy overlaps this step's compute and result copy"}
-        # the last step's copied-back result against the same reduction of x on the parameters that
-        # step selected (calibration moves them a little every step)
-        check = torch.empty_like(res[0])
-        if args.path == "split":
-            hq.hq_quantize_pack(x, B.keep_idx, B.rest_idx, B.inv_scale, B.zero, B.codes, B.side)
-            hq.hq_dequant_reduce(B.codes, B.side, B.keep_idx, B.rest_idx, B.scale, B.zero, check)
-        else:
-            hq.hq_compress_reduce(x, B.keep_idx, B.rest_idx, B.scale, B.inv_scale, B.zero, check)
+        # the last copied-back result against the device-resident reduction of the same input
         torch.cuda.synchronize()
+        check = W.B.out if args.path == "split" else W.fused_out
         if not torch.equal(oh[(args.e2e_steps - 1) & 1].view(torch.int16).to(dev), check.view(torch.int16)):
             raise RuntimeError("the end-to-end result differs from the device-resident reduction")
+        del xh, xd, res, oh
 
     st = hq.hq_read_device_error()
     if st != hq.HQ_OK:
         raise RuntimeError(f"device error: {hq.hq_status_string(st)}")
+
+    # ---- the second large workload, same run (per-kernel figures for the bandwidth target) -------
+    workloads = {}
+    second = SECOND_WORKLOAD.get(cfg.name)
+    if second and args.second_steps > 0 and world == 1:
+        del W
+        torch.cuda.empty_cache()
+        cfg2 = workload(second)
+        W2 = Workload(cfg2, dev)
+        m = measure_workload(W2, args.second_steps, 5, args.cold_reps, stream, flush, peak)
+        m["config"] = describe(cfg2)
+        m["compression_ratio"] = compression_ratio(cfg2)
+        workloads[second] = m
+        st = hq.hq_read_device_error()
+        if st != hq.HQ_OK:
+            raise RuntimeError(f"device error ({second}): {hq.hq_status_string(st)}")
+        del W2
 
     # ---- CPU baseline (rank 0, N = 1) -----------------------------------------------------------
     cpu = None
@@ -495,42 +586,43 @@ def run_hq(args, cfg, world, rank, local):
         t += sum(step.run(S) for _ in range(reps - 1))
         cpu = {"value": reps * P * S * H * 2 / t / 1e9, "unit": "GB/s", "cores": 1, "host_cpus": os.cpu_count(),
                "kind": "oracle",
-               "sample": f"rows 0..{S - 1} of the evaluation batch, all {P} ranks, {reps} passes of calibrate + "
-                         f"select + quantize-pack + dequant-reduce, {t:.1f} s single-threaded"}
+               "sample": f"rows 0..{S - 1} of the evaluation batch, all {P} ranks, {reps} passes of quantize-pack + "
+                         f"dequant-reduce (parameters calibrated and selected once), {t:.1f} s single-threaded"}
 
     if rank != 0:
         return
-    peak, peak_src = measured_peak()
-    ab = algo_bytes(cfg)
-    kernels = {}
-    for n, t_ms in per_kernel.items():
-        gbs = ab[n] / (t_ms * 1e-3) / 1e9
-        kernels[n] = {"us": 1e3 * t_ms, "bytes": ab[n], "GB/s": gbs, "frac": gbs / peak}
+    kernels = {n: _kernel_entry(ab[n], t_ms, peak) for n, t_ms in per_kernel.items()}
     dominant = max(per_kernel, key=per_kernel.get)
     dom_gbs = kernels[dominant]["GB/s"]
     step_bytes = sum(ab[n] for n in names)
-    part_bytes = P * T * H * 2
     value = world * part_bytes * K / (ms * 1e-3) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": describe(cfg), "P": P, "T": T, "H": H, "k": k, "path": args.path,
-                   "step": "+".join(names), "parallelism": "replicas" if world > 1 else "single GPU",
+                   "step": "+".join(names),
+                   "offline": "calibrate + select run once per calibration; timed alone under 'offline'",
+                   "parallelism": "replicas" if world > 1 else "single GPU",
                    "l2": f"inputs larger than L2 ({part_bytes / 2**20:.0f} MiB of partial sums per step), no flush"
-                   if part_bytes > 126e6 else "inputs smaller than L2 (L2-resident between steps)"},
+                   if part_bytes > L2_BYTES else "inputs smaller than L2 (L2-resident between steps)"},
         "hbm_frac_step": step_bytes * K / (ms_local * 1e-3) / 1e9 / peak,
         "compression_ratio": compression_ratio(cfg),
         "elements_per_s": world * P * T * H * K / (ms * 1e-3),
         "roofline": {"bound": "hbm", "kernel": dominant, "achieved": dom_gbs, "peak": peak, "unit": "GB/s",
                      "frac": dom_gbs / peak, "traffic": ncu_traffic(dominant, cfg.name), "peak_source": peak_src,
-                     "bytes_per_launch": ab[dominant]},
+                     "bytes_per_launch": ab[dominant], "frac_nominal": dom_gbs / NOMINAL_HBM_GBS,
+                     "nominal_peak": NOMINAL_HBM_GBS},
         "kernels": kernels,
-        "alt_paths": alt,
+        "kernels_cold": {n: _kernel_entry(ab[n], t_ms, peak) for n, t_ms in cold.items()},
+        "offline": {n: _kernel_entry(ab[n], t_ms, peak) for n, t_ms in offline.items()},
+        "alt_paths": {alt_path: {"ms_per_step": ms_alt / Ka, "value": part_bytes / (ms_alt / Ka * 1e-3) / 1e9,
+                                 "kernel_ms": per_alt}},
+        "workloads": workloads,
         "fused_equals_split": fused_equal,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": (len(names) + (1 if "select" in names else 0)) * K,
+        "gpu_launches": len(names) * K,
         "clocks": clk,
         "wall_s_timed": wall,
     }

@@ -3,8 +3,9 @@
 Integer and index results (codes, zero points, keep/rest sets, side buffers) and the fp32 results
 (moving averages, scales, reduced outputs) must all be bit-identical: both sides evaluate the same
 sequence of correctly rounded fp32 operations, and the reduction order over ranks is fixed.
-Small and mid-size problems are compared element by element; the two full-size workloads
-(prefill 7B and 70B shapes) on sampled rows and columns the oracle computes one by one.
+Small and mid-size problems are compared element by element; so are the whole wire buffers and
+outputs of the two full-size workloads (prefill 7B and 70B shapes), whose 32-batch calibration is
+compared on sampled columns the oracle computes one by one.
 """
 import numpy as np
 import pytest
@@ -288,41 +289,48 @@ def test_full_size_calibration_sampled(name):
 
 
 @pytest.mark.parametrize("name", ["prefill7b", "prefill70b"])
-def test_full_size_select_quantize_reduce_sampled(name):
+def test_full_size_select_quantize_reduce_whole_tensors(name):
+    """The full-size evaluation batch, in the launch configuration the benchmark times: selection,
+    then the whole codes and side buffers and the whole bf16 output of the split path, the fused
+    path (with and without its wire outputs) and the bf16-shard reduction, each compared with the
+    oracle element by element over all T rows.  The host regenerates the batch with the same
+    counter-based generator; the parameters come from the oracle (a shorter calibration: any
+    statistics serve as selection input)."""
     cfg = synth.CONFIGS[name]
     o = oracle.get()
     cs, outl = synth.colscale(cfg)
-    # statistics from a reduced calibration on the host (any statistics serve as select input)
     cal = _batches(cfg.with_(calib_batches=4), cs, T=48)
     emin, emax = o.calibrate_batches(cal, cfg.beta)
     sel = o.select_topk(emin, emax, cfg.k)
     B = gpu_select(torch.from_numpy(emin).to(DEV), torch.from_numpy(emax).to(DEV), cfg.k)
-    assert np.array_equal(B["keep_idx"].cpu().numpy(), sel["keep_idx"])
-    assert np.array_equal(B["rest_idx"].cpu().numpy(), sel["rest_idx"])
-    assert np.array_equal(f32bits(B["scale"]), f32bits(sel["scale"]))
-    assert np.array_equal(f32bits(B["inv_scale"]), f32bits(sel["inv_scale"]))
-    assert np.array_equal(B["zero"].cpu().numpy(), sel["zero"])
+    assert_same(B["keep_idx"].cpu().numpy(), sel["keep_idx"], "keep_idx")
+    assert_same(B["rest_idx"].cpu().numpy(), sel["rest_idx"], "rest_idx")
+    assert_same(f32bits(B["scale"]), f32bits(sel["scale"]), "scale")
+    assert_same(f32bits(B["inv_scale"]), f32bits(sel["inv_scale"]), "inv_scale")
+    assert_same(B["zero"].cpu().numpy(), sel["zero"], "zero")
     prm = params_to_dev(sel)
     x = _gpu_batch(cfg, synth.EVAL, 0, torch.from_numpy(cs).to(DEV))
     codes, side = gpu_quantize(x, prm)
     out = gpu_dequant(codes, side, prm, cfg.H)
     lit = gpu_dequant(codes, side, prm, cfg.H, bf16_shards=True)
     fused, _, _ = gpu_fused(x, prm)
+    fused_w, wcodes, wside = gpu_fused(x, prm, wire=True)
     assert_no_device_error()
-    assert torch.equal(out, fused), "fused == split over the whole output"
-    rng = np.random.default_rng(23)
-    rows = np.unique(np.concatenate([[0, cfg.T - 1], rng.integers(0, cfg.T, 10)]))
-    codes_h, side_h, out_h, lit_h = u32(codes), u16(side), u16(out), u16(lit)
-    for t in rows:
-        xr = synth.fill_cpu(cfg, synth.EVAL, 0, rows=(int(t), int(t) + 1), cs=cs)
-        c_r, s_r = o.quantize_pack(xr, sel["keep_idx"], sel["rest_idx"], sel["inv_scale"], sel["zero"])
-        o_r = o.dequant_reduce(c_r, s_r, cfg.H, sel["keep_idx"], sel["rest_idx"], sel["scale"], sel["zero"])
-        l_r = o.dequant_reduce(c_r, s_r, cfg.H, sel["keep_idx"], sel["rest_idx"], sel["scale"], sel["zero"],
-                               bf16_shards=True)
-        assert np.array_equal(codes_h[:, t:t + 1], c_r), f"codes row {t}"
-        assert np.array_equal(side_h[:, :, t:t + 1], s_r), f"side row {t}"
-        assert np.array_equal(out_h[t:t + 1], o_r), f"out row {t}"
-        assert np.array_equal(lit_h[t:t + 1], l_r), f"bf16-shard reduction row {t}"
+    del x
+    xh = synth.fill_cpu(cfg, synth.EVAL, 0, cs=cs)
+    c_r, s_r = o.quantize_pack(xh, sel["keep_idx"], sel["rest_idx"], sel["inv_scale"], sel["zero"])
+    del xh
+    assert_same(u32(codes), c_r, "codes")
+    assert_same(u16(side), s_r, "side")
+    assert_same(u32(wcodes), c_r, "fused wire codes")
+    assert_same(u16(wside), s_r, "fused wire side")
+    o_r = o.dequant_reduce(c_r, s_r, cfg.H, sel["keep_idx"], sel["rest_idx"], sel["scale"], sel["zero"])
+    assert_same(u16(out), o_r, "out bf16")
+    assert_same(u16(fused), o_r, "fused bf16")
+    assert_same(u16(fused_w), o_r, "fused bf16 (wire written too)")
+    l_r = o.dequant_reduce(c_r, s_r, cfg.H, sel["keep_idx"], sel["rest_idx"], sel["scale"], sel["zero"],
+                           bf16_shards=True)
+    assert_same(u16(lit), l_r, "bf16-shard reduction")
 
 
 # ---------------------------------------------------------------------------------------------
