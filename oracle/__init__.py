@@ -62,6 +62,8 @@ class Oracle:
         lib.hq_ref_dequant_reduce_bf16_shards.restype = None
         lib.hq_ref_compress_reduce.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, i32, vp, vp]
         lib.hq_ref_compress_reduce.restype = i32
+        lib.hq_ref_partial_sync.argtypes = [vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp]
+        lib.hq_ref_partial_sync.restype = i32
         lib.hq_ref_bf16_round.argtypes = [f32]
         lib.hq_ref_bf16_round.restype = ctypes.c_uint16
         lib.hq_ref_quantize_one.argtypes = [f32, f32, ctypes.c_uint]
@@ -158,6 +160,20 @@ class Oracle:
         if rc != 0:
             raise MemoryError("hq_ref_compress_reduce failed")
         return out
+
+    def partial_sync(self, x, c0, Hs, keep_idx, rest_idx, scale, inv_scale, zero):
+        """R20: every rank's output [P, T, H]: the reduced block [c0, c0 + Hs) (bf16), its own
+        partial sum elsewhere.  keep/rest index the block; scale/inv_scale/zero are [P, Hs]."""
+        x = _c(x, np.uint16)
+        P, T, H = x.shape
+        k = len(keep_idx)
+        keep, rest = _c(keep_idx, np.int32), _c(rest_idx, np.int32)
+        scale, inv, zero = _c(scale, np.float32), _c(inv_scale, np.float32), _c(zero, np.uint8)
+        y = np.empty_like(x)
+        if self.lib.hq_ref_partial_sync(_p(x), P, T, H, c0, Hs, k, _p(keep), _p(rest), _p(scale), _p(inv),
+                                        _p(zero), _p(y)) != 0:
+            raise ValueError("hq_ref_partial_sync failed")
+        return y
 
     def bf16_round(self, f: float) -> int:
         return int(self.lib.hq_ref_bf16_round(f))

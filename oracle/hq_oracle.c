@@ -41,6 +41,9 @@
  *       rounded to bf16 (nearest, ties to even) before the rank-ordered fp32 sum:
  *       acc = +0; for r = 0..P-1: acc = acc + bf16(v_r).  Kept columns and the output
  *       rounding are as in R10 and R11.
+ *   R20 partial-channel synchronisation: only the block of features [c0, c0 + Hs) goes through
+ *       the hybrid wire and the rank-ordered sum; every rank keeps its own partial sum in the
+ *       other features.
  * Calibration detail: batch min/max ignore NaN (no comparison with NaN is true); a batch
  * minimum or maximum of -0 is stored as +0 (adding +0.0f), so that results do not depend
  * on which zero a comparison happened to keep.
@@ -323,6 +326,48 @@ int hq_ref_compress_reduce(const uint16_t* x, int P, int T, int H, int k, const 
   }
   if (c != codes) free(c);
   if (s != side) free(s);
+  return rc;
+}
+
+/*
+ * Partial-channel synchronisation (the abstract of "Communication-Aware Architecture for
+ * Tensor-parallelism" (CAAT-Net) on the first page: tensor-parallel ranks can do without
+ * synchronising every activation channel), with the synchronised channels sent through the hybrid
+ * wire.  Reading R20: the synchronised features are the block [c0, c0 + Hs) of consecutive
+ * features; the block alone is quantize-packed (R6, R7) and reduced (R9-R11, bf16 output), and
+ * every rank keeps its own partial sum in the other features:
+ *   y[r][t][h] = reduced block value at h - c0   for c0 <= h < c0 + Hs
+ *   y[r][t][h] = x[r][t][h]                      otherwise
+ * keep_idx / rest_idx index the block (0 .. Hs-1); scale, inv_scale, zero are [P][Hs].
+ * Returns 0, or 1 on bad arguments / allocation failure.
+ */
+int hq_ref_partial_sync(const uint16_t* x, int P, int T, int H, int c0, int Hs, int k, const int32_t* keep_idx,
+                        const int32_t* rest_idx, const float* scale, const float* inv_scale, const uint8_t* zero,
+                        uint16_t* y) {
+  if (c0 < 0 || Hs < 0 || c0 + Hs > H || k < 0 || k > Hs) return 1;
+  const size_t rows = (size_t)P * T;
+  for (size_t i = 0; i < rows * (size_t)H; ++i) y[i] = x[i];
+  if (Hs == 0 || T == 0) return 0;
+  uint16_t* xb = (uint16_t*)malloc(sizeof(uint16_t) * rows * (size_t)Hs);
+  uint32_t* codes = (uint32_t*)malloc(sizeof(uint32_t) * (rows * (size_t)(Hs - k) / 8 + 1));
+  uint16_t* side = (uint16_t*)malloc(sizeof(uint16_t) * (rows * (size_t)k + 1));
+  uint16_t* red = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)T * Hs);
+  int rc = 0;
+  if (!xb || !codes || !side || !red) {
+    rc = 1;
+  } else {
+    for (size_t i = 0; i < rows; ++i)
+      for (int h = 0; h < Hs; ++h) xb[i * Hs + h] = x[i * H + c0 + h];
+    hq_ref_quantize_pack(xb, P, T, Hs, k, keep_idx, rest_idx, inv_scale, zero, codes, side);
+    hq_ref_dequant_reduce(codes, side, P, T, Hs, k, keep_idx, rest_idx, scale, zero, red, 0);
+    for (int r = 0; r < P; ++r)
+      for (int t = 0; t < T; ++t)
+        for (int h = 0; h < Hs; ++h) y[((size_t)r * T + t) * H + c0 + h] = red[(size_t)t * Hs + h];
+  }
+  free(xb);
+  free(codes);
+  free(side);
+  free(red);
   return rc;
 }
 

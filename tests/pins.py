@@ -590,6 +590,59 @@ def pin_bf16_shards_rounding_bound(o):
     assert off_grid.sum() > 100 and (err[off_grid] > 0).all(), "shards were not rounded"
 
 
+# ---------------------------------------------------------------------------------------------
+# Partial-channel synchronisation (reading R20)
+# ---------------------------------------------------------------------------------------------
+def pin_partial_sync_golden(o):
+    """A case worked by hand (tests/golden/partial_sync_example.json): the block's grid-point
+    values sum exactly, with and without the block kept in bf16; outside the block every rank
+    keeps its own input."""
+    g = _golden("partial_sync_example.json")
+    P, H, c0, Hs = g["P"], g["H"], g["c0"], g["Hs"]
+    x = f32_to_bf16_torch(np.array(g["x"], np.float32)).reshape(P, 1, H)
+    assert np.array_equal(bf16_to_f32(x).reshape(P, H), np.array(g["x"], np.float32))
+    for k in g["k_cases"]:
+        keep = np.arange(k, dtype=np.int32)
+        rest = np.arange(k, Hs, dtype=np.int32)
+        y = o.partial_sync(x, c0, Hs, keep, rest, np.full((P, Hs), g["scale"], np.float32),
+                           np.full((P, Hs), g["inv_scale"], np.float32), np.full((P, Hs), g["zero"], np.uint8))
+        assert bf16_to_f32(y).reshape(P, H).tolist() == g["expect_y"], f"k={k}: {bf16_to_f32(y).reshape(P, H)}"
+
+
+def pin_partial_sync_extremes(o):
+    """Hs = H is the whole path (every rank gets the reduced tensor); Hs = 0 leaves every rank
+    its own partial sum; outside any block each rank's output is its input, bit for bit, and
+    values outside the block do not change the block's result."""
+    rng = _rng(51)
+    P, T, H, k = 3, 5, 64, 8
+    x = _bf16_values(rng, P * T * H, 2.0).reshape(P, T, H)
+    emin, emax = o.calibrate(x, 0.9, True)
+    sel = o.select_topk(emin, emax, k)
+    full = o.compress_reduce(x, sel["keep_idx"], sel["rest_idx"], sel["scale"], sel["inv_scale"], sel["zero"])
+    y = o.partial_sync(x, 0, H, sel["keep_idx"], sel["rest_idx"], sel["scale"], sel["inv_scale"], sel["zero"])
+    for r in range(P):
+        assert np.array_equal(y[r], full), f"Hs = H, rank {r}"
+    y0 = o.partial_sync(x, 8, 0, np.zeros(0, np.int32), np.zeros(0, np.int32), np.zeros((P, 0), np.float32),
+                        np.zeros((P, 0), np.float32), np.zeros((P, 0), np.uint8))
+    assert np.array_equal(y0, x), "Hs = 0"
+    c0, Hs = 16, 32
+    xb = np.ascontiguousarray(x[:, :, c0:c0 + Hs])
+    eb_min, eb_max = o.calibrate(xb, 0.9, True)
+    sb = o.select_topk(eb_min, eb_max, k)
+    args = (sb["keep_idx"], sb["rest_idx"], sb["scale"], sb["inv_scale"], sb["zero"])
+    yb = o.partial_sync(x, c0, Hs, *args)
+    blk = o.compress_reduce(xb, *args[:2], sb["scale"], sb["inv_scale"], sb["zero"])
+    outside = np.ones(H, bool)
+    outside[c0:c0 + Hs] = False
+    assert np.array_equal(yb[:, :, outside], x[:, :, outside]), "outside the block"
+    for r in range(P):
+        assert np.array_equal(yb[r, :, c0:c0 + Hs], blk), f"block, rank {r}"
+    x2 = x.copy()
+    x2[:, :, outside] = _bf16_values(rng, int(outside.sum()) * P * T, 5.0).reshape(P, T, -1)
+    yb2 = o.partial_sync(x2, c0, Hs, *args)
+    assert np.array_equal(yb2[:, :, c0:c0 + Hs], yb[:, :, c0:c0 + Hs]), "the block depends on values outside it"
+
+
 ALL_PINS = [
     pin_bf16_round, pin_quantize_golden, pin_quantize_nearest_grid, pin_params_golden,
     pin_params_closed_form, pin_calibrate_single_batch, pin_calibrate_ema, pin_calibrate_ema_golden,
@@ -597,4 +650,5 @@ ALL_PINS = [
     pin_reduce_all_kept, pin_nan_outputs, pin_reduce_dequant_sum, pin_reduce_order_golden, pin_reduce_error_bound,
     pin_irwin_hall, pin_outliers_selected,
     pin_selection_benefit, pin_bf16_shards_golden, pin_bf16_shards_exact_products, pin_bf16_shards_rounding_bound,
+    pin_partial_sync_golden, pin_partial_sync_extremes,
 ]

@@ -74,6 +74,13 @@ MUTANTS = [
      "ema_max[i] = (float)((double)beta * ema_max[i] + (double)one_minus_beta * bmax);"),
     ("inv_scale_15_over_range", "float inv = 1.0f / s;", "float inv = 15.0f / rg;"),
     ("scale_times_reciprocal", "float s = rg / 15.0f;", "float s = rg * (1.0f / 15.0f);"),
+    # partial-channel synchronisation (R20)
+    ("partial_sync_block_shifted", "y[((size_t)r * T + t) * H + c0 + h] = red[(size_t)t * Hs + h];",
+     "y[((size_t)r * T + t) * H + (c0 + h + 1) % H] = red[(size_t)t * Hs + h];"),
+    ("partial_sync_outside_zeroed", "for (size_t i = 0; i < rows * (size_t)H; ++i) y[i] = x[i];",
+     "for (size_t i = 0; i < rows * (size_t)H; ++i) y[i] = 0;"),
+    ("partial_sync_rank0_outside", "for (size_t i = 0; i < rows * (size_t)H; ++i) y[i] = x[i];",
+     "for (size_t i = 0; i < rows * (size_t)H; ++i) y[i] = x[i % ((size_t)T * H)];"),
 ]
 
 
