@@ -43,6 +43,15 @@ _lib.hq_status_string.argtypes = [_i32]
 _lib.hq_status_string.restype = ctypes.c_char_p
 _lib.hq_selftest_bounded_wait.argtypes = [ctypes.c_longlong, _vp]
 _lib.hq_selftest_bounded_wait.restype = _i32
+_lib.hq_dequant_reduce_ranks.argtypes = [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _i32, _vp]
+_lib.hq_dequant_reduce_ranks.restype = _i32
+_lib.hq_calibrate_ld.argtypes = [_vp, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp]
+_lib.hq_quantize_pack_ld.argtypes = [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+_lib.hq_dequant_reduce_ld.argtypes = [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp]
+_lib.hq_compress_reduce_ld.argtypes = [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32,
+                                       _vp, _vp, _vp]
+for _f in ("hq_calibrate_ld", "hq_quantize_pack_ld", "hq_dequant_reduce_ld", "hq_compress_reduce_ld"):
+    getattr(_lib, _f).restype = _i32
 _lib.hq_selftest_set_pipeline_stall.argtypes = [ctypes.c_longlong, ctypes.c_longlong]
 _lib.hq_selftest_set_pipeline_stall.restype = _i32
 _lib.hq_wire_bytes_per_row.argtypes = [_i32, _i32]
@@ -53,7 +62,8 @@ HQ_OUT_BF16, HQ_OUT_F32 = 0, 1
 
 EXPORTS = ["hq_calibrate", "hq_select_topk", "hq_quantize_pack", "hq_dequant_reduce",
            "hq_dequant_reduce_bf16_shards", "hq_compress_reduce", "hq_status_string", "hq_read_device_error", "hq_wire_bytes_per_row",
-           "hq_selftest_bounded_wait", "hq_selftest_set_pipeline_stall"]
+           "hq_selftest_bounded_wait", "hq_selftest_set_pipeline_stall", "hq_calibrate_ld", "hq_quantize_pack_ld",
+           "hq_dequant_reduce_ld", "hq_compress_reduce_ld", "hq_dequant_reduce_ranks"]
 
 
 class HQError(RuntimeError):
@@ -95,6 +105,22 @@ def _ptr(t, dtypes, shape, name):
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     return t.data_ptr() if t.numel() else None
+
+
+def _ptr_rows(t, dtypes, shape, name):
+    """(pointer, row pitch in elements) of a view whose rows are dense but may be further apart
+    than their width, e.g. x[:, :, c0:c0 + Hs] of a contiguous [P, T, ld] tensor."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name}: dtype {t.dtype} not in {dtypes}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    st = t.stride()
+    ld = st[-2]
+    if st[-1] != 1 or (t.dim() == 3 and t.shape[0] > 1 and st[0] != t.shape[1] * ld):
+        raise ValueError(f"{name}: rows must be dense, ld apart, and the ranks' rows back to back")
+    return (t.data_ptr() if t.numel() else None), ld
 
 
 _BF16 = (torch.bfloat16, torch.int16, torch.uint16)
@@ -173,6 +199,77 @@ def hq_compress_reduce(x, keep_idx, rest_idx, scale, inv_scale, zero, out, codes
             _ptr(codes, _CODES, (P, T, (H - k) // 8), "codes"), _ptr(side, _BF16, (P, k, T), "side"),
             _stream(stream, x.device))
     _check(_lib.hq_compress_reduce(*args), "hq_compress_reduce")
+
+
+def hq_dequant_reduce_ranks(codes, side, keep_idx, rest_idx, scale, zero, out, stream=None) -> None:
+    """The reduction over P separate wire buffers: codes is a list of P [T, (H-k)/8] int32 tensors,
+    side a list of P [k, T] bf16 tensors (each may live on another GPU this process can read)."""
+    P = len(codes)
+    T, W = codes[0].shape
+    k = keep_idx.shape[0]
+    H = out.shape[1]
+    if W != (H - k) // 8 or len(side) != P:
+        raise ValueError("codes width, H, k and the number of side buffers must agree")
+    cptr = (ctypes.c_void_p * P)(*[_ptr(c, _CODES, (T, W), f"codes[{r}]") for r, c in enumerate(codes)])
+    sptr = (ctypes.c_void_p * P)(*[_ptr(s_, _BF16, (k, T), f"side[{r}]") for r, s_ in enumerate(side)])
+    odt = HQ_OUT_F32 if out.dtype == torch.float32 else HQ_OUT_BF16
+    args = (ctypes.cast(cptr, _vp), ctypes.cast(sptr, _vp) if k else None, P, T, H, k,
+            _ptr(keep_idx, _I32, (k,), "keep_idx"), _ptr(rest_idx, _I32, (H - k,), "rest_idx"),
+            _ptr(scale, _F32, (P, H), "scale"), _ptr(zero, _U8, (P, H), "zero"),
+            _ptr(out, _BF16 + _F32, (T, H), "out"), odt, _stream(stream, out.device))
+    _check(_lib.hq_dequant_reduce_ranks(*args), "hq_dequant_reduce_ranks")
+
+
+# -- partial-channel synchronisation: the same calls on a block of features [c0, c0 + Hs) -------
+# Pass column views: x[:, :, c0:c0 + Hs] of a contiguous [P, T, ld] tensor, out[:, c0:c0 + Hs] of a
+# contiguous [T, ld] tensor.  Only the block's columns of out are written.
+def hq_calibrate_ld(x, ema_min, ema_max, beta: float, first_batch: bool, stream=None) -> None:
+    P, T, H = x.shape
+    px, ldx = _ptr_rows(x, _BF16, (P, T, H), "x")
+    args = (px, ldx, P, T, H, float(beta), int(bool(first_batch)), _ptr(ema_min, _F32, (P, H), "ema_min"),
+            _ptr(ema_max, _F32, (P, H), "ema_max"), _stream(stream, x.device))
+    _check(_lib.hq_calibrate_ld(*args), "hq_calibrate_ld")
+
+
+def hq_quantize_pack_ld(x, keep_idx, rest_idx, inv_scale, zero, codes, side, stream=None) -> None:
+    P, T, H = x.shape
+    k = keep_idx.shape[0]
+    px, ldx = _ptr_rows(x, _BF16, (P, T, H), "x")
+    args = (px, ldx, P, T, H, k, _ptr(keep_idx, _I32, (k,), "keep_idx"), _ptr(rest_idx, _I32, (H - k,), "rest_idx"),
+            _ptr(inv_scale, _F32, (P, H), "inv_scale"), _ptr(zero, _U8, (P, H), "zero"),
+            _ptr(codes, _CODES, (P, T, (H - k) // 8), "codes"), _ptr(side, _BF16, (P, k, T), "side"),
+            _stream(stream, x.device))
+    _check(_lib.hq_quantize_pack_ld(*args), "hq_quantize_pack_ld")
+
+
+def hq_dequant_reduce_ld(codes, side, keep_idx, rest_idx, scale, zero, out, stream=None) -> None:
+    P, T, W = codes.shape
+    k = keep_idx.shape[0]
+    H = out.shape[1]
+    if W != (H - k) // 8:
+        raise ValueError("codes width does not match the block width and k")
+    odt = HQ_OUT_F32 if out.dtype == torch.float32 else HQ_OUT_BF16
+    po, ldo = _ptr_rows(out, _BF16 + _F32, (T, H), "out")
+    args = (_ptr(codes, _CODES, (P, T, W), "codes"), _ptr(side, _BF16, (P, k, T), "side"), P, T, H, k,
+            _ptr(keep_idx, _I32, (k,), "keep_idx"), _ptr(rest_idx, _I32, (H - k,), "rest_idx"),
+            _ptr(scale, _F32, (P, H), "scale"), _ptr(zero, _U8, (P, H), "zero"), po, ldo, odt,
+            _stream(stream, codes.device))
+    _check(_lib.hq_dequant_reduce_ld(*args), "hq_dequant_reduce_ld")
+
+
+def hq_compress_reduce_ld(x, keep_idx, rest_idx, scale, inv_scale, zero, out, codes=None, side=None,
+                          stream=None) -> None:
+    P, T, H = x.shape
+    k = keep_idx.shape[0]
+    odt = HQ_OUT_F32 if out.dtype == torch.float32 else HQ_OUT_BF16
+    px, ldx = _ptr_rows(x, _BF16, (P, T, H), "x")
+    po, ldo = _ptr_rows(out, _BF16 + _F32, (T, H), "out")
+    args = (px, ldx, P, T, H, k, _ptr(keep_idx, _I32, (k,), "keep_idx"), _ptr(rest_idx, _I32, (H - k,), "rest_idx"),
+            _ptr(scale, _F32, (P, H), "scale"), _ptr(inv_scale, _F32, (P, H), "inv_scale"),
+            _ptr(zero, _U8, (P, H), "zero"), po, ldo, odt,
+            _ptr(codes, _CODES, (P, T, (H - k) // 8), "codes"), _ptr(side, _BF16, (P, k, T), "side"),
+            _stream(stream, x.device))
+    _check(_lib.hq_compress_reduce_ld(*args), "hq_compress_reduce_ld")
 
 
 def hq_selftest_bounded_wait(limit_cycles: int, stream=None, device=None) -> None:

@@ -9,6 +9,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <cstring>
 #include <type_traits>
 #include <mutex>
 
@@ -71,14 +72,14 @@ bool get_encode() {
   return true;
 }
 
-// Row-major 2-D tensor [rows][cols] of `elem`-byte elements (row pitch cols*elem bytes, a
-// multiple of 16) read in boxes of box_rows x box_cols; out-of-range box elements read as 0.
+// Row-major 2-D tensor [rows][cols] of `elem`-byte elements (row pitch `pitch` bytes, cols*elem
+// when 0; a multiple of 16) read in boxes of box_rows x box_cols; out-of-range box elements read as 0.
 bool encode_2d(CUtensorMap* map, const void* base, CUtensorMapDataType type, size_t elem, uint64_t cols,
                uint64_t rows, uint32_t box_cols, uint32_t box_rows,
-               CUtensorMapL2promotion promo = CU_TENSOR_MAP_L2_PROMOTION_L2_256B) {
+               CUtensorMapL2promotion promo = CU_TENSOR_MAP_L2_PROMOTION_L2_256B, uint64_t pitch = 0) {
   if (!get_encode()) return false;
   cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * elem};
+  cuuint64_t strides[1] = {pitch ? pitch : cols * elem};
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
   return g_encode(map, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -153,22 +154,46 @@ void slice_chunks(int T, int S, long long resident, int rows_per_block, int* chu
   *chunks = (int)ceil_div(T, rpc);
 }
 
+// Where dequant-reduce reads the P ranks' wires: one stacked buffer [P][T][W] / [P][k][T], or one
+// buffer per rank (host arrays of P device pointers; each may be a peer GPU's memory).
+struct WireSrc {
+  const uint32_t* codes = nullptr;
+  const uint16_t* side = nullptr;
+  const uint32_t* const* codes_r = nullptr;
+  const uint16_t* const* side_r = nullptr;
+  bool per_rank = false;
+};
+
 template <typename OutT, bool kShard>
-hq_status launch_dequant(const uint32_t* codes, const uint16_t* side, int P, int T, int H, int k,
-                         const int32_t* keep_idx, const float* scale, const uint8_t* zero, void* out,
-                         cudaStream_t st, DeviceInfo& d) {
+hq_status launch_dequant(const WireSrc& src, int P, int T, int H, int k, const int32_t* keep_idx, const float* scale,
+                         const uint8_t* zero, void* out, int ldo, cudaStream_t st, DeviceInfo& d) {
   const int S = (H + 8 * hq::kDqSliceGroups - 1) / (8 * hq::kDqSliceGroups);
   const int Wr = (H - k) / 8;
-  CUtensorMap map, map_side;
-  const bool tma = Wr >= 4 && Wr % 4 == 0 && aligned(codes, 16) &&
-                   encode_2d(&map, codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)Wr, (uint64_t)P * T,
-                             hq::kDtWords, hq::kDtTileRows);
-  // side[r][j][t] as [P*k][T]: boxes of 32 rows (inner) x 32 kept features; needs rows of a
+  hq::DqWire wire;
+  memset(&wire, 0, sizeof wire);
+  wire.per_rank = src.per_rank ? 1 : 0;
+  bool tma = Wr >= 4 && Wr % 4 == 0;
+  // side[r][j][t] as [k][T] rows: boxes of 32 rows (inner) x 32 kept features; needs rows of a
   // multiple of 16 bytes (T % 8 == 0), else the kept sums read the side buffer directly
-  const bool side_tma = tma && k > 0 && T % 8 == 0 &&
-                        encode_2d(&map_side, side, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)T, (uint64_t)P * k,
-                                  hq::kDtTileRows, hq::kDtSideCols, CU_TENSOR_MAP_L2_PROMOTION_NONE);
-  if (!side_tma) map_side = map;  // never read
+  bool side_tma = k > 0 && T % 8 == 0;
+  if (!src.per_rank) {
+    tma = tma && aligned(src.codes, 16) &&
+          encode_2d(&wire.code[0], src.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)Wr, (uint64_t)P * T,
+                    hq::kDtWords, hq::kDtTileRows);
+    side_tma = tma && side_tma &&
+               encode_2d(&wire.side[0], src.side, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)T, (uint64_t)P * k,
+                         hq::kDtTileRows, hq::kDtSideCols, CU_TENSOR_MAP_L2_PROMOTION_NONE);
+  } else {
+    for (int r = 0; r < P && tma; ++r)
+      tma = encode_2d(&wire.code[r], src.codes_r[r], CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)Wr, (uint64_t)T,
+                      hq::kDtWords, hq::kDtTileRows);
+    for (int r = 0; r < P && side_tma; ++r)
+      side_tma = encode_2d(&wire.side[r], src.side_r[r], CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)T, (uint64_t)k,
+                           hq::kDtTileRows, hq::kDtSideCols, CU_TENSOR_MAP_L2_PROMOTION_NONE);
+    for (int r = 0; r < P; ++r) wire.side_ptr[r] = k > 0 ? src.side_r[r] : nullptr;
+    if (!tma) return HQ_ERR_INVALID_ARG;  // per-rank buffers are read by the TMA kernel only
+    side_tma = side_tma && tma;
+  }
   constexpr int kF32 = std::is_same<OutT, float>::value ? 1 : 0;
   if (tma) {
     const size_t smem = hq::dt_smem_bytes(P);
@@ -177,10 +202,9 @@ hq_status launch_dequant(const uint32_t* codes, const uint16_t* side, int P, int
     if (occupancy(d.dequant_tma[kF32][kShard], kern, hq::kDtThreads, smem, P, &per_sm) != HQ_OK) return HQ_ERR_CUDA;
     int chunks, rpc;
     slice_chunks(T, S, (long long)d.sms * per_sm, hq::kDtTileRows, &chunks, &rpc);
-    kern<<<(unsigned)(S * chunks), hq::kDtThreads, smem, st>>>(map, map_side, side_tma ? 1 : 0, side, P, T, H, k,
-                                                                keep_idx, scale, zero,
-                                                                static_cast<OutT*>(out), S, chunks, rpc,
-                                                                wait_limits());
+    kern<<<(unsigned)(S * chunks), hq::kDtThreads, smem, st>>>(wire, side_tma ? 1 : 0, src.side, P, T, H, k,
+                                                                keep_idx, scale, zero, static_cast<OutT*>(out), ldo,
+                                                                S, chunks, rpc, wait_limits());
     return launched();
   }
   const size_t smem = hq::dq_smem_bytes(P);
@@ -189,19 +213,19 @@ hq_status launch_dequant(const uint32_t* codes, const uint16_t* side, int P, int
   if (occupancy(d.dequant_cp[kF32][kShard], kern, hq::kDqThreads, smem, P, &per_sm) != HQ_OK) return HQ_ERR_CUDA;
   int chunks, rpc;
   slice_chunks(T, S, (long long)d.sms * per_sm, hq::kDqR, &chunks, &rpc);
-  kern<<<(unsigned)(S * chunks), hq::kDqThreads, smem, st>>>(codes, side, P, T, H, k, keep_idx, scale,
-                                                              zero, static_cast<OutT*>(out), S, chunks, rpc);
+  kern<<<(unsigned)(S * chunks), hq::kDqThreads, smem, st>>>(src.codes, src.side, P, T, H, k, keep_idx, scale,
+                                                              zero, static_cast<OutT*>(out), ldo, S, chunks, rpc);
   return launched();
 }
 
 template <typename OutT>
-hq_status launch_fused(const uint16_t* x, int P, int T, int H, int k, const int32_t* keep_idx,
-                       const float* scale, const float* inv_scale, const uint8_t* zero, void* out,
+hq_status launch_fused(const uint16_t* x, int ldx, int P, int T, int H, int k, const int32_t* keep_idx,
+                       const float* scale, const float* inv_scale, const uint8_t* zero, void* out, int ldo,
                        cudaStream_t st, DeviceInfo& d) {
   const int S = (H + hq::kFuSlice - 1) / hq::kFuSlice;
   CUtensorMap map;
   if (!encode_2d(&map, x, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)H, (uint64_t)P * T, hq::kFuSlice,
-                 hq::kFuTileRows))
+                 hq::kFuTileRows, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, (uint64_t)ldx * 2))
     return HQ_ERR_CUDA;
   const size_t smem = hq::fu_smem_bytes(P);
   auto kern = hq::compress_reduce_kernel<OutT>;
@@ -211,7 +235,7 @@ hq_status launch_fused(const uint16_t* x, int P, int T, int H, int k, const int3
   int chunks, rpc;
   slice_chunks(T, S, (long long)d.sms * per_sm, hq::kFuTileRows, &chunks, &rpc);
   kern<<<(unsigned)(S * chunks), hq::kFuThreads, smem, st>>>(map, P, T, H, k, keep_idx, scale, inv_scale, zero,
-                                                              static_cast<OutT*>(out), S, chunks, rpc,
+                                                              static_cast<OutT*>(out), ldo, S, chunks, rpc,
                                                               wait_limits());
   return launched();
 }
@@ -233,13 +257,16 @@ __global__ void selftest_wait_kernel(long long limit) {
   hq::mbar_wait(&bar, 0, &abort, limit);
 }
 
+// A leading dimension: at least the width, and rows of a multiple of 16 bytes.
+bool ld_ok(int ld, int H) { return ld >= H && ld % 8 == 0; }
+
 // Argument checks and launch shared by the two reductions (kShard: each rank's value rounded to
-// bf16 before it is added).
+// bf16 before it is added); the output has a row pitch of ldo elements.
 template <bool kShard>
 hq_status dequant_entry(const uint32_t* codes, const uint16_t* side, int P, int T, int H, int k,
                         const int32_t* keep_idx, const int32_t* rest_idx, const float* scale,
-                        const uint8_t* zero, void* out, hq_out_dtype out_dtype, void* stream) {
-  if (check_shape(P, H, k) != HQ_OK || T < 0) return HQ_ERR_INVALID_ARG;
+                        const uint8_t* zero, void* out, int ldo, hq_out_dtype out_dtype, void* stream) {
+  if (check_shape(P, H, k) != HQ_OK || T < 0 || !ld_ok(ldo, H)) return HQ_ERR_INVALID_ARG;
   if (out_dtype != HQ_OUT_BF16 && out_dtype != HQ_OUT_F32) return HQ_ERR_INVALID_ARG;
   if (!scale || !zero) return HQ_ERR_INVALID_ARG;
   if ((k > 0 && !keep_idx) || (k < H && !rest_idx)) return HQ_ERR_INVALID_ARG;
@@ -251,9 +278,120 @@ hq_status dequant_entry(const uint32_t* codes, const uint16_t* side, int P, int 
   DeviceInfo* d = nullptr;
   if (device_info(&d) != HQ_OK) return HQ_ERR_CUDA;
   cudaStream_t st = (cudaStream_t)stream;
+  WireSrc src;
+  src.codes = codes;
+  src.side = side;
   if (out_dtype == HQ_OUT_BF16)
-    return launch_dequant<uint16_t, kShard>(codes, side, P, T, H, k, keep_idx, scale, zero, out, st, *d);
-  return launch_dequant<float, kShard>(codes, side, P, T, H, k, keep_idx, scale, zero, out, st, *d);
+    return launch_dequant<uint16_t, kShard>(src, P, T, H, k, keep_idx, scale, zero, out, ldo, st, *d);
+  return launch_dequant<float, kShard>(src, P, T, H, k, keep_idx, scale, zero, out, ldo, st, *d);
+}
+
+// The wires of the P ranks in P separate buffers (each possibly a peer GPU's memory).
+hq_status dequant_ranks_entry(const uint32_t* const* codes, const uint16_t* const* side, int P, int T, int H, int k,
+                              const int32_t* keep_idx, const int32_t* rest_idx, const float* scale,
+                              const uint8_t* zero, void* out, hq_out_dtype out_dtype, void* stream) {
+  if (check_shape(P, H, k) != HQ_OK || P > hq::kMaxRankMaps || T < 0) return HQ_ERR_INVALID_ARG;
+  if (H - k < 32 || (H - k) % 32 != 0) return HQ_ERR_INVALID_ARG;  // code rows staged by TMA
+  if (out_dtype != HQ_OUT_BF16 && out_dtype != HQ_OUT_F32) return HQ_ERR_INVALID_ARG;
+  if (!scale || !zero || !rest_idx || (k > 0 && !keep_idx)) return HQ_ERR_INVALID_ARG;
+  if (T > 0) {
+    if (!out || !codes || (k > 0 && !side)) return HQ_ERR_INVALID_ARG;
+    for (int r = 0; r < P; ++r) {
+      if (!codes[r] || (k > 0 && !side[r])) return HQ_ERR_INVALID_ARG;
+      if (!aligned(codes[r], 16) || (k > 0 && !aligned(side[r], 16))) return HQ_ERR_MISALIGNED;
+    }
+  }
+  if (!aligned(out, 16) || !aligned(scale, 16) || !aligned(zero, 16) || !aligned(keep_idx, 4) ||
+      !aligned(rest_idx, 4))
+    return HQ_ERR_MISALIGNED;
+  if (T == 0) return HQ_OK;
+  DeviceInfo* d = nullptr;
+  if (device_info(&d) != HQ_OK) return HQ_ERR_CUDA;
+  WireSrc src;
+  src.codes_r = codes;
+  src.side_r = k > 0 ? side : nullptr;
+  src.per_rank = true;
+  if (k == 0) {
+    static const uint16_t* const kNone[hq::kMaxRankMaps] = {};
+    src.side_r = kNone;
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  if (out_dtype == HQ_OUT_BF16)
+    return launch_dequant<uint16_t, false>(src, P, T, H, k, keep_idx, scale, zero, out, H, st, *d);
+  return launch_dequant<float, false>(src, P, T, H, k, keep_idx, scale, zero, out, H, st, *d);
+}
+
+hq_status calibrate_entry(const uint16_t* x, int ldx, int P, int T, int H, float beta, int first_batch,
+                          float* ema_min, float* ema_max, void* stream) {
+  if (check_shape(P, H, 0) != HQ_OK || T < 1 || !ld_ok(ldx, H)) return HQ_ERR_INVALID_ARG;
+  if (!(beta >= 0.0f && beta < 1.0f)) return HQ_ERR_INVALID_ARG;
+  if (!x || !ema_min || !ema_max) return HQ_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(ema_min, 16) || !aligned(ema_max, 16)) return HQ_ERR_MISALIGNED;
+  const float one_minus_beta = 1.0f - beta;
+  dim3 grid((unsigned)((H + hq::kCalCols - 1) / hq::kCalCols), (unsigned)P);
+  hq::calibrate_kernel<<<grid, hq::kCalThreads, 0, (cudaStream_t)stream>>>(
+      x, ldx, T, H, beta, one_minus_beta, first_batch ? 1 : 0, ema_min, ema_max);
+  return launched();
+}
+
+hq_status quantize_entry(const uint16_t* x, int ldx, int P, int T, int H, int k, const int32_t* keep_idx,
+                         const int32_t* rest_idx, const float* inv_scale, const uint8_t* zero, uint32_t* codes,
+                         uint16_t* side, void* stream) {
+  if (check_shape(P, H, k) != HQ_OK || T < 0 || !ld_ok(ldx, H)) return HQ_ERR_INVALID_ARG;
+  if (!inv_scale || !zero) return HQ_ERR_INVALID_ARG;
+  if ((k > 0 && !keep_idx) || (k < H && !rest_idx)) return HQ_ERR_INVALID_ARG;
+  if (T > 0 && (!x || (k > 0 && !side) || (k < H && !codes))) return HQ_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(side, 16) || !aligned(codes, 4) || !aligned(inv_scale, 16) ||
+      !aligned(zero, 16) || !aligned(keep_idx, 4) || !aligned(rest_idx, 4))
+    return HQ_ERR_MISALIGNED;
+  if (T == 0) return HQ_OK;
+  DeviceInfo* d = nullptr;
+  if (device_info(&d) != HQ_OK) return HQ_ERR_CUDA;
+  const int S = (H + hq::kQtSlice - 1) / hq::kQtSlice;
+  CUtensorMap map_x;  // x as 32-bit pairs of bf16: the box is 132 pairs = 264 features wide
+  if (!encode_2d(&map_x, x, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)H / 2, (uint64_t)P * T, hq::kQtBoxU32,
+                 hq::kQtTileRows, CU_TENSOR_MAP_L2_PROMOTION_NONE,  // 528-byte rows: no 256-byte over-fetch
+                 (uint64_t)ldx * 2))
+    return HQ_ERR_CUDA;
+  // J CTAs per slice, one wave; each takes a balanced contiguous range of (rank, 64-row block) units
+  const long long units = (long long)P * ceil_div(T, hq::kQtTileRows);
+  long long J = (long long)d->sms * d->qt_blocks / S;
+  if (J < 1) J = 1;
+  if (J > units) J = units;
+  hq::quantize_pack_tma_kernel<<<(unsigned)(S * J), hq::kQtThreads, sizeof(hq::QtSmem) + 128,
+                                 (cudaStream_t)stream>>>(map_x, x, ldx, P, T, H, k, keep_idx, rest_idx,
+                                                         inv_scale, zero, codes, side, S, (int)J,
+                                                         wait_limits());
+  return launched();
+}
+
+hq_status compress_entry(const uint16_t* x, int ldx, int P, int T, int H, int k, const int32_t* keep_idx,
+                         const int32_t* rest_idx, const float* scale, const float* inv_scale, const uint8_t* zero,
+                         void* out, int ldo, hq_out_dtype out_dtype, uint32_t* codes_or_null,
+                         uint16_t* side_or_null, void* stream) {
+  if (check_shape(P, H, k) != HQ_OK || T < 0 || !ld_ok(ldx, H) || !ld_ok(ldo, H)) return HQ_ERR_INVALID_ARG;
+  if (out_dtype != HQ_OUT_BF16 && out_dtype != HQ_OUT_F32) return HQ_ERR_INVALID_ARG;
+  if (!scale || !inv_scale || !zero) return HQ_ERR_INVALID_ARG;
+  if ((k > 0 && !keep_idx) || (k < H && !rest_idx)) return HQ_ERR_INVALID_ARG;
+  if (T > 0 && (!x || !out)) return HQ_ERR_INVALID_ARG;
+  const bool wire = codes_or_null || side_or_null;
+  if (T > 0 && wire && ((k > 0 && !side_or_null) || (k < H && !codes_or_null))) return HQ_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(out, 16) || !aligned(scale, 16) || !aligned(inv_scale, 16) ||
+      !aligned(zero, 16) || !aligned(keep_idx, 4) || !aligned(rest_idx, 4) ||
+      !aligned(codes_or_null, 4) || !aligned(side_or_null, 16))
+    return HQ_ERR_MISALIGNED;
+  if (T == 0) return HQ_OK;
+  DeviceInfo* d = nullptr;
+  if (device_info(&d) != HQ_OK) return HQ_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (wire) {
+    const hq_status q = quantize_entry(x, ldx, P, T, H, k, keep_idx, rest_idx, inv_scale, zero, codes_or_null,
+                                       side_or_null, stream);
+    if (q != HQ_OK) return q;
+  }
+  if (out_dtype == HQ_OUT_BF16)
+    return launch_fused<uint16_t>(x, ldx, P, T, H, k, keep_idx, scale, inv_scale, zero, out, ldo, st, *d);
+  return launch_fused<float>(x, ldx, P, T, H, k, keep_idx, scale, inv_scale, zero, out, ldo, st, *d);
 }
 
 }  // namespace
@@ -262,15 +400,12 @@ extern "C" {
 
 hq_status hq_calibrate(const uint16_t* x, int P, int T, int H, float beta, int first_batch,
                        float* ema_min, float* ema_max, void* stream) {
-  if (check_shape(P, H, 0) != HQ_OK || T < 1) return HQ_ERR_INVALID_ARG;
-  if (!(beta >= 0.0f && beta < 1.0f)) return HQ_ERR_INVALID_ARG;
-  if (!x || !ema_min || !ema_max) return HQ_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(ema_min, 16) || !aligned(ema_max, 16)) return HQ_ERR_MISALIGNED;
-  const float one_minus_beta = 1.0f - beta;
-  dim3 grid((unsigned)((H + hq::kCalCols - 1) / hq::kCalCols), (unsigned)P);
-  hq::calibrate_kernel<<<grid, hq::kCalThreads, 0, (cudaStream_t)stream>>>(
-      x, T, H, beta, one_minus_beta, first_batch ? 1 : 0, ema_min, ema_max);
-  return launched();
+  return calibrate_entry(x, H, P, T, H, beta, first_batch, ema_min, ema_max, stream);
+}
+
+hq_status hq_calibrate_ld(const uint16_t* x, int ldx, int P, int T, int H, float beta, int first_batch,
+                          float* ema_min, float* ema_max, void* stream) {
+  return calibrate_entry(x, ldx, P, T, H, beta, first_batch, ema_min, ema_max, stream);
 }
 
 hq_status hq_select_topk(const float* ema_min, const float* ema_max, int P, int H, int k,
@@ -306,72 +441,54 @@ hq_status hq_select_topk(const float* ema_min, const float* ema_max, int P, int 
 hq_status hq_quantize_pack(const uint16_t* x, int P, int T, int H, int k, const int32_t* keep_idx,
                            const int32_t* rest_idx, const float* inv_scale, const uint8_t* zero,
                            uint32_t* codes, uint16_t* side, void* stream) {
-  if (check_shape(P, H, k) != HQ_OK || T < 0) return HQ_ERR_INVALID_ARG;
-  if (!inv_scale || !zero) return HQ_ERR_INVALID_ARG;
-  if ((k > 0 && !keep_idx) || (k < H && !rest_idx)) return HQ_ERR_INVALID_ARG;
-  if (T > 0 && (!x || (k > 0 && !side) || (k < H && !codes))) return HQ_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(side, 16) || !aligned(codes, 4) || !aligned(inv_scale, 16) ||
-      !aligned(zero, 16) || !aligned(keep_idx, 4) || !aligned(rest_idx, 4))
-    return HQ_ERR_MISALIGNED;
-  if (T == 0) return HQ_OK;
-  DeviceInfo* d = nullptr;
-  if (device_info(&d) != HQ_OK) return HQ_ERR_CUDA;
-  const int S = (H + hq::kQtSlice - 1) / hq::kQtSlice;
-  CUtensorMap map_x;  // x as 32-bit pairs of bf16: the box is 132 pairs = 264 features wide
-  if (!encode_2d(&map_x, x, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)H / 2, (uint64_t)P * T, hq::kQtBoxU32,
-                 hq::kQtTileRows, CU_TENSOR_MAP_L2_PROMOTION_NONE))  // 528-byte rows: no 256-byte over-fetch
-    return HQ_ERR_CUDA;
-  // J CTAs per slice, one wave; each takes a balanced contiguous range of (rank, 64-row block) units
-  const long long units = (long long)P * ceil_div(T, hq::kQtTileRows);
-  long long J = (long long)d->sms * d->qt_blocks / S;
-  if (J < 1) J = 1;
-  if (J > units) J = units;
-  hq::quantize_pack_tma_kernel<<<(unsigned)(S * J), hq::kQtThreads, sizeof(hq::QtSmem) + 128,
-                                 (cudaStream_t)stream>>>(map_x, x, P, T, H, k, keep_idx, rest_idx,
-                                                         inv_scale, zero, codes, side, S, (int)J,
-                                                         wait_limits());
-  return launched();
+  return quantize_entry(x, H, P, T, H, k, keep_idx, rest_idx, inv_scale, zero, codes, side, stream);
+}
+
+hq_status hq_quantize_pack_ld(const uint16_t* x, int ldx, int P, int T, int H, int k, const int32_t* keep_idx,
+                              const int32_t* rest_idx, const float* inv_scale, const uint8_t* zero,
+                              uint32_t* codes, uint16_t* side, void* stream) {
+  return quantize_entry(x, ldx, P, T, H, k, keep_idx, rest_idx, inv_scale, zero, codes, side, stream);
 }
 
 hq_status hq_dequant_reduce(const uint32_t* codes, const uint16_t* side, int P, int T, int H, int k,
                             const int32_t* keep_idx, const int32_t* rest_idx, const float* scale,
                             const uint8_t* zero, void* out, hq_out_dtype out_dtype, void* stream) {
-  return dequant_entry<false>(codes, side, P, T, H, k, keep_idx, rest_idx, scale, zero, out, out_dtype, stream);
+  return dequant_entry<false>(codes, side, P, T, H, k, keep_idx, rest_idx, scale, zero, out, H, out_dtype, stream);
+}
+
+hq_status hq_dequant_reduce_ld(const uint32_t* codes, const uint16_t* side, int P, int T, int H, int k,
+                               const int32_t* keep_idx, const int32_t* rest_idx, const float* scale,
+                               const uint8_t* zero, void* out, int ldo, hq_out_dtype out_dtype, void* stream) {
+  return dequant_entry<false>(codes, side, P, T, H, k, keep_idx, rest_idx, scale, zero, out, ldo, out_dtype,
+                              stream);
+}
+
+hq_status hq_dequant_reduce_ranks(const uint32_t* const* codes, const uint16_t* const* side, int P, int T, int H,
+                                  int k, const int32_t* keep_idx, const int32_t* rest_idx, const float* scale,
+                                  const uint8_t* zero, void* out, hq_out_dtype out_dtype, void* stream) {
+  return dequant_ranks_entry(codes, side, P, T, H, k, keep_idx, rest_idx, scale, zero, out, out_dtype, stream);
 }
 
 hq_status hq_dequant_reduce_bf16_shards(const uint32_t* codes, const uint16_t* side, int P, int T, int H, int k,
                                         const int32_t* keep_idx, const int32_t* rest_idx, const float* scale,
                                         const uint8_t* zero, void* out, hq_out_dtype out_dtype, void* stream) {
-  return dequant_entry<true>(codes, side, P, T, H, k, keep_idx, rest_idx, scale, zero, out, out_dtype, stream);
+  return dequant_entry<true>(codes, side, P, T, H, k, keep_idx, rest_idx, scale, zero, out, H, out_dtype, stream);
 }
 
 hq_status hq_compress_reduce(const uint16_t* x, int P, int T, int H, int k, const int32_t* keep_idx,
                              const int32_t* rest_idx, const float* scale, const float* inv_scale,
                              const uint8_t* zero, void* out, hq_out_dtype out_dtype,
                              uint32_t* codes_or_null, uint16_t* side_or_null, void* stream) {
-  if (check_shape(P, H, k) != HQ_OK || T < 0) return HQ_ERR_INVALID_ARG;
-  if (out_dtype != HQ_OUT_BF16 && out_dtype != HQ_OUT_F32) return HQ_ERR_INVALID_ARG;
-  if (!scale || !inv_scale || !zero) return HQ_ERR_INVALID_ARG;
-  if ((k > 0 && !keep_idx) || (k < H && !rest_idx)) return HQ_ERR_INVALID_ARG;
-  if (T > 0 && (!x || !out)) return HQ_ERR_INVALID_ARG;
-  const bool wire = codes_or_null || side_or_null;
-  if (T > 0 && wire && ((k > 0 && !side_or_null) || (k < H && !codes_or_null))) return HQ_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(out, 16) || !aligned(scale, 16) || !aligned(inv_scale, 16) ||
-      !aligned(zero, 16) || !aligned(keep_idx, 4) || !aligned(rest_idx, 4) ||
-      !aligned(codes_or_null, 4) || !aligned(side_or_null, 16))
-    return HQ_ERR_MISALIGNED;
-  if (T == 0) return HQ_OK;
-  DeviceInfo* d = nullptr;
-  if (device_info(&d) != HQ_OK) return HQ_ERR_CUDA;
-  cudaStream_t st = (cudaStream_t)stream;
-  if (wire) {
-    const hq_status q = hq_quantize_pack(x, P, T, H, k, keep_idx, rest_idx, inv_scale, zero,
-                                         codes_or_null, side_or_null, stream);
-    if (q != HQ_OK) return q;
-  }
-  if (out_dtype == HQ_OUT_BF16)
-    return launch_fused<uint16_t>(x, P, T, H, k, keep_idx, scale, inv_scale, zero, out, st, *d);
-  return launch_fused<float>(x, P, T, H, k, keep_idx, scale, inv_scale, zero, out, st, *d);
+  return compress_entry(x, H, P, T, H, k, keep_idx, rest_idx, scale, inv_scale, zero, out, H, out_dtype,
+                        codes_or_null, side_or_null, stream);
+}
+
+hq_status hq_compress_reduce_ld(const uint16_t* x, int ldx, int P, int T, int H, int k, const int32_t* keep_idx,
+                                const int32_t* rest_idx, const float* scale, const float* inv_scale,
+                                const uint8_t* zero, void* out, int ldo, hq_out_dtype out_dtype,
+                                uint32_t* codes_or_null, uint16_t* side_or_null, void* stream) {
+  return compress_entry(x, ldx, P, T, H, k, keep_idx, rest_idx, scale, inv_scale, zero, out, ldo, out_dtype,
+                        codes_or_null, side_or_null, stream);
 }
 
 const char* hq_status_string(hq_status s) {

@@ -30,7 +30,7 @@ __device__ __forceinline__ uint32_t as_u32(__nv_bfloat162 v) {
 }
 
 __global__ void __launch_bounds__(kCalThreads) calibrate_kernel(
-    const uint16_t* __restrict__ x, int T, int H, float beta, float one_minus_beta, int first_batch,
+    const uint16_t* __restrict__ x, int ldx, int T, int H, float beta, float one_minus_beta, int first_batch,
     float* __restrict__ ema_min, float* __restrict__ ema_max) {
   __shared__ uint32_t s_min[kCalThreads / 32][32];  // [warp][group*4 + pair]
   __shared__ uint32_t s_max[kCalThreads / 32][32];
@@ -49,7 +49,7 @@ __global__ void __launch_bounds__(kCalThreads) calibrate_kernel(
   }
 
   if (h0 < H) {
-    const size_t row_stride = (size_t)H;
+    const size_t row_stride = (size_t)ldx;
     const uint16_t* base = x + (size_t)r * T * row_stride + h0;
     int t = lane_row;
 #pragma unroll 1

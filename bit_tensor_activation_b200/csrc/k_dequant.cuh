@@ -242,13 +242,13 @@ __device__ __forceinline__ void dq_patch_kept(const DqLane& D, float (&acc)[R][8
 }
 
 template <typename OutT, int R>
-__device__ __forceinline__ void dq_store_rows(const DqLane& D, const float (&acc)[R][8], int H, int t0,
+__device__ __forceinline__ void dq_store_rows(const DqLane& D, const float (&acc)[R][8], int ldo, int t0,
                                               int t_last, OutT* __restrict__ out) {
   if (D.active) {
 #pragma unroll
     for (int m = 0; m < R; ++m) {
       const int t = t0 + m;
-      if (t < t_last) store_row8<OutT>(out + (size_t)t * H + D.h0, acc[m]);
+      if (t < t_last) store_row8<OutT>(out + (size_t)t * ldo + D.h0, acc[m]);
     }
   }
 }
@@ -263,22 +263,25 @@ __device__ __forceinline__ void dq_store_rows(const DqLane& D, const float (&acc
 // memory per warp).
 template <typename OutT, int R, bool kVec>
 __device__ __forceinline__ void dq_finish_block(const DqLane& D, float (&acc)[R][8],
-                                                const uint16_t* __restrict__ side, float* kept, int P,
+                                                const uint16_t* __restrict__ side,
+                                                const uint16_t* const* side_ranks, float* kept, int P,
                                                 int T, int H, int k, int ja, int jb, int t0, int t_last,
-                                                OutT* __restrict__ out) {
+                                                OutT* __restrict__ out, int ldo) {
   const int lane = threadIdx.x & 31;
   const int nk = jb - ja;
   const size_t rank_stride = (size_t)k * T;
+  // rank r's side buffer: r*k*T into the stacked one, or its own (side_ranks[r])
+  auto rank_side = [&](int r) { return side_ranks ? side_ranks[r] : side + r * rank_stride; };
   const bool vec = kVec && R == 4 && (T & 3) == 0 && t0 + R <= t_last;
   for (int kc = 0; kc < nk; kc += 32) {
     const int kw = min(32, nk - kc);
     if (vec) {
       if (lane < kw) {
-        const uint16_t* sp = side + (size_t)(ja + kc + lane) * T + t0;  // side[r][j][t], feature-major
+        const size_t off = (size_t)(ja + kc + lane) * T + t0;  // side[r][j][t], feature-major
         float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
 #pragma unroll 4
         for (int r = 0; r < P; ++r) {
-          const uint2 w = __ldg(reinterpret_cast<const uint2*>(sp + r * rank_stride));
+          const uint2 w = __ldg(reinterpret_cast<const uint2*>(rank_side(r) + off));
           a0 = __fadd_rn(a0, __uint_as_float(w.x << 16));
           a1 = __fadd_rn(a1, __uint_as_float(w.x & 0xFFFF0000u));
           a2 = __fadd_rn(a2, __uint_as_float(w.y << 16));
@@ -295,10 +298,10 @@ __device__ __forceinline__ void dq_finish_block(const DqLane& D, float (&acc)[R]
         const int t = t0 + m;
         float a = 0.0f;
         if (t < t_last) {
-          const uint16_t* sp = side + (size_t)(ja + kc + jj) * T + t;
+          const size_t off = (size_t)(ja + kc + jj) * T + t;
 #pragma unroll 8
           for (int r = 0; r < P; ++r)
-            a = __fadd_rn(a, __uint_as_float((uint32_t)__ldg(sp + r * rank_stride) << 16));
+            a = __fadd_rn(a, __uint_as_float((uint32_t)__ldg(rank_side(r) + off) << 16));
         }
         kept[m * 32 + jj] = a;
       }
@@ -307,7 +310,7 @@ __device__ __forceinline__ void dq_finish_block(const DqLane& D, float (&acc)[R]
     dq_patch_kept<R>(D, acc, kept, ja, kc, kw);
     __syncwarp();
   }
-  dq_store_rows<OutT, R>(D, acc, H, t0, t_last, out);
+  dq_store_rows<OutT, R>(D, acc, ldo, t0, t_last, out);
 }
 
 // Slice bookkeeping shared by both kernels.
@@ -467,12 +470,25 @@ __device__ __forceinline__ void dt_patch_kept(const DqLane& D, float (&acc)[kDtR
   }
 }
 
+// Where the P ranks' wires lie.  per_rank == 0: code[0] is one tensor map over the stacked codes
+// [P*T][W] and side[0] over the stacked side buffer [P*k][T] (rank r's rows start at r*T, r*k).
+// per_rank != 0: code[r] and side[r] cover rank r's own buffers, [T][W] and [k][T] -- each may be
+// another GPU's memory mapped into this process, which these loads then read over the
+// interconnect (TMA loads without multicast); side_ptr[r] is rank r's side buffer for the kept
+// sums of slices whose side tiles are not staged.
+constexpr int kMaxRankMaps = 8;
+struct DqWire {
+  CUtensorMap code[kMaxRankMaps];
+  CUtensorMap side[kMaxRankMaps];
+  const uint16_t* side_ptr[kMaxRankMaps];
+  int per_rank;
+};
+
 template <typename OutT, bool kShard>
 __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_kernel(
-    const __grid_constant__ CUtensorMap tmap_codes, const __grid_constant__ CUtensorMap tmap_side, int side_tma,
-    const uint16_t* __restrict__ side, int P, int T, int H,
+    const __grid_constant__ DqWire wire, int side_tma, const uint16_t* __restrict__ side, int P, int T, int H,
     int k, const int32_t* __restrict__ keep_idx, const float* __restrict__ scale,
-    const uint8_t* __restrict__ zero, OutT* __restrict__ out, int S, int chunks, int rows_per_chunk,
+    const uint8_t* __restrict__ zero, OutT* __restrict__ out, int ldo, int S, int chunks, int rows_per_chunk,
     WaitLimits lim) {
   extern __shared__ __align__(128) unsigned char s_raw[];
   DtSmem& sm = *reinterpret_cast<DtSmem*>(s_raw);
@@ -505,8 +521,11 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
 
   if (warp == kDtWarps) {  // ------------------------------------------------ producer
     if (lane == 0) {
-      prefetch_tensor_map(&tmap_codes);
-      if (stage_side) prefetch_tensor_map(&tmap_side);
+      const int n_maps = wire.per_rank ? P : 1;
+      for (int r = 0; r < n_maps; ++r) {
+        prefetch_tensor_map(&wire.code[r]);
+        if (stage_side) prefetch_tensor_map(&wire.side[r]);
+      }
       producer_start_delay(lim.start_delay);
       int issued = 0, bi = 0, g = 0;
       for (int i = 0; i < n_slots_total; ++i) {
@@ -515,10 +534,12 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
         const int r0 = g * kDtG, nr = min(kDtG, P - r0);
         mbar_arrive_expect_tx(&sm.ring.full[st], (unsigned)nr * (kDtTileBytes + (stage_side ? kDtSideBytes : 0u)));
         for (int j = 0; j < nr; ++j) {
-          const int row = (r0 + j) * T + t_first + bi * kDtTileRows;
-          tma_load_2d(&sm.tile[st][j][0][0], &tmap_codes, w_a, row, &sm.ring.full[st]);
+          const int r = r0 + j, m = wire.per_rank ? r : 0;
+          const int t = t_first + bi * kDtTileRows;
+          tma_load_2d(&sm.tile[st][j][0][0], &wire.code[m], w_a, (wire.per_rank ? 0 : r * T) + t,
+                      &sm.ring.full[st]);
           if (stage_side)
-            tma_load_2d(&sm.side[st][j][0][0], &tmap_side, t_first + bi * kDtTileRows, (r0 + j) * k + q.ja,
+            tma_load_2d(&sm.side[st][j][0][0], &wire.side[m], t, (wire.per_rank ? 0 : r * k) + q.ja,
                         &sm.ring.full[st]);
         }
         ++issued;
@@ -606,9 +627,10 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
       dt_patch_kept(D, acc, &sm.k.ksum[buf][0][0], q.ja, nk, warp);
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.ksum_empty[buf]);
-      dq_store_rows<OutT, kDtR>(D, acc, H, t0, t_last, out);
+      dq_store_rows<OutT, kDtR>(D, acc, ldo, t0, t_last, out);
     } else {
-      dq_finish_block<OutT, kDtR, false>(D, acc, side, sm.k.kept[warp], P, T, H, k, q.ja, q.jb, t0, t_last, out);
+      dq_finish_block<OutT, kDtR, false>(D, acc, side, wire.per_rank ? wire.side_ptr : nullptr, sm.k.kept[warp], P,
+                                         T, H, k, q.ja, q.jb, t0, t_last, out, ldo);
     }
   }
 }
@@ -630,7 +652,7 @@ template <typename OutT, bool kShard>
 __global__ void __launch_bounds__(kDqThreads) dequant_reduce_kernel(
     const uint32_t* __restrict__ codes, const uint16_t* __restrict__ side, int P, int T, int H,
     int k, const int32_t* __restrict__ keep_idx, const float* __restrict__ scale,
-    const uint8_t* __restrict__ zero, OutT* __restrict__ out, int S, int chunks, int rows_per_chunk) {
+    const uint8_t* __restrict__ zero, OutT* __restrict__ out, int ldo, int S, int chunks, int rows_per_chunk) {
   extern __shared__ float4 s_dyn[];
   float4* s_const = s_dyn;                                                    // [P][4][32]
   uint32_t* s_tiles = reinterpret_cast<uint32_t*>(s_const + (size_t)P * 4 * 32);
@@ -700,7 +722,7 @@ __global__ void __launch_bounds__(kDqThreads) dequant_reduce_kernel(
       }
       __syncwarp();  // the stage is free for the copy issued next iteration
     }
-    dq_finish_block<OutT, kDqR, true>(D, acc, side, my_kept, P, T, H, k, q.ja, q.jb, t0, t_last, out);
+    dq_finish_block<OutT, kDqR, true>(D, acc, side, nullptr, my_kept, P, T, H, k, q.ja, q.jb, t0, t_last, out, ldo);
   }
   cp_async_wait<0>();
 }

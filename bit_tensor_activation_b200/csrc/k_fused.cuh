@@ -46,7 +46,7 @@ template <typename OutT>
 __global__ void __launch_bounds__(kFuThreads, 2) compress_reduce_kernel(
     const __grid_constant__ CUtensorMap tmap_x, int P, int T, int H, int k,
     const int32_t* __restrict__ keep_idx, const float* __restrict__ scale,
-    const float* __restrict__ inv_scale, const uint8_t* __restrict__ zero, OutT* __restrict__ out, int S,
+    const float* __restrict__ inv_scale, const uint8_t* __restrict__ zero, OutT* __restrict__ out, int ldo, int S,
     int chunks, int rows_per_chunk, WaitLimits lim) {
   extern __shared__ __align__(128) unsigned char s_raw[];
   FuSmem& sm = *reinterpret_cast<FuSmem*>(s_raw);
@@ -185,7 +185,7 @@ __global__ void __launch_bounds__(kFuThreads, 2) compress_reduce_kernel(
     if (active) {
 #pragma unroll
       for (int m = 0; m < kFuR; ++m)
-        if (t0 + m < t_last) store_row8<OutT>(out + (size_t)(t0 + m) * H + h0, acc[m]);
+        if (t0 + m < t_last) store_row8<OutT>(out + (size_t)(t0 + m) * ldo + h0, acc[m]);
     }
   }
 }

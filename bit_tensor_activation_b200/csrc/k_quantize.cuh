@@ -90,7 +90,7 @@ __device__ __forceinline__ QtSlice qt_slice(int ja, int jb, const int32_t* __res
 }
 
 __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
-    const __grid_constant__ CUtensorMap tmap_x, const uint16_t* __restrict__ x, int P, int T, int H,
+    const __grid_constant__ CUtensorMap tmap_x, const uint16_t* __restrict__ x, int ldx, int P, int T, int H,
     int k, const int32_t* __restrict__ keep_idx, const int32_t* __restrict__ rest_idx,
     const float* __restrict__ inv_scale, const uint8_t* __restrict__ zero, uint32_t* __restrict__ codes,
     uint16_t* __restrict__ side, int S, int J, WaitLimits lim) {
@@ -285,7 +285,7 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
         if (q.halo_staged) {
           hb16 = (uint32_t)tile[(warp * kQtRowsPerWarp + h_row) * kQtBoxCols + h_off] << 16;
         } else {  // halo features spread beyond the staged columns: read them directly
-          hb16 = (uint32_t)x[((size_t)r * T + t_base + h_row) * H + q.ha + h_off] << 16;
+          hb16 = (uint32_t)x[((size_t)r * T + t_base + h_row) * ldx + q.ha + h_off] << 16;
         }
         int cc = __float2int_rn(__fmul_rn(__uint_as_float(hb16), h_inv[c]));
         cc = min(max(cc, -h_z), 15 - h_z) + h_z;

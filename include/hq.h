@@ -125,6 +125,27 @@ hq_status hq_dequant_reduce(const uint32_t* codes, const uint16_t* side, int P, 
                             const uint8_t* zero, void* out, hq_out_dtype out_dtype, void* stream);
 
 /*
+ * Dequant-reduce of wires that lie in P separate buffers, one per rank: the receiving side of
+ * bullet "Inference" reading every rank's wire where it lies, with no gathering copy first.
+ * Between GPUs joined by NVLink/NVSwitch, codes[r] and side[r] can be another GPU's memory
+ * mapped into this process (peer access, or a symmetric-memory mapping): each CTA then reads the
+ * remote tiles it reduces over the interconnect with tensor-memory-accelerator loads (no
+ * multicast), so the exchange of the wire and its reduction are one kernel ("Key Observations
+ * and Future Directions" leaves the all-reduce algorithm open).  The caller orders every rank's
+ * hq_quantize_pack before this call (e.g. a stream-ordered barrier across the ranks) and keeps
+ * the buffers unchanged until it has completed.
+ *   codes  host array of P device pointers; codes[r] uint32 [T][(H-k)/8], rank r's 4-bit wire
+ *   side   host array of P device pointers; side[r] bf16 [k][T] (side may be NULL when k == 0)
+ *   1 <= P <= 8; H - k a positive multiple of 32 (code rows of a multiple of 16 bytes);
+ *   codes[r] and side[r] 16-byte aligned.
+ * Parameters, output, arithmetic (R9-R11, rank order 0..P-1) and errors as in hq_dequant_reduce;
+ * the result is bitwise that of hq_dequant_reduce on the stacked wire.
+ */
+hq_status hq_dequant_reduce_ranks(const uint32_t* const* codes, const uint16_t* const* side, int P, int T, int H,
+                                  int k, const int32_t* keep_idx, const int32_t* rest_idx, const float* scale,
+                                  const uint8_t* zero, void* out, hq_out_dtype out_dtype, void* stream);
+
+/*
  * Dequant-reduce, literal reading of bullet "Inference" (R19): after communication each rank's
  * tensor is first made BF16 and the ranks' BF16 tensors are then combined.  Same arguments,
  * layouts, ownership and errors as hq_dequant_reduce; only non-kept features differ:
@@ -151,6 +172,35 @@ hq_status hq_compress_reduce(const uint16_t* x, int P, int T, int H, int k, cons
                              const int32_t* rest_idx, const float* scale, const float* inv_scale,
                              const uint8_t* zero, void* out, hq_out_dtype out_dtype,
                              uint32_t* codes_or_null, uint16_t* side_or_null, void* stream);
+
+/*
+ * Partial-channel synchronisation -- the abstract of "Communication-Aware Architecture for
+ * Tensor-parallelism" (CAAT-Net) on the first page: tensor-parallel ranks can do without
+ * synchronising every activation channel.  Reading R20: a block of consecutive features of each
+ * rank's partial sum goes through the hybrid wire and the rank-ordered sum, and every rank keeps
+ * its own partial sum in the other features.  The four calls below are the calls above on such a
+ * block: `H` is the block's width, x points at the block's first feature of rank 0, row 0, and
+ * rows are ldx elements apart (rank r's rows start at x + r*T*ldx); out points at the block's
+ * first feature of row 0 and its rows are ldo elements apart.  Only the block's columns of out
+ * are written: a rank that keeps its own partial sum in out's other columns gets exactly the
+ * reading's result.  Statistics, parameters, codes and side are those of the dense [P][T][H]
+ * block (as if it were copied out first), so hq_select_topk and hq_wire_bytes_per_row apply as
+ * they are, and a rank sends (H-k)/2 + 2k bytes per row for the block alone.
+ *   ldx, ldo  >= H and multiples of 8; x and out 16-byte aligned (so the block starts at a
+ *             multiple of 8 features).  Other arguments, checks and errors as in the calls above.
+ */
+hq_status hq_calibrate_ld(const uint16_t* x, int ldx, int P, int T, int H, float beta, int first_batch,
+                          float* ema_min, float* ema_max, void* stream);
+hq_status hq_quantize_pack_ld(const uint16_t* x, int ldx, int P, int T, int H, int k, const int32_t* keep_idx,
+                              const int32_t* rest_idx, const float* inv_scale, const uint8_t* zero,
+                              uint32_t* codes, uint16_t* side, void* stream);
+hq_status hq_dequant_reduce_ld(const uint32_t* codes, const uint16_t* side, int P, int T, int H, int k,
+                               const int32_t* keep_idx, const int32_t* rest_idx, const float* scale,
+                               const uint8_t* zero, void* out, int ldo, hq_out_dtype out_dtype, void* stream);
+hq_status hq_compress_reduce_ld(const uint16_t* x, int ldx, int P, int T, int H, int k, const int32_t* keep_idx,
+                                const int32_t* rest_idx, const float* scale, const float* inv_scale,
+                                const uint8_t* zero, void* out, int ldo, hq_out_dtype out_dtype,
+                                uint32_t* codes_or_null, uint16_t* side_or_null, void* stream);
 
 /* A static string naming a status. */
 const char* hq_status_string(hq_status s);
