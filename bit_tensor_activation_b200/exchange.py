@@ -12,6 +12,10 @@ between GPUs):
                       itself (one exchange step; the reduction is done P times over)
   ``reduce_scatter``  the wire is split into P row blocks; rank j receives block j of every rank's
                       wire (all-to-all), reduces it, and the reduced bf16 blocks are all-gathered
+  ``peer``            (``PeerAllReduce``) every rank packs into its own part of a symmetric-memory
+                      allocation and reduces all P wires reading the peers' buffers in place over
+                      NVLink/NVSwitch (hq_dequant_reduce_ranks): the exchange and the reduction are
+                      one kernel, with a barrier on each side
   two-step            (``TwoStepAllReduce``) ``reduce_scatter``'s first step, then each reducer
                       quantizes its reduced block again with its own 4-bit grid and the step-2
                       wires are all-gathered and dequantized: the quantized reduce-scatter plus
@@ -33,7 +37,7 @@ from dataclasses import dataclass
 import torch
 import torch.distributed as dist
 
-from . import (hq_calibrate, hq_dequant_reduce, hq_quantize_pack, hq_select_topk)
+from . import (hq_calibrate, hq_dequant_reduce, hq_dequant_reduce_ranks, hq_quantize_pack, hq_select_topk)
 
 
 # ---------------------------------------------------------------------------------------------
@@ -199,6 +203,64 @@ class HybridAllReduce:
     def __call__(self, x: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
         codes, side = self.pack(x)
         return self.reduce(*self.exchange(codes, side), out=out)
+
+
+class PeerAllReduce:
+    """Scheme ``peer``: the wires stay where they are written and every rank's reduction reads the
+    others' in place.
+
+    ``wires`` is a list of P (codes [T, W] int32, side [k, T] bf16) pairs, entry r rank r's wire as
+    this process sees it: for real ranks, the ranks' parts of one symmetric-memory allocation
+    (``symmetric_wires``), so that entry r != rank is a peer GPU's memory reached over
+    NVLink/NVSwitch.  ``barrier`` orders the ranks: every rank's pack before any reduction, and
+    every reduction before the next pack overwrites a wire.  Nothing is gathered: the only data
+    movement is the reduction kernel's own loads of the P wires."""
+
+    def __init__(self, params: HybridParams, T: int, rank: int, wires, barrier=None):
+        self.p, self.T, self.rank = params, T, rank
+        if len(wires) != params.P:
+            raise ValueError("one (codes, side) pair per rank")
+        self.wires = wires
+        self.barrier = barrier or (lambda: None)
+        self.inv, self.zero = params.row(rank)
+
+    def pack(self, x: torch.Tensor, stream=None) -> None:
+        p = self.p
+        codes, side = self.wires[self.rank]
+        hq_quantize_pack(x.unsqueeze(0), p.keep_idx, p.rest_idx, self.inv, self.zero, codes.unsqueeze(0),
+                         side.unsqueeze(0), stream=stream)
+
+    def reduce(self, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        p = self.p
+        if out is None:
+            out = torch.empty((self.T, p.H), dtype=torch.bfloat16, device=p.scale.device)
+        hq_dequant_reduce_ranks([c for c, _ in self.wires], [s for _, s in self.wires], p.keep_idx, p.rest_idx,
+                                p.scale, p.zero, out, stream=stream)
+        return out
+
+    def __call__(self, x: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+        self.pack(x)
+        self.barrier()   # every rank's wire is written
+        out = self.reduce(out)
+        self.barrier()   # every rank has read the wires
+        return out
+
+
+def symmetric_wires(params: HybridParams, T: int, group=None, timeout_ms: int = 10000):
+    """The P ranks' wire buffers in one symmetric-memory allocation across the group (one process
+    per GPU, peer access between the GPUs): returns (wires, barrier) for ``PeerAllReduce``.  The
+    barrier is torch's device-side one, bounded by timeout_ms."""
+    import torch.distributed._symmetric_memory as symm_mem
+
+    P, H, k = params.P, params.H, params.k
+    W = (H - k) // 8
+    code_bytes = (T * W * 4 + 255) // 256 * 256
+    side_bytes = (k * T * 2 + 255) // 256 * 256
+    buf = symm_mem.empty(code_bytes + side_bytes, dtype=torch.uint8, device=params.scale.device)
+    hdl = symm_mem.rendezvous(buf, group if group is not None else dist.group.WORLD)
+    wires = [(hdl.get_buffer(r, (T, W), torch.int32, 0), hdl.get_buffer(r, (k, T), torch.bfloat16, code_bytes // 2))
+             for r in range(P)]
+    return wires, (lambda: hdl.barrier(channel=0, timeout_ms=timeout_ms))
 
 
 # ---------------------------------------------------------------------------------------------
