@@ -22,14 +22,14 @@ Variants:
   because they are computed for every feature.
 - ``int4_only``: k = 0.
 - ``bf16_only``: k = H, the uncompressed bf16 wire; only the fp32 summation remains.
-- ``two_step``: a two-step compressed all-reduce (reduce-scatter, then all-gather), the scheme
-  the "Flash Communication" abstract among the source pages names without an algorithm. The design
-  used here: step 1 is the ``topk`` path with bf16 output, and reducer j owns row block j of
-  it. In step 2 each reducer quantizes its block again with the same hybrid scheme, and every
-  rank dequantizes all blocks (a reduction over P = 1). The step-2 grids and kept features come
-  from calibration and selection with P = 1 on the reduced calibration batches. On one GPU the
-  row blocks together are the whole output, so step 2 is one quantize-pack and one
-  dequant-reduce call with P = 1; the time reported is step 2's.
+- ``two_step``: the two-step compressed all-reduce of ``bit_tensor_activation_b200.exchange``
+  (reduce-scatter, then all-gather), the scheme the "Flash Communication" abstract among the
+  source pages names without an algorithm: step 1 is the ``topk`` path with bf16 output, and
+  reducer j owns row block j of it; in step 2 each reducer quantizes its block again with its
+  own grid (calibrated on its reduced calibration blocks; one kept set selected over the
+  reducers' statistics) and every block is dequantized with its reducer's grid. On one GPU the
+  P blocks are handled one by one, a P = 1 quantize-pack and dequant-reduce each; the time
+  reported is step 2's.
 
 For every variant the tool reports MSE, MSE relative to the mean square of the exact sum, the
 largest absolute error and the wire compression ratio.  It also times the variant's reduction:
@@ -156,45 +156,40 @@ def run_workload(cfg: synth.Config, reps: int, flush: torch.Tensor, seed: int) -
     return rows
 
 
-def one_step_bf16(x, keep, rest, scale, inv, zero):
-    """Step 1: the hybrid quantize-pack of every rank and the rank-ordered reduction, bf16 out."""
-    P, T, H = x.shape
-    k = keep.shape[0]
-    codes = torch.empty((P, T, (H - k) // 8), dtype=torch.int32, device=x.device)
-    side = torch.empty((P, k, T), dtype=torch.int16, device=x.device)
-    hq.hq_quantize_pack(x, keep, rest, inv, zero, codes, side)
-    y = torch.empty((T, H), dtype=torch.int16, device=x.device)
-    hq.hq_dequant_reduce(codes, side, keep, rest, scale, zero, y)
-    return y
-
-
 def two_step(cfg, x, exact, mean_sq, keep, rest, scale, inv, zero, cs_dev, reps, flush) -> dict:
+    """The two-step all-reduce of the exchange module on one GPU: step 1 is the hybrid reduction;
+    in step 2 every reducer re-quantizes its row block with its own grid (calibrated on its
+    reduced calibration blocks) and the blocks are dequantized one by one."""
+    from bit_tensor_activation_b200 import exchange as ex
+
     dev = x.device
     P, T, H, k = cfg.P, cfg.T, cfg.H, cfg.k
-    # step-2 grids: calibration (P = 1) on the reduced calibration batches, then selection
-    e2min = torch.empty((1, H), dtype=torch.float32, device=dev)
-    e2max = torch.empty_like(e2min)
-    cal = torch.empty((P, cfg.calib_T, H), dtype=torch.int16, device=dev)
-    for b in range(cfg.calib_batches):
-        synth.fill_gpu(cfg, synth.CALIB, b, cal, cs_dev, T=cfg.calib_T)
-        y_cal = one_step_bf16(cal, keep, rest, scale, inv, zero)
-        hq.hq_calibrate(y_cal[None], e2min, e2max, cfg.beta, b == 0)
-    del cal
-    keep2 = torch.empty(k, dtype=torch.int32, device=dev)
-    rest2 = torch.empty(H - k, dtype=torch.int32, device=dev)
-    scale2 = torch.empty((1, H), dtype=torch.float32, device=dev)
-    inv2 = torch.empty_like(scale2)
-    zero2 = torch.empty((1, H), dtype=torch.uint8, device=dev)
-    hq.hq_select_topk(e2min, e2max, k, keep2, rest2, scale2, inv2, zero2)
-    # step 1 on the evaluation batch, then step 2: quantize the reduced rows again, dequantize
-    y = one_step_bf16(x, keep, rest, scale, inv, zero)[None].contiguous()
-    codes2 = torch.empty((1, T, (H - k) // 8), dtype=torch.int32, device=dev)
-    side2 = torch.empty((1, k, T), dtype=torch.int16, device=dev)
+    params = ex.HybridParams(keep, rest, scale, inv, zero)
+
+    def cal_batches():
+        cal = torch.empty((P, cfg.calib_T, H), dtype=torch.int16, device=dev)
+        for b in range(cfg.calib_batches):
+            synth.fill_gpu(cfg, synth.CALIB, b, cal, cs_dev, T=cfg.calib_T)
+            yield cal.view(torch.bfloat16)
+
+    p2 = ex.step_two_params_simulated(cal_batches(), params, k, cfg.beta)
+    Tb = T // P
+    out1 = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
     out = torch.empty((T, H), dtype=torch.float32, device=dev)
+    codes = torch.empty((P, T, (H - k) // 8), dtype=torch.int32, device=dev)
+    side = torch.empty((P, k, T), dtype=torch.bfloat16, device=dev)
+    codes2 = torch.empty((P, Tb, (H - k) // 8), dtype=torch.int32, device=dev)
+    side2 = torch.empty((P, k, Tb), dtype=torch.bfloat16, device=dev)
+    xb = x.view(torch.bfloat16)
+    ex.two_step_simulated(xb, params, p2, out1, out, codes, side, codes2, side2)
 
     def step2():
-        hq.hq_quantize_pack(y, keep2, rest2, inv2, zero2, codes2, side2)
-        hq.hq_dequant_reduce(codes2, side2, keep2, rest2, scale2, zero2, out)
+        for j in range(P):
+            rows = slice(j * Tb, (j + 1) * Tb)
+            hq.hq_quantize_pack(out1[rows].unsqueeze(0), p2.keep_idx, p2.rest_idx, p2.inv_scale[j:j + 1],
+                                p2.zero[j:j + 1], codes2[j:j + 1], side2[j:j + 1])
+            hq.hq_dequant_reduce(codes2[j:j + 1], side2[j:j + 1], p2.keep_idx, p2.rest_idx, p2.scale[j:j + 1],
+                                 p2.zero[j:j + 1], out[rows])
 
     us = timed_us(step2, reps, flush)
     step2()
