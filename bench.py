@@ -49,6 +49,8 @@ def parse_args():
     ap.add_argument("--cold-reps", type=int, default=20, help="launches of each kernel timed alone, L2 flushed")
     ap.add_argument("--second-steps", type=int, default=400,
                     help="timed steps of the second large workload (0: skip it)")
+    ap.add_argument("--no-next", dest="next_paths", action="store_false",
+                    help="skip the two-step, partial-sync and per-rank-buffer measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-clocks", action="store_true")
@@ -427,6 +429,104 @@ def measure_workload(W: Workload, K, warmup, cold_reps, stream, flush, peak):
     }
 
 
+def measure_next(W: Workload, reps, stream, flush, peak):
+    """The next stages on the same workload, each timed with the L2 flushed before every call:
+    the two-step all-reduce on one GPU (step 1 = the split path, step 2 = the reducers' blocks
+    re-quantized and dequantized one by one), partial-channel synchronisation of the first half
+    of the features (the _ld calls on the column block), and the reduction over one wire buffer
+    per rank against the stacked buffer."""
+    import torch
+
+    import bit_tensor_activation_b200 as hq
+    from bit_tensor_activation_b200 import exchange as ex
+
+    cfg, B, dev = W.cfg, W.B, W.dev
+    P, T, H, k = cfg.P, cfg.T, cfg.H, cfg.k
+    res = {}
+    params = ex.HybridParams(B.keep_idx, B.rest_idx, B.scale, B.inv_scale, B.zero)
+    part = P * T * H * 2
+
+    # two-step: step-2 grids from two calibration batches through step 1
+    k2 = k
+    cs_dev = torch.from_numpy(synth.colscale(cfg)[0]).to(dev)
+    cal = []
+    for b in range(2):
+        c = torch.empty((P, T, H), dtype=torch.int16, device=dev)
+        synth.fill_gpu(cfg, synth.CALIB, 100 + b, c, cs_dev)
+        cal.append(c.view(torch.bfloat16))
+    p2 = ex.step_two_params_simulated(cal, params, k2, cfg.beta)
+    del cal
+    Tb = T // P
+    out1 = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    out2 = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    codes2 = torch.empty((P, Tb, (H - k2) // 8), dtype=torch.int32, device=dev)
+    side2 = torch.empty((P, k2, Tb), dtype=torch.bfloat16, device=dev)
+    x = W.x.view(torch.bfloat16)
+
+    ws = torch.empty(hq.hq_two_step_workspace_bytes(P, T, H, k, k2), dtype=torch.uint8, device=dev)
+
+    def two_step():
+        hq.hq_two_step_reduce(x, params.keep_idx, params.rest_idx, params.scale, params.inv_scale, params.zero,
+                              p2.keep_idx, p2.rest_idx, p2.scale, p2.inv_scale, p2.zero, ws, out2)
+
+    def step2():
+        for j in range(P):
+            rows = slice(j * Tb, (j + 1) * Tb)
+            hq.hq_quantize_pack(out1[rows].unsqueeze(0), p2.keep_idx, p2.rest_idx, p2.inv_scale[j:j + 1],
+                                p2.zero[j:j + 1], codes2[j:j + 1], side2[j:j + 1])
+            hq.hq_dequant_reduce(codes2[j:j + 1], side2[j:j + 1], p2.keep_idx, p2.rest_idx, p2.scale[j:j + 1],
+                                 p2.zero[j:j + 1], out2[rows])
+
+    t = time_cold([("two_step", two_step), ("step2", step2)], reps, stream, flush)
+    ex.two_step_simulated(x, params, p2, out1, B.out, B.codes, B.side, codes2, side2)
+    hq.hq_two_step_reduce(x, params.keep_idx, params.rest_idx, params.scale, params.inv_scale, params.zero,
+                          p2.keep_idx, p2.rest_idx, p2.scale, p2.inv_scale, p2.zero, ws, out2)
+    torch.cuda.synchronize()
+    same = bool(torch.equal(out2.view(torch.int16), B.out.view(torch.int16)))
+    del ws
+    res["two_step"] = {"call": "hq_two_step_reduce", "equals_python_composition": same,
+                       "ms_per_step": t["two_step"], "value": part / (t["two_step"] * 1e-3) / 1e9, "unit": "GB/s",
+                       "step2_us": 1e3 * t["step2"], "launches_per_step": 2 + 2 * P,
+                       "step2_wire_bytes_per_reducer": Tb * ((H - k2) // 2 + 2 * k2)}
+
+    # partial-channel synchronisation of features [0, H/2)
+    Hs = H // 2
+    ks = k // 2
+    emin = torch.empty((P, Hs), dtype=torch.float32, device=dev)
+    emax = torch.empty_like(emin)
+    hq.hq_calibrate_ld(W.x[:, :, :Hs], emin, emax, cfg.beta, True)
+    Bs = hq.Buffers(P, T, Hs, ks, device=dev)
+    hq.hq_select_topk(emin, emax, ks, Bs.keep_idx, Bs.rest_idx, Bs.scale, Bs.inv_scale, Bs.zero)
+    outp = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+
+    def partial():
+        hq.hq_quantize_pack_ld(W.x[:, :, :Hs], Bs.keep_idx, Bs.rest_idx, Bs.inv_scale, Bs.zero, Bs.codes, Bs.side)
+        hq.hq_dequant_reduce_ld(Bs.codes, Bs.side, Bs.keep_idx, Bs.rest_idx, Bs.scale, Bs.zero, outp[:, :Hs])
+
+    t = time_cold([("partial", partial)], reps, stream, flush)
+    sync_bytes = P * T * Hs * 2
+    res["partial_sync"] = {"features_synced": Hs, "kept": ks, "ms_per_step": t["partial"],
+                           "value": sync_bytes / (t["partial"] * 1e-3) / 1e9, "unit": "GB/s of synchronised partial sums",
+                           "wire_bytes_per_rank_row": hq.hq_wire_bytes_per_row(Hs, ks),
+                           "full_wire_bytes_per_rank_row": hq.hq_wire_bytes_per_row(H, k)}
+
+    # the reduction over one wire buffer per rank (what a rank reading its peers in place runs)
+    W.quantize_pack()
+    cl = [B.codes[r].clone() for r in range(P)]
+    sl = [B.side[r].clone() for r in range(P)]
+    outr = torch.empty_like(B.out)
+
+    def ranks():
+        hq.hq_dequant_reduce_ranks(cl, sl, B.keep_idx, B.rest_idx, B.scale, B.zero, outr)
+
+    t = time_cold([("ranks", ranks), ("stacked", W.dequant_reduce)], reps, stream, flush)
+    ab = algo_bytes(cfg)["dequant_reduce"]
+    torch.cuda.synchronize()
+    res["ranks"] = {"per_rank_buffers": _kernel_entry(ab, t["ranks"], peak), "stacked": _kernel_entry(ab, t["stacked"], peak),
+                    "equal": bool(torch.equal(outr.view(torch.int16), B.out.view(torch.int16)))}
+    return res
+
+
 def run_hq(args, cfg, world, rank, local):
     import torch
 
@@ -486,6 +586,7 @@ def run_hq(args, cfg, world, rank, local):
     offline = time_cold([("calibrate", W.calibrate), ("select", W.select)], max(3, args.cold_reps // 4), stream,
                         flush)
     W.select()  # the parameters the checks below use
+    nxt = measure_next(W, max(3, args.cold_reps // 2), stream, flush, peak) if args.next_paths else None
 
     # ---- fused output equals split output on this workload -------------------------------------------
     W.quantize_pack()
@@ -619,6 +720,7 @@ def run_hq(args, cfg, world, rank, local):
         "alt_paths": {alt_path: {"ms_per_step": ms_alt / Ka, "value": part_bytes / (ms_alt / Ka * 1e-3) / 1e9,
                                  "kernel_ms": per_alt}},
         "workloads": workloads,
+        "next": nxt,
         "fused_equals_split": fused_equal,
         "cpu_baseline": cpu,
         "e2e": e2e,

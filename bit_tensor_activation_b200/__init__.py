@@ -45,6 +45,11 @@ _lib.hq_selftest_bounded_wait.argtypes = [ctypes.c_longlong, _vp]
 _lib.hq_selftest_bounded_wait.restype = _i32
 _lib.hq_dequant_reduce_ranks.argtypes = [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _i32, _vp]
 _lib.hq_dequant_reduce_ranks.restype = _i32
+_lib.hq_two_step_reduce.argtypes = [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp,
+                                    _vp, _vp, ctypes.c_size_t, _vp, _i32, _vp]
+_lib.hq_two_step_reduce.restype = _i32
+_lib.hq_two_step_workspace_bytes.argtypes = [_i32, _i32, _i32, _i32, _i32]
+_lib.hq_two_step_workspace_bytes.restype = ctypes.c_size_t
 _lib.hq_calibrate_ld.argtypes = [_vp, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp]
 _lib.hq_quantize_pack_ld.argtypes = [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.hq_dequant_reduce_ld.argtypes = [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp]
@@ -63,7 +68,8 @@ HQ_OUT_BF16, HQ_OUT_F32 = 0, 1
 EXPORTS = ["hq_calibrate", "hq_select_topk", "hq_quantize_pack", "hq_dequant_reduce",
            "hq_dequant_reduce_bf16_shards", "hq_compress_reduce", "hq_status_string", "hq_read_device_error", "hq_wire_bytes_per_row",
            "hq_selftest_bounded_wait", "hq_selftest_set_pipeline_stall", "hq_calibrate_ld", "hq_quantize_pack_ld",
-           "hq_dequant_reduce_ld", "hq_compress_reduce_ld", "hq_dequant_reduce_ranks"]
+           "hq_dequant_reduce_ld", "hq_compress_reduce_ld", "hq_dequant_reduce_ranks", "hq_two_step_reduce",
+           "hq_two_step_workspace_bytes"]
 
 
 class HQError(RuntimeError):
@@ -218,6 +224,29 @@ def hq_dequant_reduce_ranks(codes, side, keep_idx, rest_idx, scale, zero, out, s
             _ptr(scale, _F32, (P, H), "scale"), _ptr(zero, _U8, (P, H), "zero"),
             _ptr(out, _BF16 + _F32, (T, H), "out"), odt, _stream(stream, out.device))
     _check(_lib.hq_dequant_reduce_ranks(*args), "hq_dequant_reduce_ranks")
+
+
+def hq_two_step_workspace_bytes(P: int, T: int, H: int, k: int, k2: int) -> int:
+    return int(_lib.hq_two_step_workspace_bytes(P, T, H, k, k2))
+
+
+def hq_two_step_reduce(x, keep_idx, rest_idx, scale, inv_scale, zero, keep2, rest2, scale2, inv_scale2, zero2,
+                       workspace, out, stream=None) -> None:
+    """The two-step all-reduce of P simulated ranks x [P, T, H] on one GPU; workspace is a uint8
+    device tensor of at least hq_two_step_workspace_bytes(...) bytes."""
+    P, T, H = x.shape
+    k, k2 = keep_idx.shape[0], keep2.shape[0]
+    odt = HQ_OUT_F32 if out.dtype == torch.float32 else HQ_OUT_BF16
+    if not isinstance(workspace, torch.Tensor) or not workspace.is_cuda or not workspace.is_contiguous():
+        raise TypeError("workspace must be a contiguous CUDA tensor")
+    args = (_ptr(x, _BF16, (P, T, H), "x"), P, T, H, k, _ptr(keep_idx, _I32, (k,), "keep_idx"),
+            _ptr(rest_idx, _I32, (H - k,), "rest_idx"), _ptr(scale, _F32, (P, H), "scale"),
+            _ptr(inv_scale, _F32, (P, H), "inv_scale"), _ptr(zero, _U8, (P, H), "zero"), k2,
+            _ptr(keep2, _I32, (k2,), "keep2"), _ptr(rest2, _I32, (H - k2,), "rest2"),
+            _ptr(scale2, _F32, (P, H), "scale2"), _ptr(inv_scale2, _F32, (P, H), "inv_scale2"),
+            _ptr(zero2, _U8, (P, H), "zero2"), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+            _ptr(out, _BF16 + _F32, (T, H), "out"), odt, _stream(stream, x.device))
+    _check(_lib.hq_two_step_reduce(*args), "hq_two_step_reduce")
 
 
 # -- partial-channel synchronisation: the same calls on a block of features [c0, c0 + Hs) -------

@@ -394,9 +394,89 @@ hq_status compress_entry(const uint16_t* x, int ldx, int P, int T, int H, int k,
   return launch_fused<float>(x, ldx, P, T, H, k, keep_idx, scale, inv_scale, zero, out, ldo, st, *d);
 }
 
+// The two-step all-reduce's workspace: step-1 wire (codes, side), the reduced tensor, and the P
+// reducers' step-2 wires, each region 256-byte aligned.
+struct TwoStepLayout {
+  size_t codes, side, red, codes2, side2, total;
+};
+size_t round256(size_t n) { return (n + 255) & ~size_t(255); }
+TwoStepLayout two_step_layout(int P, int T, int H, int k, int k2) {
+  TwoStepLayout L;
+  size_t off = 0;
+  L.codes = off;
+  off += round256((size_t)P * T * (H - k) / 2);
+  L.side = off;
+  off += round256((size_t)P * k * T * 2);
+  L.red = off;
+  off += round256((size_t)T * H * 2);
+  L.codes2 = off;
+  off += round256((size_t)T * (H - k2) / 2);  // P blocks of T/P rows
+  L.side2 = off;
+  off += round256((size_t)k2 * T * 2);
+  L.total = off;
+  return L;
+}
+
+hq_status two_step_entry(const uint16_t* x, int P, int T, int H, int k, const int32_t* keep_idx,
+                         const int32_t* rest_idx, const float* scale, const float* inv_scale, const uint8_t* zero,
+                         int k2, const int32_t* keep2, const int32_t* rest2, const float* scale2,
+                         const float* inv_scale2, const uint8_t* zero2, void* workspace, size_t workspace_bytes,
+                         void* out, hq_out_dtype out_dtype, void* stream) {
+  if (check_shape(P, H, k) != HQ_OK || check_shape(P, H, k2) != HQ_OK || T < 0 || T % P != 0 || H % 16 != 0)
+    return HQ_ERR_INVALID_ARG;  // H % 16: every reducer's row of zero2 starts on a 16-byte boundary
+  if (out_dtype != HQ_OUT_BF16 && out_dtype != HQ_OUT_F32) return HQ_ERR_INVALID_ARG;
+  if (!scale2 || !inv_scale2 || !zero2 || (k2 > 0 && !keep2) || (k2 < H && !rest2)) return HQ_ERR_INVALID_ARG;
+  if (!aligned(scale2, 16) || !aligned(inv_scale2, 16) || !aligned(zero2, 16) || !aligned(keep2, 4) ||
+      !aligned(rest2, 4))
+    return HQ_ERR_MISALIGNED;
+  if (T == 0) return HQ_OK;
+  const TwoStepLayout L = two_step_layout(P, T, H, k, k2);
+  if (!workspace || workspace_bytes < L.total) return HQ_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256)) return HQ_ERR_MISALIGNED;
+  char* ws = static_cast<char*>(workspace);
+  uint32_t* codes = reinterpret_cast<uint32_t*>(ws + L.codes);
+  uint16_t* side = reinterpret_cast<uint16_t*>(ws + L.side);
+  uint16_t* red = reinterpret_cast<uint16_t*>(ws + L.red);
+  uint32_t* codes2 = reinterpret_cast<uint32_t*>(ws + L.codes2);
+  uint16_t* side2 = reinterpret_cast<uint16_t*>(ws + L.side2);
+  // step 1: every rank's wire, the rank-ordered reduction into the reduced tensor (bf16)
+  hq_status st = quantize_entry(x, H, P, T, H, k, keep_idx, rest_idx, inv_scale, zero, codes, side, stream);
+  if (st != HQ_OK) return st;
+  st = dequant_entry<false>(codes, side, P, T, H, k, keep_idx, rest_idx, scale, zero, red, H, HQ_OUT_BF16, stream);
+  if (st != HQ_OK) return st;
+  // step 2: reducer j re-quantizes its row block with grid row j; the block is dequantized with it
+  const int Tb = T / P;
+  const size_t esz = out_dtype == HQ_OUT_F32 ? 4 : 2;
+  for (int j = 0; j < P; ++j) {
+    uint32_t* cj = codes2 + (size_t)j * Tb * ((H - k2) / 8);
+    uint16_t* sj = side2 + (size_t)j * k2 * Tb;
+    st = quantize_entry(red + (size_t)j * Tb * H, H, 1, Tb, H, k2, keep2, rest2, inv_scale2 + (size_t)j * H,
+                        zero2 + (size_t)j * H, cj, sj, stream);
+    if (st != HQ_OK) return st;
+    st = dequant_entry<false>(cj, sj, 1, Tb, H, k2, keep2, rest2, scale2 + (size_t)j * H, zero2 + (size_t)j * H,
+                              static_cast<char*>(out) + (size_t)j * Tb * H * esz, H, out_dtype, stream);
+    if (st != HQ_OK) return st;
+  }
+  return HQ_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t hq_two_step_workspace_bytes(int P, int T, int H, int k, int k2) {
+  if (check_shape(P, H, k) != HQ_OK || check_shape(P, H, k2) != HQ_OK || T < 0) return 0;
+  return two_step_layout(P, T, H, k, k2).total;
+}
+
+hq_status hq_two_step_reduce(const uint16_t* x, int P, int T, int H, int k, const int32_t* keep_idx,
+                             const int32_t* rest_idx, const float* scale, const float* inv_scale, const uint8_t* zero,
+                             int k2, const int32_t* keep2, const int32_t* rest2, const float* scale2,
+                             const float* inv_scale2, const uint8_t* zero2, void* workspace, size_t workspace_bytes,
+                             void* out, hq_out_dtype out_dtype, void* stream) {
+  return two_step_entry(x, P, T, H, k, keep_idx, rest_idx, scale, inv_scale, zero, k2, keep2, rest2, scale2,
+                        inv_scale2, zero2, workspace, workspace_bytes, out, out_dtype, stream);
+}
 
 hq_status hq_calibrate(const uint16_t* x, int P, int T, int H, float beta, int first_batch,
                        float* ema_min, float* ema_max, void* stream) {

@@ -42,6 +42,7 @@
 #ifndef HQ_H
 #define HQ_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -201,6 +202,33 @@ hq_status hq_compress_reduce_ld(const uint16_t* x, int ldx, int P, int T, int H,
                                 const int32_t* rest_idx, const float* scale, const float* inv_scale,
                                 const uint8_t* zero, void* out, int ldo, hq_out_dtype out_dtype,
                                 uint32_t* codes_or_null, uint16_t* side_or_null, void* stream);
+
+/*
+ * The two-step compressed all-reduce of P simulated ranks on one GPU -- the quantized
+ * reduce-scatter then re-quantized all-gather of the "Flash Communication" abstract (third page),
+ * reading R22 (no formula there).  Step 1: hq_quantize_pack and hq_dequant_reduce of x [P][T][H]
+ * with the step-1 selection and grids, the reduced tensor rounded to bf16.  Step 2: reducer j owns
+ * rows [j*T/P, (j+1)*T/P); it quantize-packs its block with row j of the step-2 grids
+ * (scale2/inv_scale2/zero2 [P][H]) and the step-2 kept set (keep2 [k2], rest2 [H-k2]), and the
+ * block is dequantized with the same grid (P = 1, nothing summed) into those rows of out.
+ *   x, keep_idx .. zero   as in hq_compress_reduce (step 1)
+ *   k2, keep2 .. zero2    the step-2 selection and the reducers' grids
+ *   workspace             device memory of at least hq_two_step_workspace_bytes(P, T, H, k, k2)
+ *                         bytes, 256-byte aligned, owned by the caller: it holds the step-1 wire,
+ *                         the reduced tensor and the step-2 wires (its contents are scratch)
+ *   out                   [T][H], bf16 or fp32
+ *   T % P == 0 and H % 16 == 0 (every reducer's row of zero2 then starts on a 16-byte boundary).
+ * Enqueues 2 + 2P kernels on `stream`.  Errors as in the calls above; a workspace that is NULL or
+ * too small is HQ_ERR_INVALID_ARG, one below 256-byte alignment HQ_ERR_MISALIGNED.
+ */
+hq_status hq_two_step_reduce(const uint16_t* x, int P, int T, int H, int k, const int32_t* keep_idx,
+                             const int32_t* rest_idx, const float* scale, const float* inv_scale, const uint8_t* zero,
+                             int k2, const int32_t* keep2, const int32_t* rest2, const float* scale2,
+                             const float* inv_scale2, const uint8_t* zero2, void* workspace, size_t workspace_bytes,
+                             void* out, hq_out_dtype out_dtype, void* stream);
+
+/* Bytes of workspace hq_two_step_reduce needs (0 for sizes it rejects). */
+size_t hq_two_step_workspace_bytes(int P, int T, int H, int k, int k2);
 
 /* A static string naming a status. */
 const char* hq_status_string(hq_status s);

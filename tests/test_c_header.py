@@ -24,12 +24,20 @@ static void expect(hq_status got, hq_status want, const char* what) {
 }
 
 int main(void) {
-  static uint16_t x[64];  /* only the address is used: every call below fails its checks first */
-  static float f[64];
-  static int32_t idx[16];
-  static uint8_t z[64];
-  static uint32_t codes[16];
-  static uint16_t side[16];
+  /* only the addresses are used: every call below fails its checks first.  The unions with a
+     long double give every buffer the 16-byte alignment the checks ask for (C99 has no alignas). */
+  static union { uint16_t v[64]; long double a; } ux;
+  static union { float v[64]; long double a; } uf;
+  static union { int32_t v[16]; long double a; } ui;
+  static union { uint8_t v[64]; long double a; } uz;
+  static union { uint32_t v[16]; long double a; } uc;
+  static union { uint16_t v[16]; long double a; } us;
+  uint16_t* x = ux.v;
+  float* f = uf.v;
+  int32_t* idx = ui.v;
+  uint8_t* z = uz.v;
+  uint32_t* codes = uc.v;
+  uint16_t* side = us.v;
   const uint16_t* odd = (const uint16_t*)((const char*)x + 2);
 
   expect(hq_calibrate(NULL, 1, 1, 8, 0.9f, 1, f, f, NULL), HQ_ERR_INVALID_ARG, "calibrate x NULL");
@@ -50,6 +58,14 @@ int main(void) {
   expect(hq_selftest_bounded_wait(-1, NULL), HQ_ERR_INVALID_ARG, "self-test negative limit");
   expect(hq_selftest_set_pipeline_stall(1, 0), HQ_ERR_INVALID_ARG, "stall with one bound");
   expect(hq_selftest_set_pipeline_stall(0, 0), HQ_OK, "stall cleared");
+  expect(hq_two_step_reduce(x, 2, 3, 16, 8, idx, idx, f, f, z, 8, idx, idx, f, f, z, x, 1 << 20, x, HQ_OUT_BF16, NULL),
+         HQ_ERR_INVALID_ARG, "two-step T % P");
+  expect(hq_two_step_reduce(x, 2, 4, 16, 8, idx, idx, f, f, z, 8, idx, idx, f, f, z, x, 1, x, HQ_OUT_BF16, NULL),
+         HQ_ERR_INVALID_ARG, "two-step workspace too small");
+  if (hq_two_step_workspace_bytes(2, 4, 16, 8, 8) == 0 || hq_two_step_workspace_bytes(2, 4, 12, 8, 8) != 0) {
+    puts("FAIL two-step workspace bytes");
+    ++fails;
+  }
   if (hq_wire_bytes_per_row(8192, 256) != (8192 - 256) / 2 + 2 * 256) { puts("FAIL wire bytes"); ++fails; }
   if (hq_wire_bytes_per_row(8, 16) != -1) { puts("FAIL wire bytes k > H"); ++fails; }
   if (strcmp(hq_status_string(HQ_ERR_BAD_INDEX), "HQ_ERR_BAD_INDEX") != 0) { puts("FAIL string"); ++fails; }

@@ -126,6 +126,27 @@ def test_two_step_loopback_and_simulated():
     ex.two_step_simulated(xd, params, p2, out1, out, codes, side, codes2, side2)
     assert_same(u16(out1), ref, "simulated step 1")
     assert_same(u16(out), want, "simulated two-step")
+    # the same scheme as one call of the C ABI, in a caller-owned workspace
+    import bit_tensor_activation_b200 as hq
+
+    nbytes = hq.hq_two_step_workspace_bytes(P, T, H, k, k2)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=DEV)
+    args = (xd, params.keep_idx, params.rest_idx, params.scale, params.inv_scale, params.zero, p2.keep_idx,
+            p2.rest_idx, p2.scale, p2.inv_scale, p2.zero)
+    out_c = torch.empty((T, H), dtype=torch.bfloat16, device=DEV)
+    hq.hq_two_step_reduce(*args, ws, out_c)
+    assert_same(u16(out_c), want, "hq_two_step_reduce, bf16")
+    out_f = torch.empty((T, H), dtype=torch.float32, device=DEV)
+    hq.hq_two_step_reduce(*args, ws, out_f)
+    want_f = []
+    for j in range(P):
+        cj, sj = o.quantize_pack(ref[None, j * Tb:(j + 1) * Tb], p2_ref["keep_idx"], p2_ref["rest_idx"],
+                                 p2_ref["inv_scale"][j:j + 1], p2_ref["zero"][j:j + 1])
+        want_f.append(o.dequant_reduce(cj, sj, H, p2_ref["keep_idx"], p2_ref["rest_idx"], p2_ref["scale"][j:j + 1],
+                                       p2_ref["zero"][j:j + 1], out_f32=True))
+    assert_same(out_f.cpu().numpy().view(np.uint32), np.concatenate(want_f).view(np.uint32), "hq_two_step_reduce, fp32")
+    with pytest.raises(hq.HQError):  # a workspace one byte short
+        hq.hq_two_step_reduce(*args, ws[:nbytes - 1], out_c)
     assert_no_device_error()
 
 
