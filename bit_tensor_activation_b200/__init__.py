@@ -48,6 +48,9 @@ _lib.hq_dequant_reduce_ranks.restype = _i32
 _lib.hq_two_step_reduce.argtypes = [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp,
                                     _vp, _vp, ctypes.c_size_t, _vp, _i32, _vp]
 _lib.hq_two_step_reduce.restype = _i32
+_lib.hq_two_step_reduce_noalloc.argtypes = [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp,
+                                            _vp, _vp, _vp, _vp, _i32, _vp]
+_lib.hq_two_step_reduce_noalloc.restype = _i32
 _lib.hq_two_step_workspace_bytes.argtypes = [_i32, _i32, _i32, _i32, _i32]
 _lib.hq_two_step_workspace_bytes.restype = ctypes.c_size_t
 _lib.hq_calibrate_ld.argtypes = [_vp, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp]
@@ -69,7 +72,7 @@ EXPORTS = ["hq_calibrate", "hq_select_topk", "hq_quantize_pack", "hq_dequant_red
            "hq_dequant_reduce_bf16_shards", "hq_compress_reduce", "hq_status_string", "hq_read_device_error", "hq_wire_bytes_per_row",
            "hq_selftest_bounded_wait", "hq_selftest_set_pipeline_stall", "hq_calibrate_ld", "hq_quantize_pack_ld",
            "hq_dequant_reduce_ld", "hq_compress_reduce_ld", "hq_dequant_reduce_ranks", "hq_two_step_reduce",
-           "hq_two_step_workspace_bytes"]
+           "hq_two_step_workspace_bytes", "hq_two_step_reduce_noalloc"]
 
 
 class HQError(RuntimeError):
@@ -247,6 +250,24 @@ def hq_two_step_reduce(x, keep_idx, rest_idx, scale, inv_scale, zero, keep2, res
             _ptr(zero2, _U8, (P, H), "zero2"), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
             _ptr(out, _BF16 + _F32, (T, H), "out"), odt, _stream(stream, x.device))
     _check(_lib.hq_two_step_reduce(*args), "hq_two_step_reduce")
+
+
+def hq_two_step_reduce_noalloc(x, keep_idx, rest_idx, scale, inv_scale, zero, keep2, rest2, scale2, inv_scale2,
+                               zero2, out, stream=None) -> None:
+    """hq_two_step_reduce with the library's fixed scratch array instead of a workspace, for
+    callers that cannot allocate device memory (problems up to HQ_TWO_STEP_NOALLOC_MAX_BYTES of
+    workspace; calls that overlap on the GPU race on the array)."""
+    P, T, H = x.shape
+    k, k2 = keep_idx.shape[0], keep2.shape[0]
+    odt = HQ_OUT_F32 if out.dtype == torch.float32 else HQ_OUT_BF16
+    args = (_ptr(x, _BF16, (P, T, H), "x"), P, T, H, k, _ptr(keep_idx, _I32, (k,), "keep_idx"),
+            _ptr(rest_idx, _I32, (H - k,), "rest_idx"), _ptr(scale, _F32, (P, H), "scale"),
+            _ptr(inv_scale, _F32, (P, H), "inv_scale"), _ptr(zero, _U8, (P, H), "zero"), k2,
+            _ptr(keep2, _I32, (k2,), "keep2"), _ptr(rest2, _I32, (H - k2,), "rest2"),
+            _ptr(scale2, _F32, (P, H), "scale2"), _ptr(inv_scale2, _F32, (P, H), "inv_scale2"),
+            _ptr(zero2, _U8, (P, H), "zero2"), _ptr(out, _BF16 + _F32, (T, H), "out"), odt,
+            _stream(stream, x.device))
+    _check(_lib.hq_two_step_reduce_noalloc(*args), "hq_two_step_reduce_noalloc")
 
 
 # -- partial-channel synchronisation: the same calls on a block of features [c0, c0 + Hs) -------

@@ -460,9 +460,46 @@ hq_status two_step_entry(const uint16_t* x, int P, int T, int H, int k, const in
   return HQ_OK;
 }
 
+// Scratch of hq_two_step_reduce_noalloc: a fixed array in every device's global memory, so that a
+// caller that may not allocate device memory needs no workspace.  In host code the array's name
+// only stands for it; its device address is fetched once per device (device_scratch) and passed to
+// the kernels like any workspace pointer.
+constexpr size_t kNoAllocScratchBytes = HQ_TWO_STEP_NOALLOC_MAX_BYTES;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+void* g_scratch_ptr[kMaxDevices] = {};
+std::mutex g_scratch_mu;
+
+// The current device's address of g_noalloc_scratch, looked up on the first call on that device.
+hq_status device_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return HQ_ERR_CUDA;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return HQ_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+hq_status hq_two_step_reduce_noalloc(const uint16_t* x, int P, int T, int H, int k, const int32_t* keep_idx,
+                                     const int32_t* rest_idx, const float* scale, const float* inv_scale,
+                                     const uint8_t* zero, int k2, const int32_t* keep2, const int32_t* rest2,
+                                     const float* scale2, const float* inv_scale2, const uint8_t* zero2, void* out,
+                                     hq_out_dtype out_dtype, void* stream) {
+  const size_t need = hq_two_step_workspace_bytes(P, T, H, k, k2);
+  if (need == 0 || need > kNoAllocScratchBytes) return HQ_ERR_INVALID_ARG;  // rejected before any launch
+  void* scratch = nullptr;
+  if (device_scratch(&scratch) != HQ_OK) return HQ_ERR_CUDA;
+  return two_step_entry(x, P, T, H, k, keep_idx, rest_idx, scale, inv_scale, zero, k2, keep2, rest2, scale2,
+                        inv_scale2, zero2, scratch, kNoAllocScratchBytes, out, out_dtype, stream);
+}
 
 size_t hq_two_step_workspace_bytes(int P, int T, int H, int k, int k2) {
   if (check_shape(P, H, k) != HQ_OK || check_shape(P, H, k2) != HQ_OK || T < 0) return 0;

@@ -230,6 +230,34 @@ hq_status hq_two_step_reduce(const uint16_t* x, int P, int T, int H, int k, cons
 /* Bytes of workspace hq_two_step_reduce needs (0 for sizes it rejects). */
 size_t hq_two_step_workspace_bytes(int P, int T, int H, int k, int k2);
 
+/*
+ * hq_two_step_reduce without a workspace argument: it allocates nothing and takes no memory from
+ * the caller beyond its inputs and outputs.  (The pages have no counterpart: this is a service of
+ * the library, not a step of the method.)  It is meant for callers that cannot call cudaMalloc --
+ * a serving process whose device memory is fixed at start-up, a plugin running inside another
+ * framework's memory pool, or a latency-critical loop where an allocation's device-wide
+ * synchronisation is not acceptable.
+ *
+ * The scratch lives in a fixed array of HQ_TWO_STEP_NOALLOC_MAX_BYTES bytes in the global memory
+ * of every GPU that loads the library, held until the process exits.  Problems whose
+ * hq_two_step_workspace_bytes(P, T, H, k, k2) exceeds it (or is 0) return HQ_ERR_INVALID_ARG before
+ * anything is enqueued: decode-size problems fit (P = 4, T = 32, H = 4096 needs under 1 MiB), the
+ * prefill shapes need hq_two_step_reduce and a workspace of their own.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
+ *     that device current) and keeps it; make that first call before any stream capture.
+ *   - Every call on a device shares the one array, and it keeps the last call's contents.  Nothing
+ *     in it needs to start at zero: every byte a call reads, the same call has written first.
+ *   - Calls whose work overlaps on the GPU (for example on two streams without an order between
+ *     them) race on the array and give undefined results: order them.
+ * Arguments, result and errors otherwise as in hq_two_step_reduce; the result is bitwise the same.
+ */
+#define HQ_TWO_STEP_NOALLOC_MAX_BYTES ((size_t)16 << 20)
+hq_status hq_two_step_reduce_noalloc(const uint16_t* x, int P, int T, int H, int k, const int32_t* keep_idx,
+                                     const int32_t* rest_idx, const float* scale, const float* inv_scale,
+                                     const uint8_t* zero, int k2, const int32_t* keep2, const int32_t* rest2,
+                                     const float* scale2, const float* inv_scale2, const uint8_t* zero2, void* out,
+                                     hq_out_dtype out_dtype, void* stream);
+
 /* A static string naming a status. */
 const char* hq_status_string(hq_status s);
 
