@@ -138,6 +138,13 @@ def select_shared(ema_min: torch.Tensor, ema_max: torch.Tensor, k: int, group=No
 # ---------------------------------------------------------------------------------------------
 # The compressed all-reduce
 # ---------------------------------------------------------------------------------------------
+def _check_row_aligned(H: int) -> None:
+    """A rank's row of the parameters is passed to the library on its own; zero rows (one byte per
+    feature) start on a 16-byte boundary only when H is a multiple of 16."""
+    if H % 16:
+        raise ValueError(f"the per-rank calls need H % 16 == 0 (H = {H})")
+
+
 class HybridAllReduce:
     """All-reduce of this rank's partial sum x [T, H] (bf16) through the hybrid wire.
 
@@ -150,6 +157,7 @@ class HybridAllReduce:
         if scheme not in ("allgather", "reduce_scatter"):
             raise ValueError(f"unknown scheme {scheme}")
         P, H, k = params.P, params.H, params.k
+        _check_row_aligned(H)
         if scheme == "reduce_scatter" and T % P:
             raise ValueError(f"reduce_scatter needs T % P == 0 (T={T}, P={P})")
         self.p, self.T, self.rank, self.scheme, self.group = params, T, rank, scheme, group
@@ -220,6 +228,7 @@ class PeerAllReduce:
         self.p, self.T, self.rank = params, T, rank
         if len(wires) != params.P:
             raise ValueError("one (codes, side) pair per rank")
+        _check_row_aligned(params.H)
         self.wires = wires
         self.barrier = barrier or (lambda: None)
         self.inv, self.zero = params.row(rank)
