@@ -8,6 +8,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstring>
 #include <type_traits>
@@ -200,11 +201,12 @@ hq_status launch_dequant(const WireSrc& src, int P, int T, int H, int k, const i
     auto kern = hq::dequant_reduce_tma_kernel<OutT, kShard>;
     int per_sm = 0;
     if (occupancy(d.dequant_tma[kF32][kShard], kern, hq::kDtThreads, smem, P, &per_sm) != HQ_OK) return HQ_ERR_CUDA;
-    int chunks, rpc;
-    slice_chunks(T, S, (long long)d.sms * per_sm, hq::kDtTileRows, &chunks, &rpc);
+    // one wave: each slice's row blocks split evenly over as many CTAs as fit
+    const long long nb_all = ceil_div(T, hq::kDtTileRows);
+    const int chunks = (int)std::max(1LL, std::min((long long)d.sms * per_sm / S, nb_all));
     kern<<<(unsigned)(S * chunks), hq::kDtThreads, smem, st>>>(wire, side_tma ? 1 : 0, src.side, P, T, H, k,
                                                                 keep_idx, scale, zero, static_cast<OutT*>(out), ldo,
-                                                                S, chunks, rpc, wait_limits());
+                                                                S, chunks, wait_limits());
     return launched();
   }
   const size_t smem = hq::dq_smem_bytes(P);

@@ -195,6 +195,46 @@ __device__ __forceinline__ SliceKept slice_kept(const int32_t* __restrict__ keep
   return r;
 }
 
+// slice_kept() for a group of threads that has already loaded the first entry of keep_idx each
+// (v0 = keep_idx[tid] for tid < k, INT_MAX otherwise), so that load can be issued together with
+// the caller's other set-up loads; with a third bound hi2 >= hi: jc = #{keep_idx < hi2}, and
+// list gets keep_idx[ja .. ja + min(jc - ja, cap)).  s_cnt holds 3 ints.
+struct SliceKept3 {
+  int ja, jb, jc;
+};
+__device__ __forceinline__ SliceKept3 slice_kept3(int v0, const int32_t* __restrict__ keep_idx, int k, int lo,
+                                                  int hi, int hi2, int* s_cnt, int* list, int cap, int nthreads) {
+  int a = v0 < lo, b = v0 < hi, c = v0 < hi2;
+  for (int i = threadIdx.x + nthreads; i < k; i += nthreads) {
+    const int v = __ldg(keep_idx + i);
+    a += v < lo;
+    b += v < hi;
+    c += v < hi2;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    a += __shfl_down_sync(0xFFFFFFFFu, a, off);
+    b += __shfl_down_sync(0xFFFFFFFFu, b, off);
+    c += __shfl_down_sync(0xFFFFFFFFu, c, off);
+  }
+  if (threadIdx.x == 0) s_cnt[0] = s_cnt[1] = s_cnt[2] = 0;
+  group_sync(nthreads);
+  if ((threadIdx.x & 31) == 0) {
+    atomicAdd(&s_cnt[0], a);
+    atomicAdd(&s_cnt[1], b);
+    atomicAdd(&s_cnt[2], c);
+  }
+  group_sync(nthreads);
+  const SliceKept3 r{s_cnt[0], s_cnt[1], s_cnt[2]};
+  const int n = min(r.jc - r.ja, cap);
+  const int i0 = (int)threadIdx.x - r.ja;  // this thread's own entry, already in v0
+  if ((int)threadIdx.x < k && i0 >= 0 && i0 < n) list[i0] = v0;
+  for (int i = r.ja + threadIdx.x; i < r.ja + n; i += nthreads)
+    if (i >= nthreads) list[i - r.ja] = __ldg(keep_idx + i);
+  group_sync(nthreads);
+  return r;
+}
+
 // group_layout() for a group inside a range whose kept features are list[0..n) (= keep_idx[ja..),
 // ascending), without touching global memory.
 __device__ __forceinline__ GroupLayout group_layout_list(const int* list, int n, int ja, int H, int k, int h0) {

@@ -103,6 +103,14 @@ __device__ __forceinline__ void prefetch_tensor_map(const CUtensorMap* map) {
 __device__ __forceinline__ void named_barrier_sync(int nthreads) {
   asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
 }
+// Named barrier `id` among `nthreads` threads (whole warps): bar.arrive signals without waiting,
+// bar.sync waits for all.  Used to order a producer's first loads after the consumers' set-up loads.
+__device__ __forceinline__ void named_barrier_arrive_id(int id, int nthreads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+__device__ __forceinline__ void named_barrier_sync_id(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
 // Same barrier, returning whether `pred` held in any participating thread.
 __device__ __forceinline__ bool named_barrier_or(int nthreads, bool pred) {
   uint32_t r;

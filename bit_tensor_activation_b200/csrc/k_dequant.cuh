@@ -174,6 +174,59 @@ __device__ __forceinline__ void dq_fill_constants(float4* s_const, const int32_t
   }
 }
 
+// One (rank, group) pair of slice s, idx = rank * 32 + group: the scale and zero of its 8
+// features, loaded ahead of the rest of the set-up (nothing in the address depends on the kept
+// features).  Pairs past the tensor load nothing.
+struct DqPair {
+  float4 s0, s1;
+  uint2 z;
+};
+__device__ __forceinline__ DqPair dq_load_pair(const float* __restrict__ scale, const uint8_t* __restrict__ zero,
+                                               int P, int H, int s, int idx) {
+  DqPair d;
+  d.s0 = d.s1 = make_float4(1.0f, 1.0f, 1.0f, 1.0f);
+  d.z = make_uint2(0u, 0u);
+  const int r = idx >> 5, hg = 8 * (s * kDqSliceGroups + (idx & 31));
+  if (r < P && hg < H) {  // r*H + hg is a multiple of 8; scale and zero are 16-byte aligned
+    const size_t p = (size_t)r * H + hg;
+    d.s0 = __ldg(reinterpret_cast<const float4*>(scale + p));
+    d.s1 = __ldg(reinterpret_cast<const float4*>(scale + p) + 1);
+    d.z = __ldg(reinterpret_cast<const uint2*>(zero + p));
+  }
+  return d;
+}
+__device__ __forceinline__ bool dq_pair_tiny(const DqPair& d) {
+  return d.s0.x < 0x1p-109f || d.s0.y < 0x1p-109f || d.s0.z < 0x1p-109f || d.s0.w < 0x1p-109f ||
+         d.s1.x < 0x1p-109f || d.s1.y < 0x1p-109f || d.s1.z < 0x1p-109f || d.s1.w < 0x1p-109f;
+}
+// dq_fill_constants() for one pair from its loaded parameters (group_kmask in shared memory).
+__device__ __forceinline__ void dq_fill_pair(float4* s_const, const uint32_t* group_kmask, const DqPair& d, int H,
+                                             int s, int idx, bool generic) {
+  const int r = idx >> 5, g = idx & 31;
+  const int hg = 8 * (s * kDqSliceGroups + g);
+  const uint32_t km = hg < H ? group_kmask[g] : 0u;
+  int pos[8], jpos[8];
+  dq_positions(km, pos, jpos);
+  const float scv[8] = {d.s0.x, d.s0.y, d.s0.z, d.s0.w, d.s1.x, d.s1.y, d.s1.z, d.s1.w};
+  float sc[8], off[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    sc[i] = 0.0f;
+    off[i] = -8388608.0f;  // kept / inactive: decodes to a small value times scale 0
+    if (hg < H && !((km >> i) & 1u)) {
+      const int e = generic ? 0 : 4 * pos[i];
+      const uint32_t z = ((i < 4 ? d.z.x : d.z.y) >> (8 * (i & 3))) & 0xFFu;
+      sc[i] = __fmul_rn(scv[i], __int_as_float((127 - e) << 23));  // scale / 16^p, exact
+      off[i] = -__int_as_float(0x4B000000 | ((int)z << e));         // -(2^23 + zero*16^p)
+    }
+  }
+  float4* dst = s_const + (size_t)r * 4 * 32 + g;
+  dst[0] = make_float4(sc[0], sc[1], sc[2], sc[3]);
+  dst[32] = make_float4(sc[4], sc[5], sc[6], sc[7]);
+  dst[64] = make_float4(off[0], off[1], off[2], off[3]);
+  dst[96] = make_float4(off[4], off[5], off[6], off[7]);
+}
+
 // Adds one rank's contribution for R staged rows (row m at st + m * stride words).  kShard: the
 // literal reading of the reduction, in which the rank's dequantized value (q - zero) * scale is
 // first rounded to bf16 and then added (the default adds the exact product with one FMA).
@@ -367,7 +420,7 @@ struct DtSmem {
   uint64_t ksum_full[2];   // the kept-sum warp has written ksum[b]
   uint64_t ksum_empty[2];  // every consumer warp has read ksum[b]
   int klist[8 * kDqSliceGroups];  // the slice's kept features
-  int kcnt[2];
+  int kcnt[3];
   uint32_t gkmask[kDqSliceGroups];  // per group of the slice: kept mask and kept features before it
   int gj0[kDqSliceGroups];
   TmaRing<kDtStages> ring;
@@ -488,15 +541,17 @@ template <typename OutT, bool kShard>
 __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_kernel(
     const __grid_constant__ DqWire wire, int side_tma, const uint16_t* __restrict__ side, int P, int T, int H,
     int k, const int32_t* __restrict__ keep_idx, const float* __restrict__ scale,
-    const uint8_t* __restrict__ zero, OutT* __restrict__ out, int ldo, int S, int chunks, int rows_per_chunk,
-    WaitLimits lim) {
+    const uint8_t* __restrict__ zero, OutT* __restrict__ out, int ldo, int S, int chunks, WaitLimits lim) {
   extern __shared__ __align__(128) unsigned char s_raw[];
   DtSmem& sm = *reinterpret_cast<DtSmem*>(s_raw);
   float4* s_const = reinterpret_cast<float4*>(s_raw + ((sizeof(DtSmem) + 127) & ~size_t(127)));
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int s = blockIdx.x / chunks, chunk = blockIdx.x - s * chunks;
-  const int t_first = chunk * rows_per_chunk, t_last = min(T, t_first + rows_per_chunk);
-  const int nblk = (t_last - t_first + kDtTileRows - 1) / kDtTileRows;
+  // the slice's row blocks split evenly over its `chunks` CTAs (counts differ by one at most)
+  const int nb_all = (T + kDtTileRows - 1) / kDtTileRows;
+  const int b_first = (int)((long long)chunk * nb_all / chunks), b_end = (int)((long long)(chunk + 1) * nb_all / chunks);
+  const int t_first = b_first * kDtTileRows, t_last = min(T, b_end * kDtTileRows);
+  const int nblk = b_end - b_first;
   const int n_groups = (P + kDtG - 1) / kDtG;  // ring slots per block
   const int n_slots_total = nblk * n_groups;     // slot i = (block i / n_groups, rank group i % n_groups)
 
@@ -509,9 +564,15 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
     sm.abort = 0;
     fence_barrier_init();
   }
-  // the slice's kept features, counted by the whole CTA (no dependent searches before the loads)
+  // Set-up loads first, independent of one another so that they cost one round trip together:
+  // each consumer thread's (rank, group) pair of parameters, and one keep_idx entry per thread.
+  // The producer's first tiles need the slice's kept count, so they follow this round trip.
+  const DqPair pre = warp < kDtWarps ? dq_load_pair(scale, zero, P, H, s, threadIdx.x) : DqPair{};
+  const int kv0 = (int)threadIdx.x < k ? __ldg(keep_idx + threadIdx.x) : 0x7FFFFFFF;
+  // the slice's kept features, counted by the whole CTA
   const int hs0 = 8 * s * kDqSliceGroups, he0 = min(H, hs0 + 8 * kDqSliceGroups);
-  const SliceKept sk = slice_kept(keep_idx, k, hs0, he0, sm.kcnt, sm.klist, 8 * kDqSliceGroups, kDtThreads);
+  const SliceKept3 sk = slice_kept3(kv0, keep_idx, k, hs0, he0, he0, sm.kcnt, sm.klist, 8 * kDqSliceGroups,
+                                    kDtThreads);
   const DqSlice q = dq_slice_from(sk.ja, sk.jb, H, k, s, S);
   const int w_a = q.w_first & ~3;  // 16-byte aligned x coordinate of the box
   const int nk = q.jb - q.ja;
@@ -584,8 +645,14 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
     sm.gkmask[lane] = L.kmask;
     sm.gj0[lane] = L.j0;
   }
-  const bool generic = named_barrier_or(kConsumers, dq_has_tiny_scale(scale, P, H, s, kConsumers));
-  dq_fill_constants(s_const, keep_idx, sm.gkmask, scale, zero, P, H, k, s, generic, kConsumers);
+  // the slice's (rank, group) pairs: this thread's first one preloaded, any others (P > 8) now
+  bool tiny = dq_pair_tiny(pre);
+  for (int idx = threadIdx.x + kConsumers; idx < P * 32; idx += kConsumers)
+    tiny = tiny || dq_pair_tiny(dq_load_pair(scale, zero, P, H, s, idx));
+  const bool generic = named_barrier_or(kConsumers, tiny);
+  if ((int)threadIdx.x < P * 32) dq_fill_pair(s_const, sm.gkmask, pre, H, s, threadIdx.x, generic);
+  for (int idx = threadIdx.x + kConsumers; idx < P * 32; idx += kConsumers)
+    dq_fill_pair(s_const, sm.gkmask, dq_load_pair(scale, zero, P, H, s, idx), H, s, idx, generic);
   GroupLayout Lg;
   Lg.kmask = sm.gkmask[lane];
   Lg.j0 = sm.gj0[lane];

@@ -50,29 +50,29 @@ constexpr int kQtBoxU32 = kQtBoxCols / 2;               // box inner dim in 32-b
 constexpr int kQtBufWords = 36;                         // >= 33 owned words + 2 guard slots per row
 constexpr int kQtHaloSlots = 2;                         // (row, halo feature) pairs per lane
 constexpr int kQtKeptSlots = 4;                         // (row, kept feature) pairs per lane
+constexpr int kQtHaloCand = 16;                         // features after the slice whose parameters are preloaded
+constexpr int kQtStartBarrier = 2;                      // named barrier: consumers' set-up loads issued
 constexpr int kQtMaxFastKept = 32 * kQtKeptSlots / kQtRowsPerWarp;  // slices with more copy in a loop
 constexpr unsigned kQtTileBytes = kQtTileRows * kQtBoxCols * 2;
 
 struct QtSmem {
   alignas(128) uint16_t tile[kQtStages][kQtTileRows][kQtBoxCols];
   uint32_t buf[kQtWarps][kQtRowsPerWarp][kQtBufWords];
-  int klist[kQtSlice];  // the slice's kept features
-  int kcnt[2];
+  int klist[kQtSlice + kQtHaloCand];  // the slice's kept features, then those among the halo candidates
+  int kcnt[3];
   uint32_t gkmask[kQtSlice / 8];  // per group of the slice: kept mask, kept features before it
   int gj0[kQtSlice / 8];
   TmaRing<kQtStages> ring;
   int abort;
 };
 
-// Slice facts shared by the producer and the consumers.
+// Slice facts of the consumers.
 struct QtSlice {
   int ha, hb, ja, jb, Ca, Cb, Wb, We, nw, nhalo;
-  bool halo_staged;  // every halo feature lies in the staged columns [ha, ha + kQtBoxCols)
 };
 
 // ja, jb = number of kept features before ha and before hb.
-__device__ __forceinline__ QtSlice qt_slice(int ja, int jb, const int32_t* __restrict__ rest_idx, int H, int k,
-                                            int s) {
+__device__ __forceinline__ QtSlice qt_slice(int ja, int jb, int H, int k, int s) {
   QtSlice q;
   const int Hr = H - k;
   q.ha = s * kQtSlice;
@@ -85,8 +85,53 @@ __device__ __forceinline__ QtSlice qt_slice(int ja, int jb, const int32_t* __res
   q.We = (q.Cb + 7) >> 3;
   q.nw = max(q.We - q.Wb, 0);
   q.nhalo = (q.We > q.Wb) ? (8 * q.We - q.Cb) : 0;
-  q.halo_staged = q.nhalo == 0 || checked_col(rest_idx, q.Cb + q.nhalo - 1, H) < q.ha + kQtBoxCols;
   return q;
+}
+
+// The idx-th (from 0) feature at or after hb that is not kept: compact position Cb + idx.
+// cand_kept: bit d set when feature hb + d (d < kQtHaloCand) is kept.  Features beyond the
+// candidates are found by walking keep_idx from jc (the first kept feature >= hb + kQtHaloCand);
+// every entry read is range-checked.
+__device__ __forceinline__ int qt_rest_col(int idx, int hb, uint32_t cand_kept, const int32_t* __restrict__ keep_idx,
+                                           int k, int jc, int H) {
+  int n = 0;
+#pragma unroll
+  for (int d = 0; d < kQtHaloCand; ++d) {
+    if (!((cand_kept >> d) & 1u)) {
+      if (n == idx) return hb + d;
+      ++n;
+    }
+  }
+  int j = jc;
+  for (int c = hb + kQtHaloCand; c < H; ++c) {
+    const int kj = j < k ? checked_col(keep_idx, j, H) : H;
+    if (kj == c) {
+      ++j;
+      continue;
+    }
+    if (n == idx) return c;
+    ++n;
+  }
+  record_error(HQ_ERR_BAD_INDEX);
+  return H - 1;
+}
+
+// A lane's 8 parameters: inv_scale and zero of features h0 .. h0+7 of one rank.
+struct QtParams {
+  float4 i0, i1;
+  uint2 z;
+};
+__device__ __forceinline__ QtParams qt_load_params(const float* __restrict__ inv_scale,
+                                                   const uint8_t* __restrict__ zero, size_t p, bool on) {
+  QtParams r;
+  r.i0 = r.i1 = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  r.z = make_uint2(0u, 0u);
+  if (on) {  // p is a multiple of 8; both arrays are 16-byte aligned
+    r.i0 = __ldg(reinterpret_cast<const float4*>(inv_scale + p));
+    r.i1 = __ldg(reinterpret_cast<const float4*>(inv_scale + p) + 1);
+    r.z = __ldg(reinterpret_cast<const uint2*>(zero + p));
+  }
+  return r;
 }
 
 __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
@@ -115,6 +160,9 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
 
   // ---------------------------------------------------------------- producer warp
   if (warp == kQtWarps) {
+    // the first tiles go out after the consumers' set-up loads (which then are not queued
+    // behind them); the consumers arrive on this barrier before they wait for anything
+    named_barrier_sync_id(kQtStartBarrier, kQtThreads);
     if (lane == 0) {
       prefetch_tensor_map(&tmap_x);
       producer_start_delay(lim.start_delay);
@@ -140,29 +188,53 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
   // ---------------------------------------------------------------- consumer warps
   const int Hr = H - k, Wr = Hr / 8, NG = H / 8;
   int r = u0 / NB, b = u0 - (u0 / NB) * NB;
-  bool fresh = true;  // rank changed: reload this lane's parameters
-  // the slice's kept features, counted by the consumer warps (the producer is already loading)
   constexpr int kConsumers = 32 * kQtWarps;
   const int ha0 = s * kQtSlice, hb0 = min(H, ha0 + kQtSlice);
-  const SliceKept sk = slice_kept(keep_idx, k, ha0, hb0, sm.kcnt, sm.klist, kQtSlice, kConsumers);
-  const QtSlice q = qt_slice(sk.ja, sk.jb, rest_idx, H, k, s);
+  const int g = s * (kQtSlice / 8) + lane;  // this lane's group
+  const bool active = g < NG;
+  // Set-up loads first, independent of one another so that they cost one round trip together:
+  // this lane's parameters for the first unit's rank, the parameters of the kQtHaloCand features
+  // after the slice (lane d of every warp: feature hb0 + d; the halo is among them unless kept
+  // features crowd the start of the next slice), and one keep_idx entry per thread.
+  QtParams pr = qt_load_params(inv_scale, zero, (size_t)r * H + 8 * g, active && n_units > 0);
+  float hc_inv = 0.0f;
+  uint32_t hc_z = 0;
+  if (lane < kQtHaloCand && hb0 + lane < H && n_units > 0) {
+    hc_inv = __ldg(inv_scale + (size_t)r * H + hb0 + lane);
+    hc_z = __ldg(zero + (size_t)r * H + hb0 + lane);
+  }
+  const int kv0 = (int)threadIdx.x < k ? __ldg(keep_idx + threadIdx.x) : 0x7FFFFFFF;
+  named_barrier_arrive_id(kQtStartBarrier, kQtThreads);
+  // the slice's kept features and those among the halo candidates
+  const SliceKept3 sk = slice_kept3(kv0, keep_idx, k, ha0, hb0, hb0 + kQtHaloCand, sm.kcnt, sm.klist,
+                                    kQtSlice + kQtHaloCand, kConsumers);
+  const QtSlice q = qt_slice(sk.ja, sk.jb, H, k, s);
   if (threadIdx.x == 0 && ((s == 0 && q.ja != 0) || (s == S - 1 && q.jb != k) || q.jb - q.ja > kQtSlice))
     record_error(HQ_ERR_BAD_INDEX);
   // the groups' layouts, the same for every rank
   if (warp == 0) {
-    const int g = s * (kQtSlice / 8) + lane;
-    const GroupLayout Lg = g < NG ? group_layout_list(sm.klist, min(q.jb - q.ja, kQtSlice), q.ja, H, k, 8 * g)
+    const GroupLayout Lg = active ? group_layout_list(sm.klist, min(q.jb - q.ja, kQtSlice), q.ja, H, k, 8 * g)
                                   : GroupLayout{0, 0, 0u, 0};
     sm.gkmask[lane] = Lg.kmask;
     sm.gj0[lane] = Lg.j0;
   }
+  // kept features among the halo candidates (a candidate past H counts as kept: never a halo)
+  uint32_t cand_kept = (hb0 + kQtHaloCand > H) ? ~0u << max(H - hb0, 0) : 0u;
+  for (int i = min(q.jb - q.ja, kQtSlice); i < min(sk.jc - sk.ja, kQtSlice + kQtHaloCand); ++i) {
+    const int d = sm.klist[i] - hb0;
+    if (d >= 0 && d < kQtHaloCand) cand_kept |= 1u << d;
+  }
   group_sync(kConsumers);
   GroupLayout L{0, 0, 0u, 0};
-  bool active = false;
+  if (active) {
+    L.kmask = sm.gkmask[lane];
+    L.j0 = sm.gj0[lane];
+    L.n = 8 - __popc(L.kmask);
+    L.c0 = min(max(8 * g - L.j0, 0), Hr);
+  }
   float inv[8];
   int lo[8], hi[8];
   uint32_t mul[8], zbase = 0;
-  int slot = 0, sh = 0;
   // halo work: pair p = lane + 32c (c < kQtHaloSlots) is (row p / nhalo, halo feature p % nhalo);
   // h_pack = row | shift << 4 | zero << 9 | (column - ha) << 13 (row 8: no pair)
   uint32_t h_pack[kQtHaloSlots];
@@ -181,71 +253,73 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
 #pragma unroll
   for (int c = 0; c < kQtKeptSlots; ++c) {
     if (!k_generic && k_j + 4 * c < nk) {
-      const int col = checked_col(keep_idx, q.ja + k_j + 4 * c, H);
+      const int col = sm.klist[k_j + 4 * c];
       k_cols |= (uint32_t)min(max(col - q.ha, 0), kQtSlice - 1) << (8 * c);
     }
   }
+  // This lane's parameters for rank r: inv_scale, the clamp bounds -zero and 15-zero, the nibble
+  // multipliers and the zero points' packed sum.
+  auto set_rank = [&](const QtParams& pr) {
+    const float pinv[8] = {pr.i0.x, pr.i0.y, pr.i0.z, pr.i0.w, pr.i1.x, pr.i1.y, pr.i1.z, pr.i1.w};
+    zbase = 0;
+    int j = 0;
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    inv[e] = 0.0f;
-    lo[e] = hi[e] = 0;
-    mul[e] = 0u;
-  }
+    for (int e = 0; e < 8; ++e) {
+      const bool kept = (L.kmask >> e) & 1u;
+      const int z = (int)(((e < 4 ? pr.z.x : pr.z.y) >> (8 * (e & 3))) & 0xFFu);
+      inv[e] = pinv[e];
+      lo[e] = -z;
+      hi[e] = 15 - z;
+      mul[e] = (active && !kept) ? (1u << (4 * j)) : 0u;
+      j += kept ? 0 : 1;
+      zbase += (uint32_t)z * mul[e];
+    }
+  };
+  set_rank(pr);
+  const int slot = (L.c0 >> 3) - q.Wb + 1;
+  const int sh = 4 * (L.c0 & 7);
+  // Halo pairs: pair p = lane + 32c is (row p / nhalo, halo feature p % nhalo), the feature at
+  // compact position Cb + p % nhalo, whose column stays fixed for the launch; the first rank's
+  // parameters come from the lane that loaded that candidate (or from memory past the
+  // candidates).  h_pack = row | shift << 4 | zero << 9 | (column - ha) << 13 (row 8: no pair).
+  bool halo_staged = true;  // every halo feature lies in the staged columns [ha, ha + kQtBoxCols)
+  if (q.nhalo > 0)
+    halo_staged = qt_rest_col(q.nhalo - 1, hb0, cand_kept, keep_idx, k, sk.jc, H) < q.ha + kQtBoxCols;
 #pragma unroll
   for (int c = 0; c < kQtHaloSlots; ++c) {
-    h_pack[c] = kQtRowsPerWarp;  // no pair
+    const int p = lane + 32 * c;
+    const bool has = p < q.nhalo * kQtRowsPerWarp;
+    const int col = has ? qt_rest_col(p % q.nhalo, hb0, cand_kept, keep_idx, k, sk.jc, H) : hb0;
+    const int off = min(max(col - hb0, 0), kQtHaloCand - 1);
+    float c_inv = __shfl_sync(0xFFFFFFFFu, hc_inv, off);
+    uint32_t c_z = __shfl_sync(0xFFFFFFFFu, hc_z, off);
+    h_pack[c] = kQtRowsPerWarp;
     h_inv[c] = 0.0f;
+    if (has) {
+      if (col - hb0 >= kQtHaloCand) {
+        const size_t pp = (size_t)r * H + col;
+        c_inv = __ldg(inv_scale + pp);
+        c_z = __ldg(zero + pp);
+      }
+      const int row = p / q.nhalo, idx = p - row * q.nhalo;
+      h_inv[c] = c_inv;
+      h_pack[c] = (uint32_t)row | (uint32_t)(4 * ((q.Cb + idx) & 7)) << 4 | (c_z & 15u) << 9 |
+                  (uint32_t)(col - q.ha) << 13;
+    }
   }
   uint32_t(*buf)[kQtBufWords] = sm.buf[warp];
 
   for (int i = 0; i < n_units; ++i) {
-    if (i > 0 && ++b == NB) {
+    if (i > 0 && ++b == NB) {  // a new rank: this lane's parameters, and the halo features'
       b = 0;
-      fresh = true;
       ++r;
-    }
-    if (fresh) {  // new rank: this lane's parameters
-      fresh = false;
-      const int g = s * (kQtSlice / 8) + lane;
-      active = g < NG;
-      L = GroupLayout{0, 0, 0u, 0};
-      if (active) {
-        L.kmask = sm.gkmask[lane];
-        L.j0 = sm.gj0[lane];
-        L.n = 8 - __popc(L.kmask);
-        L.c0 = min(max(8 * g - L.j0, 0), Hr);
-      }
-      zbase = 0;
-      int j = 0;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const bool kept = (L.kmask >> e) & 1u;
-        int z = 0;
-        inv[e] = 0.0f;
-        if (active) {
-          const size_t p = (size_t)r * H + 8 * g + e;
-          z = zero[p];
-          inv[e] = inv_scale[p];
-        }
-        lo[e] = -z;
-        hi[e] = 15 - z;
-        mul[e] = (active && !kept) ? (1u << (4 * j)) : 0u;
-        j += kept ? 0 : 1;
-        zbase += (uint32_t)z * mul[e];
-      }
-      slot = (L.c0 >> 3) - q.Wb + 1;
-      sh = 4 * (L.c0 & 7);
+      set_rank(qt_load_params(inv_scale, zero, (size_t)r * H + 8 * g, active));
 #pragma unroll
       for (int c = 0; c < kQtHaloSlots; ++c) {
-        const int p = lane + 32 * c;
-        h_pack[c] = kQtRowsPerWarp;
-        if (p < q.nhalo * kQtRowsPerWarp) {
-          const int row = p / q.nhalo, idx = p - row * q.nhalo;
-          const int col = checked_col(rest_idx, q.Cb + idx, H);
-          const size_t pp = (size_t)r * H + col;
-          h_inv[c] = inv_scale[pp];
-          h_pack[c] = (uint32_t)row | (uint32_t)(4 * ((q.Cb + idx) & 7)) << 4 | (uint32_t)zero[pp] << 9 |
-                      (uint32_t)(col - q.ha) << 13;
+        if ((h_pack[c] & 15u) < kQtRowsPerWarp) {
+          const size_t pp = (size_t)r * H + q.ha + (h_pack[c] >> 13);
+          h_inv[c] = __ldg(inv_scale + pp);
+          h_pack[c] = (h_pack[c] & ~(15u << 9)) | ((uint32_t)__ldg(zero + pp) & 15u) << 9;
         }
       }
     }
@@ -282,7 +356,7 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
       if (h_row < nrows) {
         const int h_shift = (h_pack[c] >> 4) & 31u, h_z = (h_pack[c] >> 9) & 15u, h_off = h_pack[c] >> 13;
         uint32_t hb16;
-        if (q.halo_staged) {
+        if (halo_staged) {
           hb16 = (uint32_t)tile[(warp * kQtRowsPerWarp + h_row) * kQtBoxCols + h_off] << 16;
         } else {  // halo features spread beyond the staged columns: read them directly
           hb16 = (uint32_t)x[((size_t)r * T + t_base + h_row) * ldx + q.ha + h_off] << 16;
