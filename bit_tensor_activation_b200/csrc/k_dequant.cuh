@@ -546,12 +546,14 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
   DtSmem& sm = *reinterpret_cast<DtSmem*>(s_raw);
   float4* s_const = reinterpret_cast<float4*>(s_raw + ((sizeof(DtSmem) + 127) & ~size_t(127)));
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int s = blockIdx.x / chunks, chunk = blockIdx.x - s * chunks;
-  // the slice's row blocks split evenly over its `chunks` CTAs (counts differ by one at most)
+  // Slice-minor numbering (blockIdx = chunk*S + s): the S CTAs of one chunk are launched together.
+  // Chunk c of every slice takes the 32-row blocks c, c + chunks, c + 2*chunks, ..., so all CTAs
+  // sweep the rows from top to bottom together and counts differ by one block at most.
+  const int chunk = blockIdx.x / S, s = blockIdx.x - chunk * S;
   const int nb_all = (T + kDtTileRows - 1) / kDtTileRows;
-  const int b_first = (int)((long long)chunk * nb_all / chunks), b_end = (int)((long long)(chunk + 1) * nb_all / chunks);
-  const int t_first = b_first * kDtTileRows, t_last = min(T, b_end * kDtTileRows);
-  const int nblk = b_end - b_first;
+  const int nblk = (nb_all - chunk + chunks - 1) / chunks;
+  const int t_last = T;
+  auto block_row = [&](int bi) { return (chunk + bi * chunks) * kDtTileRows; };
   const int n_groups = (P + kDtG - 1) / kDtG;  // ring slots per block
   const int n_slots_total = nblk * n_groups;     // slot i = (block i / n_groups, rank group i % n_groups)
 
@@ -596,7 +598,7 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
         mbar_arrive_expect_tx(&sm.ring.full[st], (unsigned)nr * (kDtTileBytes + (stage_side ? kDtSideBytes : 0u)));
         for (int j = 0; j < nr; ++j) {
           const int r = r0 + j, m = wire.per_rank ? r : 0;
-          const int t = t_first + bi * kDtTileRows;
+          const int t = block_row(bi);
           tma_load_2d(&sm.tile[st][j][0][0], &wire.code[m], w_a, (wire.per_rank ? 0 : r * T) + t,
                       &sm.ring.full[st]);
           if (stage_side)
@@ -663,7 +665,7 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
   int st_i = 0;
   unsigned phase = 0;
   for (int bi = 0; bi < nblk && !*abort; ++bi) {
-    const int t0 = t_first + bi * kDtTileRows + warp * kDtR;
+    const int t0 = block_row(bi) + warp * kDtR;
     float acc[kDtR][8];
 #pragma unroll
     for (int m = 0; m < kDtR; ++m)

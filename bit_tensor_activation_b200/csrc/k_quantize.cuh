@@ -10,7 +10,10 @@
 // the ranges differ by at most one unit and a CTA changes rank at most a few times.  The CTAs of
 // the S slices that share j write the same rows of codes and side at about the same time: the
 // 32-byte sectors those rows share at slice boundaries are completed in L2 before eviction
-// instead of costing a read-modify-write in HBM each time.  In a CTA, warp 8 is the producer: one lane issues, per unit, one TMA load of a
+// instead of costing a read-modify-write in HBM each time.  Blocks are numbered slice-minor
+// (blockIdx = j*S + s), so the S CTAs of one j are launched together and land in the same round
+// of CTAs per SM; the first CTA resident on an SM gets more of its issue slots than the second,
+// and with slice-major numbering the slices sharing rows drifted apart by up to 15%.  In a CTA, warp 8 is the producer: one lane issues, per unit, one TMA load of a
 // 64-row tile of the slice's 256 features and the 8 after them (a box of 132 32-bit elements, so
 // the halo features below are staged too in the common case), into a 3-stage ring.  Warps 0..7
 // are consumers; warp w quantizes rows 8w..8w+7 of each tile, lane l the 8 features 8l..8l+7
@@ -142,7 +145,7 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
   extern __shared__ __align__(128) unsigned char s_raw[];
   QtSmem& sm = *reinterpret_cast<QtSmem*>(s_raw);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int s = blockIdx.x / J, j = blockIdx.x - s * J;
+  const int j = blockIdx.x / S, s = blockIdx.x - j * S;  // slice-minor numbering
   const int NB = (T + kQtTileRows - 1) / kQtTileRows;  // 64-row blocks per rank
   const long long U = (long long)P * NB;
   const int u0 = (int)(U * j / J), u1 = (int)(U * (j + 1) / J);
@@ -346,7 +349,7 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
           V += (uint32_t)c0 * mul[e] + (uint32_t)c1 * mul[e + 1];
         }
         atomicOr(&buf[m][slot], V << sh);
-        atomicOr(&buf[m][slot + 1], sh ? (V >> (32 - sh)) : 0u);
+        atomicOr(&buf[m][slot + 1], __funnelshift_l(V, 0u, sh));  // V >> (32 - sh), 0 when sh == 0
       }
     }
     // halo codes: features of the next slice completing this slice's last word
