@@ -165,9 +165,11 @@ struct WireSrc {
   bool per_rank = false;
 };
 
+// nbatch > 1: nbatch independent problems of P ranks each, stacked (problem b: ranks b*P .. b*P+P-1
+// of the wire and the parameters, output rows b*T .. b*T+T-1); one launch when TMA can stage them.
 template <typename OutT, bool kShard>
 hq_status launch_dequant(const WireSrc& src, int P, int T, int H, int k, const int32_t* keep_idx, const float* scale,
-                         const uint8_t* zero, void* out, int ldo, cudaStream_t st, DeviceInfo& d) {
+                         const uint8_t* zero, void* out, int ldo, cudaStream_t st, DeviceInfo& d, int nbatch = 1) {
   const int S = (H + 8 * hq::kDqSliceGroups - 1) / (8 * hq::kDqSliceGroups);
   const int Wr = (H - k) / 8;
   hq::DqWire wire;
@@ -179,11 +181,11 @@ hq_status launch_dequant(const WireSrc& src, int P, int T, int H, int k, const i
   bool side_tma = k > 0 && T % 8 == 0;
   if (!src.per_rank) {
     tma = tma && aligned(src.codes, 16) &&
-          encode_2d(&wire.code[0], src.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)Wr, (uint64_t)P * T,
-                    hq::kDtWords, hq::kDtTileRows);
+          encode_2d(&wire.code[0], src.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)Wr,
+                    (uint64_t)nbatch * P * T, hq::kDtWords, hq::kDtTileRows);
     side_tma = tma && side_tma &&
-               encode_2d(&wire.side[0], src.side, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)T, (uint64_t)P * k,
-                         hq::kDtTileRows, hq::kDtSideCols, CU_TENSOR_MAP_L2_PROMOTION_NONE);
+               encode_2d(&wire.side[0], src.side, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)T,
+                         (uint64_t)nbatch * P * k, hq::kDtTileRows, hq::kDtSideCols, CU_TENSOR_MAP_L2_PROMOTION_NONE);
   } else {
     for (int r = 0; r < P && tma; ++r)
       tma = encode_2d(&wire.code[r], src.codes_r[r], CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)Wr, (uint64_t)T,
@@ -192,7 +194,7 @@ hq_status launch_dequant(const WireSrc& src, int P, int T, int H, int k, const i
       side_tma = encode_2d(&wire.side[r], src.side_r[r], CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)T, (uint64_t)k,
                            hq::kDtTileRows, hq::kDtSideCols, CU_TENSOR_MAP_L2_PROMOTION_NONE);
     for (int r = 0; r < P; ++r) wire.side_ptr[r] = k > 0 ? src.side_r[r] : nullptr;
-    if (!tma) return HQ_ERR_INVALID_ARG;  // per-rank buffers are read by the TMA kernel only
+    if (!tma || nbatch != 1) return HQ_ERR_INVALID_ARG;  // per-rank buffers: TMA kernel, one problem
     side_tma = side_tma && tma;
   }
   constexpr int kF32 = std::is_same<OutT, float>::value ? 1 : 0;
@@ -203,11 +205,24 @@ hq_status launch_dequant(const WireSrc& src, int P, int T, int H, int k, const i
     if (occupancy(d.dequant_tma[kF32][kShard], kern, hq::kDtThreads, smem, P, &per_sm) != HQ_OK) return HQ_ERR_CUDA;
     // one wave: each slice's row blocks split evenly over as many CTAs as fit
     const long long nb_all = ceil_div(T, hq::kDtTileRows);
-    const int chunks = (int)std::max(1LL, std::min((long long)d.sms * per_sm / S, nb_all));
-    kern<<<(unsigned)(S * chunks), hq::kDtThreads, smem, st>>>(wire, side_tma ? 1 : 0, src.side, P, T, H, k,
-                                                                keep_idx, scale, zero, static_cast<OutT*>(out), ldo,
-                                                                S, chunks, wait_limits());
+    const int chunks = (int)std::max(1LL, std::min((long long)d.sms * per_sm / ((long long)S * nbatch), nb_all));
+    const dim3 grid((unsigned)(S * chunks), (unsigned)nbatch);
+    kern<<<grid, hq::kDtThreads, smem, st>>>(wire, side_tma ? 1 : 0, src.side, P, T, H, k, keep_idx, scale, zero,
+                                             static_cast<OutT*>(out), ldo, S, chunks, wait_limits());
     return launched();
+  }
+  if (nbatch > 1) {  // the cp.async kernel takes one problem per launch
+    const int Wr2 = (H - k) / 8;
+    for (int b = 0; b < nbatch; ++b) {
+      WireSrc one;
+      one.codes = src.codes ? src.codes + (size_t)b * P * T * Wr2 : nullptr;
+      one.side = src.side ? src.side + (size_t)b * P * k * T : nullptr;
+      const hq_status r = launch_dequant<OutT, kShard>(one, P, T, H, k, keep_idx, scale + (size_t)b * P * H,
+                                                       zero + (size_t)b * P * H,
+                                                       static_cast<OutT*>(out) + (size_t)b * T * ldo, ldo, st, d, 1);
+      if (r != HQ_OK) return r;
+    }
+    return HQ_OK;
   }
   const size_t smem = hq::dq_smem_bytes(P);
   auto kern = hq::dequant_reduce_kernel<OutT, kShard>;
@@ -428,8 +443,9 @@ hq_status two_step_entry(const uint16_t* x, int P, int T, int H, int k, const in
     return HQ_ERR_INVALID_ARG;  // H % 16: every reducer's row of zero2 starts on a 16-byte boundary
   if (out_dtype != HQ_OUT_BF16 && out_dtype != HQ_OUT_F32) return HQ_ERR_INVALID_ARG;
   if (!scale2 || !inv_scale2 || !zero2 || (k2 > 0 && !keep2) || (k2 < H && !rest2)) return HQ_ERR_INVALID_ARG;
+  if (T > 0 && !out) return HQ_ERR_INVALID_ARG;
   if (!aligned(scale2, 16) || !aligned(inv_scale2, 16) || !aligned(zero2, 16) || !aligned(keep2, 4) ||
-      !aligned(rest2, 4))
+      !aligned(rest2, 4) || !aligned(out, 16))
     return HQ_ERR_MISALIGNED;
   if (T == 0) return HQ_OK;
   const TwoStepLayout L = two_step_layout(P, T, H, k, k2);
@@ -446,20 +462,22 @@ hq_status two_step_entry(const uint16_t* x, int P, int T, int H, int k, const in
   if (st != HQ_OK) return st;
   st = dequant_entry<false>(codes, side, P, T, H, k, keep_idx, rest_idx, scale, zero, red, H, HQ_OUT_BF16, stream);
   if (st != HQ_OK) return st;
-  // step 2: reducer j re-quantizes its row block with grid row j; the block is dequantized with it
+  // step 2: reducer j re-quantizes its row block with grid row j, and the block is dequantized
+  // with it.  The reduced tensor [T][H] is [P][T/P][H]: reducer j's block is "rank" j of one
+  // quantize-pack call (whose output layout is exactly the P step-2 wires, block after block),
+  // and the P blocks are P independent one-rank problems of one batched dequant-reduce launch.
   const int Tb = T / P;
-  const size_t esz = out_dtype == HQ_OUT_F32 ? 4 : 2;
-  for (int j = 0; j < P; ++j) {
-    uint32_t* cj = codes2 + (size_t)j * Tb * ((H - k2) / 8);
-    uint16_t* sj = side2 + (size_t)j * k2 * Tb;
-    st = quantize_entry(red + (size_t)j * Tb * H, H, 1, Tb, H, k2, keep2, rest2, inv_scale2 + (size_t)j * H,
-                        zero2 + (size_t)j * H, cj, sj, stream);
-    if (st != HQ_OK) return st;
-    st = dequant_entry<false>(cj, sj, 1, Tb, H, k2, keep2, rest2, scale2 + (size_t)j * H, zero2 + (size_t)j * H,
-                              static_cast<char*>(out) + (size_t)j * Tb * H * esz, H, out_dtype, stream);
-    if (st != HQ_OK) return st;
-  }
-  return HQ_OK;
+  st = quantize_entry(red, H, P, Tb, H, k2, keep2, rest2, inv_scale2, zero2, codes2, side2, stream);
+  if (st != HQ_OK) return st;
+  if (Tb == 0) return HQ_OK;
+  DeviceInfo* d = nullptr;
+  if (device_info(&d) != HQ_OK) return HQ_ERR_CUDA;
+  WireSrc src;
+  src.codes = codes2;
+  src.side = side2;
+  if (out_dtype == HQ_OUT_BF16)
+    return launch_dequant<uint16_t, false>(src, 1, Tb, H, k2, keep2, scale2, zero2, out, H, (cudaStream_t)stream, *d, P);
+  return launch_dequant<float, false>(src, 1, Tb, H, k2, keep2, scale2, zero2, out, H, (cudaStream_t)stream, *d, P);
 }
 
 // Scratch of hq_two_step_reduce_noalloc: a fixed array in every device's global memory, so that a

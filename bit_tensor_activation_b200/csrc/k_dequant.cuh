@@ -550,6 +550,12 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
   // Chunk c of every slice takes the 32-row blocks c, c + chunks, c + 2*chunks, ..., so all CTAs
   // sweep the rows from top to bottom together and counts differ by one block at most.
   const int chunk = blockIdx.x / S, s = blockIdx.x - chunk * S;
+  // Problem blockIdx.y of a batch (gridDim.y is 1 for a single problem): ranks [y*P, (y+1)*P) of
+  // the stacked wire, their parameters, and its own T output rows.
+  const int rank0 = blockIdx.y * P;
+  scale += (size_t)rank0 * H;
+  zero += (size_t)rank0 * H;
+  out += (size_t)blockIdx.y * T * ldo;
   const int nb_all = (T + kDtTileRows - 1) / kDtTileRows;
   const int nblk = (nb_all - chunk + chunks - 1) / chunks;
   const int t_last = T;
@@ -599,10 +605,10 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
         for (int j = 0; j < nr; ++j) {
           const int r = r0 + j, m = wire.per_rank ? r : 0;
           const int t = block_row(bi);
-          tma_load_2d(&sm.tile[st][j][0][0], &wire.code[m], w_a, (wire.per_rank ? 0 : r * T) + t,
+          tma_load_2d(&sm.tile[st][j][0][0], &wire.code[m], w_a, (wire.per_rank ? 0 : (rank0 + r) * T) + t,
                       &sm.ring.full[st]);
           if (stage_side)
-            tma_load_2d(&sm.side[st][j][0][0], &wire.side[m], t, (wire.per_rank ? 0 : r * k) + q.ja,
+            tma_load_2d(&sm.side[st][j][0][0], &wire.side[m], t, (wire.per_rank ? 0 : (rank0 + r) * k) + q.ja,
                         &sm.ring.full[st]);
         }
         ++issued;
@@ -698,8 +704,8 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
       if (lane == 0) mbar_arrive(&sm.ksum_empty[buf]);
       dq_store_rows<OutT, kDtR>(D, acc, ldo, t0, t_last, out);
     } else {
-      dq_finish_block<OutT, kDtR, false>(D, acc, side, wire.per_rank ? wire.side_ptr : nullptr, sm.k.kept[warp], P,
-                                         T, H, k, q.ja, q.jb, t0, t_last, out, ldo);
+      dq_finish_block<OutT, kDtR, false>(D, acc, side + (size_t)rank0 * k * T, wire.per_rank ? wire.side_ptr : nullptr,
+                                         sm.k.kept[warp], P, T, H, k, q.ja, q.jb, t0, t_last, out, ldo);
     }
   }
 }

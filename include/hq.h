@@ -218,8 +218,11 @@ hq_status hq_compress_reduce_ld(const uint16_t* x, int ldx, int P, int T, int H,
  *                         the reduced tensor and the step-2 wires (its contents are scratch)
  *   out                   [T][H], bf16 or fp32
  *   T % P == 0 and H % 16 == 0 (every reducer's row of zero2 then starts on a 16-byte boundary).
- * Enqueues 2 + 2P kernels on `stream`.  Errors as in the calls above; a workspace that is NULL or
- * too small is HQ_ERR_INVALID_ARG, one below 256-byte alignment HQ_ERR_MISALIGNED.
+ * Enqueues 4 kernels on `stream`: step 2's P blocks are one quantize-pack over P "ranks" of T/P
+ * rows and one dequant-reduce launch over P independent one-rank problems (when H - k2 is not a
+ * multiple of 32 its code rows cannot be staged by TMA, and that dequant is one launch per block).
+ * Errors as in the calls above, all checked before anything is enqueued; a workspace that is NULL
+ * or too small is HQ_ERR_INVALID_ARG, one below 256-byte alignment HQ_ERR_MISALIGNED.
  */
 hq_status hq_two_step_reduce(const uint16_t* x, int P, int T, int H, int k, const int32_t* keep_idx,
                              const int32_t* rest_idx, const float* scale, const float* inv_scale, const uint8_t* zero,

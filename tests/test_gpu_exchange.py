@@ -90,10 +90,13 @@ def _oracle_step_two(o, cal, sel, ref, cfg, k2):
     return p2, np.concatenate(out)
 
 
-def test_two_step_loopback_and_simulated():
+# k2 = 64: step-2 code rows of 504 words, staged by TMA (one batched dequant launch); k2 = 16:
+# rows of 510 words, which TMA cannot stage (the cp.async kernel, one launch per reducer block)
+@pytest.mark.parametrize("k2", [64, 16])
+def test_two_step_loopback_and_simulated(k2):
     cfg = CFG.with_(calib_T=64)
     o, cal, sel, x, ref, params = _setup(cfg)
-    P, T, H, Tb, k2 = cfg.P, cfg.T, cfg.H, cfg.T // cfg.P, 64
+    P, T, H, Tb = cfg.P, cfg.T, cfg.H, cfg.T // cfg.P
     p2_ref, want = _oracle_step_two(o, cal, sel, ref, cfg, k2)
     # step-2 grids on the GPU from the same calibration batches
     p2 = ex.step_two_params_simulated([to_dev_u16(c).view(torch.bfloat16) for c in cal], params, k2, cfg.beta)
