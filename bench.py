@@ -49,6 +49,8 @@ def parse_args():
     ap.add_argument("--cold-reps", type=int, default=20, help="launches of each kernel timed alone, L2 flushed")
     ap.add_argument("--second-steps", type=int, default=400,
                     help="timed steps of the second large workload (0: skip it)")
+    ap.add_argument("--small-steps", type=int, default=200,
+                    help="timed steps of each of the two small workloads, decode and pr1 (0: skip them)")
     ap.add_argument("--no-next", dest="next_paths", action="store_false",
                     help="skip the two-step, partial-sync and per-rank-buffer measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -671,6 +673,22 @@ def run_hq(args, cfg, world, rank, local):
         if st != hq.HQ_OK:
             raise RuntimeError(f"device error ({second}): {hq.hq_status_string(st)}")
         del W2
+    # the two small workloads (launch-bound: reported for coverage of every configuration)
+    if args.small_steps > 0 and world == 1:
+        for small in ("decode", "pr1"):
+            if small == cfg.name:
+                continue
+            cfg3 = workload(small)
+            W3 = Workload(cfg3, dev)
+            m = measure_workload(W3, args.small_steps, 5, args.cold_reps, stream, flush, peak)
+            m["config"] = describe(cfg3)
+            m["compression_ratio"] = compression_ratio(cfg3)
+            m["elements_per_s"] = cfg3.P * cfg3.T * cfg3.H / (m["split_ms"] * 1e-3)
+            workloads[small] = m
+            st = hq.hq_read_device_error()
+            if st != hq.HQ_OK:
+                raise RuntimeError(f"device error ({small}): {hq.hq_status_string(st)}")
+            del W3
 
     # ---- CPU baseline (rank 0, N = 1) -----------------------------------------------------------
     cpu = None

@@ -135,6 +135,41 @@ def test_kept_counts_per_slice_bit_exact(P, T):
     assert_same(u16(lit), lit_r, "bf16-shard reduction")
 
 
+@pytest.mark.parametrize("T", [40, 37])
+def test_halo_past_the_preloaded_candidates(T):
+    """Slice 0 keeps 7 features, so its last code word needs the next 7 non-kept features (the
+    halo); slice 1 starts with 12 kept features, so 3 of those halo features lie beyond the 16
+    features after the slice whose parameters quantize-pack preloads (found by walking keep_idx)
+    and beyond the 8 columns it stages (read from x directly).  Codes, side and output bit-exact."""
+    o = oracle.get()
+    P, H = 3, 1024
+    big = np.array(sorted([3, 40, 77, 120, 160, 200, 250] + list(range(256, 268)) + [300, 333, 500, 640, 900]))
+    k = len(big)
+    assert k % 8 == 0
+    rng = np.random.default_rng(13)
+    x = synth.fill_cpu(synth.CONFIGS["decode"].with_(P=P, T=T, H=H, n_out=4), synth.EVAL, 0, cs=np.ones(H))
+    emin = -np.ones((P, H), np.float32) - rng.uniform(0, 0.01, (P, H)).astype(np.float32)
+    emax = np.ones((P, H), np.float32)
+    emax[:, big] = 40.0
+    sel = o.select_topk(emin, emax, k)
+    assert np.array_equal(sel["keep_idx"], big)
+    Cb = 256 - 7  # compact position of slice 0's first halo feature
+    assert (8 - Cb % 8) % 8 == 7 and sel["rest_idx"][Cb + 6] == 274  # the last one is past 256 + 16
+    prm = params_to_dev(sel)
+    codes_r, side_r = o.quantize_pack(x, sel["keep_idx"], sel["rest_idx"], sel["inv_scale"], sel["zero"])
+    out_r = o.dequant_reduce(codes_r, side_r, H, sel["keep_idx"], sel["rest_idx"], sel["scale"], sel["zero"])
+    codes, side = gpu_quantize(to_dev_u16(x), prm)
+    out = gpu_dequant(codes, side, prm, H)
+    fused, fcodes, fside = gpu_fused(to_dev_u16(x), prm, wire=True)
+    assert_no_device_error()
+    assert_same(u32(codes), codes_r, "codes")
+    assert_same(u16(side), side_r, "side")
+    assert_same(u16(out), out_r, "out")
+    assert_same(u16(fused), out_r, "fused")
+    assert_same(u32(fcodes), codes_r, "fused codes")
+    assert_same(u16(fside), side_r, "fused side")
+
+
 def test_select_ties_and_special_values():
     o = oracle.get()
     P, H = 3, 4096
