@@ -28,10 +28,12 @@
 //
 // Ownership of compact words: a slice owns the words whose first nibble one of its groups
 // produces; it drops nibbles that fall into the previous slice's last word and completes its own
-// last word from the next <= 7 non-kept features of the next slice (the "halo", read through
-// rest_idx, spread over the lanes as (row, feature) pairs; read from the staged tile when they lie
-// within its 8 extra columns, else from global memory).  So every codes word is written by
-// exactly one CTA.  Kept values are copied from the staged tile to the side buffer.
+// last word from the next <= 7 non-kept features of the next slice (the "halo": their columns
+// come from the kept list, rest_idx being the complement of keep_idx; they are spread over the
+// lanes as (row, feature) pairs and read from the staged tile when they lie within its 8 extra
+// columns, else from global memory).  So every codes word is written by
+// exactly one CTA.  Kept values are copied from the staged tile to the side buffer (16 bytes per
+// kept feature and warp when T % 8 == 0).
 //
 // Roofline: HBM-bound; 2 bytes read + 0.5 byte written per non-kept element, 2 + 2 per kept one.
 // No memory beyond the inputs and outputs is used.
@@ -242,11 +244,14 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
   // h_pack = row | shift << 4 | zero << 9 | (column - ha) << 13 (row 8: no pair)
   uint32_t h_pack[kQtHaloSlots];
   float h_inv[kQtHaloSlots];
-  // kept copies: pair p = lane + 32c (c < kQtKeptSlots) is (row lane % 8, kept feature
-  // lane / 8 + 4c), present while lane / 8 + 4c < nk; byte c of k_cols = its column - ha.  The
-  // side buffer is feature-major, side[r][j][t]: the pair's element, counted from the unit's
-  // rank and the warp's first row, is k_side0 + 4c*T, and the 8 rows of one kept feature are
-  // contiguous (the CTA's warps fill 128 contiguous bytes per kept feature and tile).
+  // Kept copies.  The side buffer is feature-major, side[r][j][t], so the warp's 8 rows of one
+  // kept feature are 16 contiguous bytes (the CTA's warps fill 128 per kept feature and tile).
+  // When they are 16-byte aligned (T % 8 == 0) and the slice has at most 32 kept features, lane
+  // j copies kept feature j with one 16-byte store (k_vcol = its column - ha).  Otherwise, for a
+  // slice with at most kQtMaxFastKept: pair p = lane + 32c (c < kQtKeptSlots) is (row lane % 8,
+  // kept feature lane / 8 + 4c), present while lane / 8 + 4c < nk, byte c of k_cols = its column
+  // - ha, and the pair's element counted from the unit's rank and the warp's first row is
+  // k_side0 + 4c*T; more kept features are copied in a loop.
   const int nk = q.jb - q.ja;
   const bool k_generic = nk > kQtMaxFastKept;
   const int k_m = lane % kQtRowsPerWarp, k_j = lane / kQtRowsPerWarp;
@@ -260,6 +265,8 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
       k_cols |= (uint32_t)min(max(col - q.ha, 0), kQtSlice - 1) << (8 * c);
     }
   }
+  const bool k_vec = (T % 8) == 0 && nk <= 32;
+  const int k_vcol = lane < nk ? min(max(sm.klist[lane] - q.ha, 0), kQtSlice - 1) : 0;
   // This lane's parameters for rank r: inv_scale, the clamp bounds -zero and 15-zero, the nibble
   // multipliers and the zero points' packed sum.
   auto set_rank = [&](const QtParams& pr) {
@@ -371,7 +378,17 @@ __global__ void __launch_bounds__(kQtThreads, 2) quantize_pack_tma_kernel(
     }
     // kept values straight from the staged tile
     uint16_t* srow = side + (size_t)r * k * T + t_base;
-    if (!k_generic) {
+    if (k_vec && nrows == kQtRowsPerWarp) {
+      if (lane < nk) {
+        const uint16_t* tc = tile + (warp * kQtRowsPerWarp) * kQtBoxCols + k_vcol;
+        uint4 v;
+        v.x = (uint32_t)tc[0] | (uint32_t)tc[kQtBoxCols] << 16;
+        v.y = (uint32_t)tc[2 * kQtBoxCols] | (uint32_t)tc[3 * kQtBoxCols] << 16;
+        v.z = (uint32_t)tc[4 * kQtBoxCols] | (uint32_t)tc[5 * kQtBoxCols] << 16;
+        v.w = (uint32_t)tc[6 * kQtBoxCols] | (uint32_t)tc[7 * kQtBoxCols] << 16;
+        *reinterpret_cast<uint4*>(srow + (size_t)(q.ja + lane) * T) = v;
+      }
+    } else if (!k_generic) {
 #pragma unroll
       for (int c = 0; c < kQtKeptSlots; ++c)
         if (k_j + 4 * c < nk && k_m < nrows)
