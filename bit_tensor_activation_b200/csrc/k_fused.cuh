@@ -33,12 +33,63 @@ constexpr int kFuSlice = 256;
 constexpr int kFuStages = 3;
 constexpr unsigned kFuTileBytes = kFuTileRows * kFuSlice * 2;
 
+constexpr int kFuStartBarrier = 2;  // named barrier: consumers' set-up loads issued
+
 struct FuSmem {
   alignas(128) uint16_t tile[kFuStages][kFuTileRows][kFuSlice];
   TmaRing<kFuStages> ring;
   int abort;
+  int klist[kFuSlice];  // the slice's kept features
+  int kcnt[3];
+  uint32_t gkmask[kFuSlice / 8];
   // followed by the constants: float4 [P][5][32]
 };
+
+// One (rank, group) pair's parameters, idx = rank * 32 + group of the slice starting at hs,
+// loaded ahead of the rest of the set-up (nothing in the address depends on the kept features).
+struct FuPair {
+  float4 i0, i1, s0, s1;
+  uint2 z;
+};
+__device__ __forceinline__ FuPair fu_load_pair(const float* __restrict__ inv_scale, const float* __restrict__ scale,
+                                               const uint8_t* __restrict__ zero, int P, int H, int hs, int idx) {
+  FuPair d;
+  d.i0 = d.i1 = d.s0 = d.s1 = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  d.z = make_uint2(0u, 0u);
+  const int r = idx >> 5, hg = hs + 8 * (idx & 31);
+  if (r < P && hg < H) {  // r*H + hg is a multiple of 8; the arrays are 16-byte aligned
+    const size_t p = (size_t)r * H + hg;
+    d.i0 = __ldg(reinterpret_cast<const float4*>(inv_scale + p));
+    d.i1 = __ldg(reinterpret_cast<const float4*>(inv_scale + p) + 1);
+    d.s0 = __ldg(reinterpret_cast<const float4*>(scale + p));
+    d.s1 = __ldg(reinterpret_cast<const float4*>(scale + p) + 1);
+    d.z = __ldg(reinterpret_cast<const uint2*>(zero + p));
+  }
+  return d;
+}
+// The pair's constants: inv 0-3, inv 4-7, scale 0-3, scale 4-7 (1 for kept), (-zero as signed
+// bytes, kmask); features past H get zeros.
+__device__ __forceinline__ void fu_fill_pair(float4* s_const, const FuPair& d, uint32_t km, int H, int hs, int idx) {
+  const int r = idx >> 5, g = idx & 31;
+  const bool in = hs + 8 * g < H;
+  const float sv[8] = {d.s0.x, d.s0.y, d.s0.z, d.s0.w, d.s1.x, d.s1.y, d.s1.z, d.s1.w};
+  float sc[8];
+  uint32_t zlo = 0, zhi = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    sc[i] = !in ? 0.0f : ((km >> i) & 1u) ? 1.0f : sv[i];
+    const uint32_t zi = ((i < 4 ? d.z.x : d.z.y) >> (8 * (i & 3))) & 0xFFu;
+    const uint32_t nz = (uint32_t)(-(int)zi) & 0xFFu;  // -zero as a signed byte
+    if (i < 4) zlo |= nz << (8 * i);
+    else zhi |= nz << (8 * (i - 4));
+  }
+  float4* dst = s_const + (size_t)r * 5 * 32 + g;
+  dst[0] = d.i0;
+  dst[32] = d.i1;
+  dst[64] = make_float4(sc[0], sc[1], sc[2], sc[3]);
+  dst[96] = make_float4(sc[4], sc[5], sc[6], sc[7]);
+  dst[128] = make_float4(__uint_as_float(zlo), __uint_as_float(zhi), __uint_as_float(in ? km : 0u), 0.0f);
+}
 
 inline size_t fu_smem_bytes(int P) { return sizeof(FuSmem) + 128 + (size_t)P * 5 * 32 * 16; }
 
@@ -62,15 +113,15 @@ __global__ void __launch_bounds__(kFuThreads, 2) compress_reduce_kernel(
     sm.ring.init(kFuWarps);
     sm.abort = 0;
     fence_barrier_init();
-    // an index outside [0, H) belongs to no slice's groups: the end slices look for one
-    if (k > 0 && ((s == 0 && keep_idx[0] < 0) || (s == S - 1 && keep_idx[k - 1] >= H)))
-      record_error(HQ_ERR_BAD_INDEX);
   }
   __syncthreads();
   volatile int* abort = &sm.abort;
   constexpr int kConsumers = 32 * kFuWarps;
 
   if (warp == kFuWarps) {  // ------------------------------------------------ producer
+    // the first tiles go out after the consumers' set-up loads, which then are not queued
+    // behind them; the consumers arrive on this barrier before they wait for anything
+    named_barrier_sync_id(kFuStartBarrier, kFuThreads);
     if (lane == 0) {
       prefetch_tensor_map(&tmap_x);
       producer_start_delay(lim.start_delay);
@@ -92,35 +143,26 @@ __global__ void __launch_bounds__(kFuThreads, 2) compress_reduce_kernel(
   }
 
   // ---------------------------------------------------------------------- consumers
-  // constants [P][5][32]: inv 0-3, inv 4-7, scale 0-3, scale 4-7 (1 for kept), (-zero as signed bytes, kmask),
-  // filled while the producer is already loading
-  for (int idx = threadIdx.x; idx < P * 32; idx += kConsumers) {
-    const int r = idx >> 5, g = idx & 31;
-    const int hg = hs + 8 * g;
-    float iv[8], sc[8];
-    uint32_t zlo = 0, zhi = 0, km = 0;
-    if (hg < H) {
-      km = group_layout(keep_idx, k, H, hg).kmask;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const size_t p = (size_t)r * H + hg + i;
-        iv[i] = inv_scale[p];
-        sc[i] = ((km >> i) & 1u) ? 1.0f : scale[p];
-        const uint32_t nz = (uint32_t)(-(int)zero[p]) & 0xFFu;  // -zero as a signed byte
-        if (i < 4) zlo |= nz << (8 * i);
-        else zhi |= nz << (8 * (i - 4));
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) iv[i] = sc[i] = 0.0f;
-    }
-    float4* dst = s_const + (size_t)r * 5 * 32 + g;
-    dst[0] = make_float4(iv[0], iv[1], iv[2], iv[3]);
-    dst[32] = make_float4(iv[4], iv[5], iv[6], iv[7]);
-    dst[64] = make_float4(sc[0], sc[1], sc[2], sc[3]);
-    dst[96] = make_float4(sc[4], sc[5], sc[6], sc[7]);
-    dst[128] = make_float4(__uint_as_float(zlo), __uint_as_float(zhi), __uint_as_float(km), 0.0f);
+  // Set-up loads first, independent of one another so that they cost one round trip together:
+  // each thread's (rank, group) pair of parameters and one keep_idx entry.  Then the slice's
+  // kept features are counted in one coalesced pass and the groups' kept masks laid out from
+  // that list, and the constants [P][5][32] filled.
+  const FuPair pre = fu_load_pair(inv_scale, scale, zero, P, H, hs, threadIdx.x);
+  const int kv0 = (int)threadIdx.x < k ? __ldg(keep_idx + threadIdx.x) : 0x7FFFFFFF;
+  named_barrier_arrive_id(kFuStartBarrier, kFuThreads);
+  const int he = min(H, hs + kFuSlice);
+  const SliceKept3 sk = slice_kept3(kv0, keep_idx, k, hs, he, he, sm.kcnt, sm.klist, kFuSlice, kConsumers);
+  // an index outside [0, H) belongs to no slice's groups: the end slices find it missing
+  if (threadIdx.x == 0 && ((s == 0 && sk.ja != 0) || (s == S - 1 && sk.jb != k) || sk.jb - sk.ja > kFuSlice))
+    record_error(HQ_ERR_BAD_INDEX);
+  if (warp == 0) {
+    const int hg = hs + 8 * lane;
+    sm.gkmask[lane] = hg < H ? group_layout_list(sm.klist, min(sk.jb - sk.ja, kFuSlice), sk.ja, H, k, hg).kmask : 0u;
   }
+  named_barrier_sync(kConsumers);
+  if ((int)threadIdx.x < P * 32) fu_fill_pair(s_const, pre, sm.gkmask[threadIdx.x & 31], H, hs, threadIdx.x);
+  for (int idx = threadIdx.x + kConsumers; idx < P * 32; idx += kConsumers)
+    fu_fill_pair(s_const, fu_load_pair(inv_scale, scale, zero, P, H, hs, idx), sm.gkmask[idx & 31], H, hs, idx);
   named_barrier_sync(kConsumers);
   const int h0 = hs + 8 * lane;
   const bool active = h0 < H;
