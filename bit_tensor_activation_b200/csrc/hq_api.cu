@@ -249,10 +249,11 @@ hq_status launch_fused(const uint16_t* x, int ldx, int P, int T, int H, int k, c
   int per_sm = 0;
   if (occupancy(d.fused[std::is_same<OutT, float>::value ? 1 : 0], kern, hq::kFuThreads, smem, P, &per_sm) != HQ_OK)
     return HQ_ERR_CUDA;
-  int chunks, rpc;
-  slice_chunks(T, S, (long long)d.sms * per_sm, hq::kFuTileRows, &chunks, &rpc);
+  // one wave: as many row chunks per slice as the resident CTAs allow, at most one per 32-row block
+  const int nb_all = (T + hq::kFuTileRows - 1) / hq::kFuTileRows;
+  const int chunks = std::max(1, std::min(d.sms * per_sm / S, nb_all));
   kern<<<(unsigned)(S * chunks), hq::kFuThreads, smem, st>>>(map, P, T, H, k, keep_idx, scale, inv_scale, zero,
-                                                              static_cast<OutT*>(out), ldo, S, chunks, rpc,
+                                                              static_cast<OutT*>(out), ldo, S, chunks,
                                                               wait_limits());
   return launched();
 }

@@ -9,8 +9,8 @@
 // float(c) is formed without a conversion instruction: the bits c + 0x4B400000 are the float
 // 1.5*2^23 + c, from which 1.5*2^23 is subtracted exactly.
 //
-// Work decomposition as in dequant-reduce: a CTA covers a slice of 256 features and a range of
-// rows; its per-(rank, feature) constants live in shared memory.  Warp 8 is the producer: one
+// Work decomposition as in dequant-reduce: a CTA covers a slice of 256 features and every
+// chunks-th 32-row block; its per-(rank, feature) constants live in shared memory.  Warp 8 is the producer: one
 // lane loads, per (32-row block, rank), the 32 x 256 bf16 tile (16 KB) with one TMA instruction
 // into a 3-stage mbarrier ring.  Warps 0..7 consume 4 rows each (lane l: features 8l..8l+7),
 // walking the ranks in order with 4 x 8 fp32 sums in registers.
@@ -98,14 +98,18 @@ __global__ void __launch_bounds__(kFuThreads, 2) compress_reduce_kernel(
     const __grid_constant__ CUtensorMap tmap_x, int P, int T, int H, int k,
     const int32_t* __restrict__ keep_idx, const float* __restrict__ scale,
     const float* __restrict__ inv_scale, const uint8_t* __restrict__ zero, OutT* __restrict__ out, int ldo, int S,
-    int chunks, int rows_per_chunk, WaitLimits lim) {
+    int chunks, WaitLimits lim) {
   extern __shared__ __align__(128) unsigned char s_raw[];
   FuSmem& sm = *reinterpret_cast<FuSmem*>(s_raw);
   float4* s_const = reinterpret_cast<float4*>(s_raw + ((sizeof(FuSmem) + 127) & ~size_t(127)));
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int s = blockIdx.x / chunks, chunk = blockIdx.x - s * chunks;
-  const int t_first = chunk * rows_per_chunk, t_last = min(T, t_first + rows_per_chunk);
-  const int nblk = (t_last - t_first + kFuTileRows - 1) / kFuTileRows;
+  // Slice-minor numbering (blockIdx = chunk*S + s), and chunk c of every slice takes the 32-row
+  // blocks c, c + chunks, c + 2*chunks, ...: as in dequant-reduce, the CTAs sweep the rows
+  // together and their block counts differ by one at most.
+  const int chunk = blockIdx.x / S, s = blockIdx.x - chunk * S;
+  const int nb_all = (T + kFuTileRows - 1) / kFuTileRows;
+  const int nblk = (nb_all - chunk + chunks - 1) / chunks;
+  auto block_row = [&](int bi) { return (chunk + bi * chunks) * kFuTileRows; };
   const int n_tiles = nblk * P;  // tile i = (block i / P, rank i % P)
   const int hs = s * kFuSlice;
 
@@ -130,7 +134,7 @@ __global__ void __launch_bounds__(kFuThreads, 2) compress_reduce_kernel(
         if (!sm.ring.acquire(i, abort, lim.producer)) break;
         const int st = i % kFuStages;
         mbar_arrive_expect_tx(&sm.ring.full[st], kFuTileBytes);
-        tma_load_2d(&sm.tile[st][0][0], &tmap_x, hs, r * T + t_first + bi * kFuTileRows, &sm.ring.full[st]);
+        tma_load_2d(&sm.tile[st][0][0], &tmap_x, hs, r * T + block_row(bi), &sm.ring.full[st]);
         ++issued;
         if (++r == P) {
           r = 0;
@@ -170,7 +174,7 @@ __global__ void __launch_bounds__(kFuThreads, 2) compress_reduce_kernel(
   int st_i = 0;  // ring stage of the next tile and the parity of its fill
   unsigned phase = 0;
   for (int bi = 0; bi < nblk && !*abort; ++bi) {
-    const int t0 = t_first + bi * kFuTileRows + warp * kFuR;
+    const int t0 = block_row(bi) + warp * kFuR;
     float acc[kFuR][8];
 #pragma unroll
     for (int m = 0; m < kFuR; ++m)
@@ -227,7 +231,7 @@ __global__ void __launch_bounds__(kFuThreads, 2) compress_reduce_kernel(
     if (active) {
 #pragma unroll
       for (int m = 0; m < kFuR; ++m)
-        if (t0 + m < t_last) store_row8<OutT>(out + (size_t)(t0 + m) * ldo + h0, acc[m]);
+        if (t0 + m < T) store_row8<OutT>(out + (size_t)(t0 + m) * ldo + h0, acc[m]);
     }
   }
 }
