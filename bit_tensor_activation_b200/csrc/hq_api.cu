@@ -144,7 +144,19 @@ hq::WaitLimits wait_limits() {
 
 long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
 
-// Slices x row chunks for the dequant-reduce and fused kernels: one wave of CTAs at most.
+// One wave of `resident` CTAs over S slices of nb_all row blocks each: every slice gets `base`
+// row chunks and slices 0..extra-1 one more; never more chunks than blocks, at least one.
+struct WaveChunks {
+  int base, extra;
+};
+WaveChunks wave_chunks(long long resident, int S, long long nb_all) {
+  long long base = resident / S, extra = resident - base * S;
+  if (base < 1) base = 1, extra = 0;
+  if (base >= nb_all) base = std::max(nb_all, 1LL), extra = 0;
+  return WaveChunks{(int)base, (int)extra};
+}
+
+// Slices x row chunks of the cp.async dequant-reduce kernel: one wave of CTAs at most.
 void slice_chunks(int T, int S, long long resident, int rows_per_block, int* chunks, int* rows_per_chunk) {
   long long c = resident / S;
   if (c < 1) c = 1;
@@ -203,12 +215,12 @@ hq_status launch_dequant(const WireSrc& src, int P, int T, int H, int k, const i
     auto kern = hq::dequant_reduce_tma_kernel<OutT, kShard>;
     int per_sm = 0;
     if (occupancy(d.dequant_tma[kF32][kShard], kern, hq::kDtThreads, smem, P, &per_sm) != HQ_OK) return HQ_ERR_CUDA;
-    // one wave: each slice's row blocks split evenly over as many CTAs as fit
+    // one wave that fills every resident CTA slot (wave_chunks)
     const long long nb_all = ceil_div(T, hq::kDtTileRows);
-    const int chunks = (int)std::max(1LL, std::min((long long)d.sms * per_sm / ((long long)S * nbatch), nb_all));
-    const dim3 grid((unsigned)(S * chunks), (unsigned)nbatch);
+    const WaveChunks wc = wave_chunks((long long)d.sms * per_sm / nbatch, S, nb_all);
+    const dim3 grid((unsigned)(S * wc.base + wc.extra), (unsigned)nbatch);
     kern<<<grid, hq::kDtThreads, smem, st>>>(wire, side_tma ? 1 : 0, src.side, P, T, H, k, keep_idx, scale, zero,
-                                             static_cast<OutT*>(out), ldo, S, chunks, wait_limits());
+                                             static_cast<OutT*>(out), ldo, S, wc.base, wc.extra, wait_limits());
     return launched();
   }
   if (nbatch > 1) {  // the cp.async kernel takes one problem per launch
@@ -249,12 +261,11 @@ hq_status launch_fused(const uint16_t* x, int ldx, int P, int T, int H, int k, c
   int per_sm = 0;
   if (occupancy(d.fused[std::is_same<OutT, float>::value ? 1 : 0], kern, hq::kFuThreads, smem, P, &per_sm) != HQ_OK)
     return HQ_ERR_CUDA;
-  // one wave: as many row chunks per slice as the resident CTAs allow, at most one per 32-row block
-  const int nb_all = (T + hq::kFuTileRows - 1) / hq::kFuTileRows;
-  const int chunks = std::max(1, std::min(d.sms * per_sm / S, nb_all));
-  kern<<<(unsigned)(S * chunks), hq::kFuThreads, smem, st>>>(map, P, T, H, k, keep_idx, scale, inv_scale, zero,
-                                                              static_cast<OutT*>(out), ldo, S, chunks,
-                                                              wait_limits());
+  // one wave that fills every resident CTA slot (wave_chunks)
+  const WaveChunks wc = wave_chunks((long long)d.sms * per_sm, S, (T + hq::kFuTileRows - 1) / hq::kFuTileRows);
+  kern<<<(unsigned)(S * wc.base + wc.extra), hq::kFuThreads, smem, st>>>(map, P, T, H, k, keep_idx, scale, inv_scale,
+                                                                          zero, static_cast<OutT*>(out), ldo, S,
+                                                                          wc.base, wc.extra, wait_limits());
   return launched();
 }
 

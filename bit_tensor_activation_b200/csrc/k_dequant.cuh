@@ -541,15 +541,18 @@ template <typename OutT, bool kShard>
 __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_kernel(
     const __grid_constant__ DqWire wire, int side_tma, const uint16_t* __restrict__ side, int P, int T, int H,
     int k, const int32_t* __restrict__ keep_idx, const float* __restrict__ scale,
-    const uint8_t* __restrict__ zero, OutT* __restrict__ out, int ldo, int S, int chunks, WaitLimits lim) {
+    const uint8_t* __restrict__ zero, OutT* __restrict__ out, int ldo, int S, int chunks, int extra, WaitLimits lim) {
   extern __shared__ __align__(128) unsigned char s_raw[];
   DtSmem& sm = *reinterpret_cast<DtSmem*>(s_raw);
   float4* s_const = reinterpret_cast<float4*>(s_raw + ((sizeof(DtSmem) + 127) & ~size_t(127)));
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   // Slice-minor numbering (blockIdx = chunk*S + s): the S CTAs of one chunk are launched together.
-  // Chunk c of every slice takes the 32-row blocks c, c + chunks, c + 2*chunks, ..., so all CTAs
-  // sweep the rows from top to bottom together and counts differ by one block at most.
+  // Slices 0..extra-1 have chunks + 1 row chunks (their last one numbered after all the others),
+  // the rest `chunks`, so that the wave fills every resident slot.  Chunk c of a slice with n
+  // chunks takes the 32-row blocks c, c + n, c + 2n, ..., so all CTAs sweep the rows from top to
+  // bottom together and counts differ by one block at most within a slice.
   const int chunk = blockIdx.x / S, s = blockIdx.x - chunk * S;
+  const int n_chunks = chunks + (s < extra ? 1 : 0);
   // Problem blockIdx.y of a batch (gridDim.y is 1 for a single problem): ranks [y*P, (y+1)*P) of
   // the stacked wire, their parameters, and its own T output rows.
   const int rank0 = blockIdx.y * P;
@@ -557,9 +560,9 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
   zero += (size_t)rank0 * H;
   out += (size_t)blockIdx.y * T * ldo;
   const int nb_all = (T + kDtTileRows - 1) / kDtTileRows;
-  const int nblk = (nb_all - chunk + chunks - 1) / chunks;
+  const int nblk = (nb_all - chunk + n_chunks - 1) / n_chunks;
   const int t_last = T;
-  auto block_row = [&](int bi) { return (chunk + bi * chunks) * kDtTileRows; };
+  auto block_row = [&](int bi) { return (chunk + bi * n_chunks) * kDtTileRows; };
   const int n_groups = (P + kDtG - 1) / kDtG;  // ring slots per block
   const int n_slots_total = nblk * n_groups;     // slot i = (block i / n_groups, rank group i % n_groups)
 
@@ -670,8 +673,11 @@ __global__ void __launch_bounds__(kDtThreads, kDtMinBlocks) dequant_reduce_tma_k
   named_barrier_sync(kConsumers);
   int st_i = 0;
   unsigned phase = 0;
-  for (int bi = 0; bi < nblk && !*abort; ++bi) {
-    const int t0 = block_row(bi) + warp * kDtR;
+  // block bi starts at row t_blk = block_row(bi); the loop ends at the first block past T
+  const int t_step = n_chunks * kDtTileRows;
+  int bi = 0;
+  for (int t_blk = block_row(0); t_blk < T && !*abort; ++bi, t_blk += t_step) {
+    const int t0 = t_blk + warp * kDtR;
     float acc[kDtR][8];
 #pragma unroll
     for (int m = 0; m < kDtR; ++m)

@@ -98,18 +98,20 @@ __global__ void __launch_bounds__(kFuThreads, 2) compress_reduce_kernel(
     const __grid_constant__ CUtensorMap tmap_x, int P, int T, int H, int k,
     const int32_t* __restrict__ keep_idx, const float* __restrict__ scale,
     const float* __restrict__ inv_scale, const uint8_t* __restrict__ zero, OutT* __restrict__ out, int ldo, int S,
-    int chunks, WaitLimits lim) {
+    int chunks, int extra, WaitLimits lim) {
   extern __shared__ __align__(128) unsigned char s_raw[];
   FuSmem& sm = *reinterpret_cast<FuSmem*>(s_raw);
   float4* s_const = reinterpret_cast<float4*>(s_raw + ((sizeof(FuSmem) + 127) & ~size_t(127)));
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  // Slice-minor numbering (blockIdx = chunk*S + s), and chunk c of every slice takes the 32-row
-  // blocks c, c + chunks, c + 2*chunks, ...: as in dequant-reduce, the CTAs sweep the rows
-  // together and their block counts differ by one at most.
+  // Slice-minor numbering (blockIdx = chunk*S + s); slices 0..extra-1 have one row chunk more,
+  // and chunk c of a slice with n chunks takes the 32-row blocks c, c + n, c + 2n, ...: as in
+  // dequant-reduce, the wave fills every resident slot, the CTAs sweep the rows together and
+  // block counts differ by one at most within a slice.
   const int chunk = blockIdx.x / S, s = blockIdx.x - chunk * S;
+  const int n_chunks = chunks + (s < extra ? 1 : 0);
   const int nb_all = (T + kFuTileRows - 1) / kFuTileRows;
-  const int nblk = (nb_all - chunk + chunks - 1) / chunks;
-  auto block_row = [&](int bi) { return (chunk + bi * chunks) * kFuTileRows; };
+  const int nblk = (nb_all - chunk + n_chunks - 1) / n_chunks;
+  auto block_row = [&](int bi) { return (chunk + bi * n_chunks) * kFuTileRows; };
   const int n_tiles = nblk * P;  // tile i = (block i / P, rank i % P)
   const int hs = s * kFuSlice;
 
